@@ -1,0 +1,110 @@
+"""P6: the chunked (WY / UT-transform) form of the gated delta rule, in fp64 numpy, equals the
+sequential oracle.  This pins the algorithm the CUDA prefill kernels implement, separately from
+their precision (CPU only).
+
+Per value head and chunk of L tokens (G = inclusive cumulative sum of g inside the chunk):
+  A_ij = beta_i exp(G_i - G_j) k_i.k_j  (j < i),   T = (I + A)^-1
+  W = T diag(beta e^G) K,   U~ = T diag(beta) V
+  U = U~ - W S^T                                  (S = state entering the chunk, [d_v, d_k])
+  O = diag(e^G) Q S^T + P U,  P_ij = e^(G_i - G_j) q_i.k_j  (j <= i)
+  S <- e^(G_L) S + U^T diag(e^(G_L - G)) K
+Derivation: unroll S_i = e^(G_i) S + sum_{j<=i} e^(G_i - G_j) u_j k_j^T inside the chunk and
+substitute it into u_i = beta_i (v_i - alpha_i S_(i-1) k_i).
+
+The kernels also rely on two facts checked here:
+  * padding a partial chunk with k = q = v = 0, beta = 0, g = 0 leaves every result unchanged;
+  * the 128-token inverse can be assembled from the two 64-token diagonal inverses:
+    T = T_h - T_h N T_h, T_h = blockdiag((I + A_00)^-1, (I + A_11)^-1), N = lower-left block of A.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_layer_02_b200 import inputs
+
+
+def _masked_decay(G, strict):
+    diff = G[:, None] - G[None, :]
+    L = len(G)
+    mask = np.tril(np.ones((L, L), bool), -1 if strict else 0)
+    return np.where(mask, np.exp(np.where(mask, diff, 0.0)), 0.0)
+
+
+def chunked_head(q, k, v, beta, g, S, C, pad_to=None):
+    """One value head over one sequence.  q, k [T, dk] (normalised), v [T, dv], S [dv, dk]."""
+    T = q.shape[0]
+    out = np.zeros((T, v.shape[1]))
+    for c0 in range(0, T, C):
+        c1 = min(T, c0 + C)
+        Q, K, V, b, gg = q[c0:c1], k[c0:c1], v[c0:c1], beta[c0:c1], g[c0:c1]
+        if pad_to is not None and c1 - c0 < pad_to:
+            p = pad_to - (c1 - c0)
+            Q, K, V = (np.pad(a, ((0, p), (0, 0))) for a in (Q, K, V))
+            b, gg = np.pad(b, (0, p)), np.pad(gg, (0, p))
+        G = np.cumsum(gg)
+        A = b[:, None] * _masked_decay(G, True) * (K @ K.T)
+        Tm = np.linalg.inv(np.eye(len(G)) + A)
+        W = Tm @ ((b * np.exp(G))[:, None] * K)
+        Ut = Tm @ (b[:, None] * V)
+        U = Ut - W @ S.T
+        P = _masked_decay(G, False) * (Q @ K.T)
+        O = np.exp(G)[:, None] * (Q @ S.T) + P @ U
+        S = np.exp(G[-1]) * S + (U * np.exp(G[-1] - G)[:, None]).T @ K
+        out[c0:c1] = O[: c1 - c0]
+    return out, S
+
+
+def _normalised_inputs(seed, lengths, hk, hv, d, g_low):
+    r = np.random.default_rng(seed)
+    T = sum(lengths)
+    q, k = r.standard_normal((T, hk, d)), r.standard_normal((T, hk, d))
+    v = r.standard_normal((T, hv, d))
+    beta = r.uniform(0, 1, (T, hv)).astype(np.float32)
+    g = r.uniform(g_low, 0, (T, hv)).astype(np.float32)
+    S0 = (r.standard_normal((len(lengths), hv, d, d)) * 0.3).astype(np.float32)
+    return q, k, v, beta, g, S0
+
+
+@pytest.mark.parametrize("C,pad", [(4, None), (16, None), (32, None), (16, 16), (64, 64)])
+@pytest.mark.parametrize("g_low", [-0.05, -1.5])
+def test_p6_chunked_equals_sequential(C, pad, g_low):
+    lengths = [1, 37, 64, 50]
+    hk, hv, d = 1, 2, 16
+    q, k, v, beta, g, S0 = _normalised_inputs(6, lengths, hk, hv, d, g_low)
+    T = sum(lengths)
+    x = np.concatenate([q.reshape(T, -1), k.reshape(T, -1), v.reshape(T, -1)], 1)
+    dims = oracle.Dims(hk, hv, d, 4, 1.0, 0.0, 1e-6)
+    ref_o, ref_S, _ = oracle.prefill(dims, torch.from_numpy(x), torch.from_numpy(beta),
+                                     torch.from_numpy(g), inputs.cu_seqlens_of(lengths),
+                                     S0=torch.from_numpy(S0), nthreads=2)
+    qn = q / np.linalg.norm(q, axis=-1, keepdims=True)
+    kn = k / np.linalg.norm(k, axis=-1, keepdims=True)
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    for n in range(len(lengths)):
+        s = slice(cu[n], cu[n + 1])
+        for h in range(hv):
+            o, S = chunked_head(qn[s, h // (hv // hk)], kn[s, h // (hv // hk)], v[s, h],
+                                beta[s, h].astype(np.float64), g[s, h].astype(np.float64),
+                                S0[n, h].astype(np.float64), C, pad)
+            np.testing.assert_allclose(o, ref_o[s, h], rtol=1e-9, atol=1e-10)
+            np.testing.assert_allclose(S, ref_S[n, h], rtol=1e-9, atol=1e-10)
+
+
+@pytest.mark.parametrize("g_low", [-0.05, -1.0])
+def test_block_inverse_assembly(g_low):
+    r = np.random.default_rng(61)
+    C, d = 128, 128
+    K = r.standard_normal((C, d)) + 0.5           # correlated keys (a mean component)
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    b = r.uniform(0, 1, C)
+    G = np.cumsum(r.uniform(g_low, 0, C))
+    A = b[:, None] * _masked_decay(G, True) * (K @ K.T)
+    h = C // 2
+    Th = np.zeros((C, C))
+    Th[:h, :h] = np.linalg.inv(np.eye(h) + A[:h, :h])
+    Th[h:, h:] = np.linalg.inv(np.eye(h) + A[h:, h:])
+    N = np.zeros((C, C))
+    N[h:, :h] = A[h:, :h]
+    T = Th - Th @ N @ Th
+    np.testing.assert_allclose(T, np.linalg.inv(np.eye(C) + A), rtol=1e-10, atol=1e-12)
