@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of the Gated DeltaNet layer on B200: one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one gdn_chunk_prefill of the T=4096 Qwen3-Next layer workload (16 key heads, 32 value
+heads, d = 128, bf16 activations, fp32 state, conv + SiLU + L2 norms + gated delta rule + gated
+RMSNorm, final recurrent and conv states returned), inputs resident in HBM, L2 flushed between
+timed steps.  `value` is whole-job tokens/s.  Alongside: the per-kernel roofline of the
+dominant kernel, the whole-step fractions of tensor and HBM peak, an end-to-end figure through
+the C ABI with host buffers, the decode workload (256 sequences x 64 steps, state GB/s) and the
+fp64 CPU oracle timed on this host.  N > 1 (torchrun, one process per GPU) runs independent
+replicas (the layer needs no collective): weak scaling, max time over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gated_deltanet_layer_02_b200 import inputs  # noqa: E402
+
+METRIC = "prefill tokens/s per GDN layer (% TC peak); decode state GB/s (% HBM peak)"
+CHUNK = 128
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------- work per token
+def flops_per_token_by_kernel(w, C=CHUNK):
+    """Useful (triangle-masked) chunk-form FLOPs per token, split by the kernel that does them.
+    Their sum is F(C) = 2 [Hv (3 d^2 + 1.5 C d + C^2/6) + Hk C d]."""
+    Hv, Hk, d = w.num_v_heads, w.num_k_heads, w.head_dim
+    return {
+        "gdn_prep": 2.0 * (Hv * (C * d + C * C / 6.0) + Hk * C * d / 2.0),   # K K^T, solve, W, U~
+        "gdn_chain": 2.0 * (Hv * 2.0 * d * d),                               # W S^T, K^T U
+        "gdn_out": 2.0 * (Hv * (d * d + C * d / 2.0) + Hk * C * d / 2.0),    # Q K^T, Q S^T, P U
+    }
+
+
+def bytes_per_token_by_kernel(w):
+    """Algorithmic HBM bytes per token (the layer's own inputs and outputs), by the kernel that
+    moves them: x, beta, g in prep; z in, output out in gdn_out."""
+    esz = 2 if w.dtype == torch.bfloat16 else 4
+    Hv, d = w.num_v_heads, w.head_dim
+    return {"gdn_prep": w.channels * esz + 2 * Hv * 4, "gdn_chain": 0,
+            "gdn_out": 2 * Hv * d * esz}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            m = json.load(f)
+        return {k: float(m[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_deltanet_layer_02_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel sources are unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    if t.get("source_hash") != source_hash():
+        return None
+    k = t.get("kernels", {}).get(kernel)
+    return None if k is None else float(k["dram_bytes_per_launch_full_size"])
+
+
+# ------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML for SM clock and throttle reasons while the timed region runs."""
+
+    HW_SLOWDOWN = 0x8
+    SW_THERMAL = 0x20
+    HW_THERMAL = 0x40
+    SW_POWER_CAP = 0x4
+
+    def __init__(self, index):
+        self.index, self.samples, self.reasons = index, [], 0
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._nv:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        names = []
+        if self.reasons & self.HW_SLOWDOWN:
+            names.append("hw_slowdown")
+        if self.reasons & self.HW_THERMAL:
+            names.append("hw_thermal_slowdown")
+        if self.reasons & self.SW_THERMAL:
+            names.append("sw_thermal_slowdown")
+        if self.reasons & self.SW_POWER_CAP:
+            names.append("sw_power_cap")
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples),
+                "source": "nvml" if self._nv else "unavailable"}
+
+
+# --------------------------------------------------------------------------- the arms
+def cpu_oracle_rate(w, seed, budget_s=10.0, cap_s=30.0):
+    """The fp64 oracle as it stands, on this host's cores, over whole copies of the workload
+    until at least budget_s of CPU work has run (at least one copy)."""
+    import oracle
+    inp = inputs.prefill_inputs(w, seed)
+    dims = oracle.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    threads = oracle.default_threads()
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.prefill(dims, inp["x"], inp["beta"], inp["g"], inp["cu_seqlens"],
+                       conv_w=inp["conv_w"], z=inp["z"], norm_w=inp["norm_w"], S0=inp["S0"],
+                       nthreads=threads)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or el * (done + 1) / done > cap_s:
+            break
+    return {"value": done * w.tokens / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} full copies of the {w.tokens}-token workload ({el:.1f} s)"}
+
+
+def run_reference(args, w, seed, rank):
+    """The fp64 CPU oracle as the reference arm, on this host's cores."""
+    if rank != 0:
+        return None
+    import oracle
+    # one step = a bounded sample of the workload: the first `sample` tokens of the sequence
+    sample = 512
+    inp = inputs.prefill_inputs(w, seed, lengths=(sample,))
+    dims = oracle.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    threads = oracle.default_threads()
+
+    def step():
+        oracle.prefill(dims, inp["x"], inp["beta"], inp["g"], inp["cu_seqlens"],
+                       conv_w=inp["conv_w"], z=inp["z"], norm_w=inp["norm_w"], nthreads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = args.steps * sample / el
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": 1, "seq_len": w.tokens,
+                   "sample_tokens_per_step": sample, "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{args.steps} steps of the first {sample} tokens"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def bench_prefill(args, w, seed, dev, gdn):
+    inp = inputs.prefill_inputs(w, seed)
+    host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    T, N = w.tokens, len(w.lengths)
+    out = torch.empty((T, w.num_v_heads, w.head_dim), dtype=w.dtype, device=dev)
+    SN = torch.empty((N, w.num_v_heads, w.head_dim, w.head_dim), dtype=torch.float32, device=dev)
+    convN = torch.empty((N, w.conv_kernel - 1, w.channels), dtype=w.dtype, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(N, T, w.dtype, dims), dtype=torch.uint8,
+                     device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(x=d["x"], beta=d["beta"], g=d["g"], z=d["z"], cu=d["cu_seqlens"], o=out):
+        gdn.chunk_prefill(x, beta, g, cu, conv_w=d["conv_w"], z=z, norm_w=d["norm_w"], S0=d["S0"],
+                          SN=SN, convN=convN, out=o, workspace=ws, dev_status=status, dims=dims)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    tr = gdn.Trace()
+    if dist_on():
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk, tr:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    if dist_on():
+        torch.distributed.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    recs = tr.records()
+    tr.close()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during the timed steps")
+    # end to end through the C ABI with host buffers: H2D inputs, the layer, D2H output
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    names = ("x", "beta", "g", "z", "cu_seqlens")
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = out_h.numel() * out_h.element_size()
+    e2e_ms = []
+    dbuf = {k: torch.empty_like(d[k]) for k in names}
+    for i in range(args.warmup + max(3, args.steps // 10)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        a.record()
+        for k in names:
+            dbuf[k].copy_(host[k], non_blocking=True)
+        step(dbuf["x"], dbuf["beta"], dbuf["g"], dbuf["z"], dbuf["cu_seqlens"])
+        out_h.copy_(out, non_blocking=True)
+        b.record()
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    return step_ms, recs, clk.summary(), (statistics.mean(e2e_ms), h2d, d2h)
+
+
+def bench_decode(w, seed, dev, gdn, steps):
+    st = inputs.decode_state(w, seed)
+    S, cs = st["S"].to(dev), st["conv_state"].to(dev)
+    cw, nw = st["conv_w"].to(dev), st["norm_w"].to(dev)
+    dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    steps_in = [{k: v.to(dev) for k, v in inputs.decode_step_inputs(w, seed, s).items()}
+                for s in range(steps)]
+    out = torch.empty((w.batch, w.num_v_heads, w.head_dim), dtype=w.dtype, device=dev)
+    for s in steps_in[:3]:
+        gdn.decode_step(s["x"], s["beta"], s["g"], cs, S, cw, z=s["z"], norm_w=nw, out=out,
+                        dims=dims)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i, s in enumerate(steps_in):
+            ev[i][0].record()
+            gdn.decode_step(s["x"], s["beta"], s["g"], cs, S, cw, z=s["z"], norm_w=nw, out=out,
+                            dims=dims)
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    state_bytes = 2 * S.numel() * 4
+    return statistics.median(ms), state_bytes, clk.summary()
+
+
+def dist_on():
+    return torch.distributed.is_available() and torch.distributed.is_initialized()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=64)
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = inputs.CONFIGS[1]
+    seed = inputs.config_seed(1)
+    if args.impl == "reference":
+        res = run_reference(args, w, seed, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from gated_deltanet_layer_02_b200 import build as gdn_build
+    gdn_build.build()
+    import gated_deltanet_layer_02_b200 as gdn
+
+    step_ms, recs, clocks, (e2e_ms, h2d, d2h) = bench_prefill(args, w, seed, dev, gdn)
+    ms = statistics.mean(step_ms)
+    if dist_on():
+        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+    n = world
+    T = w.tokens
+    value = n * T / (ms * 1e-3)
+    peaks, peak_src = load_peaks()
+
+    # per-kernel breakdown of the timed steps
+    kern = {}
+    for name, t in recs:
+        k = kern.setdefault(name, {"launches": 0, "total_ms": 0.0})
+        k["launches"] += 1
+        k["total_ms"] += t
+    fl = flops_per_token_by_kernel(w)
+    by = bytes_per_token_by_kernel(w)
+    tot = sum(k["total_ms"] for k in kern.values()) or 1.0
+    for name, k in kern.items():
+        k["avg_ms"] = k["total_ms"] / k["launches"]
+        k["share"] = k["total_ms"] / tot
+        if name in fl:
+            k["tflops"] = fl[name] * T / (k["avg_ms"] * 1e-3) / 1e12
+            k["tc_frac"] = k["tflops"] / peaks["bf16_tflops"]
+            k["gbs"] = by[name] * T / (k["avg_ms"] * 1e-3) / 1e9
+            k["hbm_frac"] = k["gbs"] / peaks["hbm_gbs"]
+    dom = max((n_ for n_ in kern if n_ in fl), key=lambda n_: kern[n_]["total_ms"])
+    dk = kern[dom]
+    if dk["hbm_frac"] > dk["tc_frac"]:
+        roof = {"bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": dk["hbm_frac"]}
+    else:
+        roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": dk["tc_frac"]}
+    roof.update({"kernel": dom, "traffic": ncu_traffic(dom),
+                 "peak_source": f"{peak_src} ({'burst bf16' if roof['bound'] == 'tensor' else 'copy'})"})
+    F = sum(fl.values())
+    B = sum(by.values())
+    step_roof = {"tc_frac": F * value / n / (peaks["bf16_tflops"] * 1e12),
+                 "hbm_frac": B * value / n / (peaks["hbm_gbs"] * 1e9),
+                 "flops_per_token": F, "bytes_per_token": B, "chunk": CHUNK,
+                 "flops_per_token_chunk64": sum(flops_per_token_by_kernel(w, 64).values())}
+
+    dec_ms, dec_bytes, dec_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev, gdn,
+                                              args.decode_steps)
+    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+    decode = {"workload": inputs.CONFIGS[3].name, "value": dec_gbs, "unit": "GB/s",
+              "ms_per_step": dec_ms, "steps": args.decode_steps,
+              "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
+                           "traffic": ncu_traffic("decode_step"),
+                           "peak_source": f"{peak_src} (copy)"},
+              "clocks": dec_clk}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_rate(w, seed)
+
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; Qwen3-Next GDN layer shapes)",
+        "config": {"workload": w.name, "global_batch": n, "seq_len": T,
+                   "parallelism": "replicas" if n == 1 else f"replicas x{n}",
+                   "l2": "flushed between timed steps (256 MiB write, untimed)",
+                   "chunk": CHUNK, "heads": [w.num_k_heads, w.num_v_heads], "head_dim": 128},
+        "roofline": roof, "step_roofline": step_roof, "kernels": kern,
+        "e2e": {"value": n * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(recs), "clocks": clocks, "decode": decode, "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist_on():
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,1 +1,273 @@
-"""B200-native Gated DeltaNet layer (placeholder; binding added with the C-ABI)."""
+"""B200-native Gated DeltaNet layer: thin Python binding over libgdn.so (see include/gdn.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of libgdn.so.
+PyTorch provides device memory and the current stream.  There is no CPU fallback: if the
+library is missing or a tensor is not on a CUDA device, the call raises.
+
+    import gated_deltanet_layer_02_b200 as gdn
+    out, SN, convN = gdn.chunk_prefill(x, beta, g, cu_seqlens, conv_w=w, z=z, norm_w=nw)
+    out = gdn.decode_step(x_t, beta_t, g_t, conv_state, S, conv_w=w, z=z_t, norm_w=nw)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
+    GDN_ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+GDN_F32, GDN_BF16 = 0, 1
+
+#: every symbol include/gdn.h declares
+EXPORTS = (
+    "gdn_abi_version", "gdn_conv_channels", "gdn_status_string", "gdn_conv1d_update",
+    "gdn_gated_rmsnorm", "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill",
+    "gdn_decode_step", "gdn_trace_create", "gdn_trace_destroy", "gdn_trace_attach",
+    "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
+)
+
+
+class GdnError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {code} ({status_string(code)})")
+        self.code = code
+
+
+class Dims(ctypes.Structure):
+    """gdn_dims: layer shape.  Defaults are the Qwen3-Next values."""
+    _fields_ = [("num_k_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("conv_kernel", ctypes.c_int32),
+                ("q_scale", ctypes.c_float), ("l2_eps", ctypes.c_float),
+                ("norm_eps", ctypes.c_float)]
+
+    def __init__(self, num_k_heads=16, num_v_heads=32, head_dim=128, conv_kernel=4, q_scale=1.0,
+                 l2_eps=1e-6, norm_eps=1e-6):
+        super().__init__(num_k_heads, num_v_heads, head_dim, conv_kernel, q_scale, l2_eps, norm_eps)
+
+    @property
+    def channels(self) -> int:
+        return (2 * self.num_k_heads + self.num_v_heads) * self.head_dim
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """The loaded libgdn.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m gated_deltanet_layer_02_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i32, dp = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(Dims)
+            L.gdn_abi_version.restype = ctypes.c_int
+            L.gdn_conv_channels.argtypes = [dp]
+            L.gdn_conv_channels.restype = ctypes.c_int64
+            L.gdn_status_string.argtypes = [ctypes.c_int]
+            L.gdn_status_string.restype = ctypes.c_char_p
+            L.gdn_conv1d_update.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, i32, i32, vp, vp, vp]
+            L.gdn_gated_rmsnorm.argtypes = [ctypes.c_int, vp, vp, vp, ctypes.c_float, i32, i32, vp, vp]
+            L.gdn_chunk_prefill_workspace_size.argtypes = [dp, ctypes.c_int, i32, i32]
+            L.gdn_chunk_prefill_workspace_size.restype = ctypes.c_size_t
+            L.gdn_chunk_prefill.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, i32, i32,
+                                            vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
+            L.gdn_decode_step.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                          vp, vp]
+            L.gdn_trace_create.argtypes = [ctypes.POINTER(vp)]
+            L.gdn_trace_destroy.argtypes = [vp]
+            L.gdn_trace_attach.argtypes = [vp]
+            L.gdn_trace_reset.argtypes = [vp]
+            L.gdn_trace_count.argtypes = [vp]
+            L.gdn_trace_get.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_char_p),
+                                        ctypes.POINTER(ctypes.c_float)]
+            L.gdn_debug_wait_probe.argtypes = [vp, ctypes.c_uint32, vp]
+            for name in EXPORTS:  # every declared symbol must resolve
+                getattr(L, name)
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().gdn_status_string(int(code)).decode()
+
+
+def _check(fn, code):
+    if code != GDN_OK:
+        raise GdnError(fn, code)
+
+
+def _ptr(t, name, dtype=None, allow_none=True):
+    if t is None:
+        if not allow_none:
+            raise ValueError(f"{name} is required")
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device (no CPU fallback)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _act_dtype(t):
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    if t.dtype == torch.float32:
+        return GDN_F32
+    raise TypeError(f"activations must be bfloat16 or float32, got {t.dtype}")
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def conv_channels(dims: Dims) -> int:
+    return int(lib().gdn_conv_channels(ctypes.byref(dims)))
+
+
+def conv1d_update(x, conv_w, cu_seqlens, conv_state_in=None, conv_state_out=None, y=None,
+                  dims: Dims | None = None):
+    """silu(causal depthwise conv) of packed sequences; returns y [T, Cc]."""
+    dims = dims or Dims()
+    dt = _act_dtype(x)
+    y = torch.empty_like(x) if y is None else y
+    N = cu_seqlens.numel() - 1
+    _check("gdn_conv1d_update", lib().gdn_conv1d_update(
+        ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(y, "y", x.dtype),
+        _ptr(conv_w, "conv_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N,
+        x.shape[0], _ptr(conv_state_in, "conv_state_in", x.dtype),
+        _ptr(conv_state_out, "conv_state_out", x.dtype), _stream()))
+    return y
+
+
+def gated_rmsnorm(o, z, w=None, eps: float = 1e-6, y=None):
+    """y = o / sqrt(mean(o^2) + eps) * w * silu(z) over the last dim."""
+    dt = _act_dtype(o)
+    y = torch.empty_like(o) if y is None else y
+    dim = o.shape[-1]
+    rows = o.numel() // dim if dim else 0
+    _check("gdn_gated_rmsnorm", lib().gdn_gated_rmsnorm(
+        dt, _ptr(o, "o", o.dtype), _ptr(z, "z", o.dtype), _ptr(w, "w", o.dtype), float(eps),
+        rows, dim, _ptr(y, "y", o.dtype), _stream()))
+    return y
+
+
+def prefill_workspace_size(num_seqs: int, num_tokens: int, dtype=torch.bfloat16,
+                           dims: Dims | None = None) -> int:
+    dims = dims or Dims()
+    return int(lib().gdn_chunk_prefill_workspace_size(
+        ctypes.byref(dims), GDN_BF16 if dtype == torch.bfloat16 else GDN_F32, num_seqs,
+        num_tokens))
+
+
+def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None, SN=None,
+                  conv0=None, convN=None, out=None, workspace=None, dev_status=None,
+                  want_state=True, dims: Dims | None = None):
+    """The whole layer over packed sequences.  Returns (out, SN, convN).
+
+    x [T, Cc], beta/g [T, Hv] fp32, z [T, Hv, d] or None, cu_seqlens [N+1] int32 (device),
+    S0 [N, Hv, d, d] fp32 or None, conv0 [N, K-1, Cc] or None.
+    """
+    dims = dims or Dims()
+    dt = _act_dtype(x)
+    T = x.shape[0]
+    N = cu_seqlens.numel() - 1
+    Hv, d, K = dims.num_v_heads, dims.head_dim, dims.conv_kernel
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, Hv, d), dtype=x.dtype, device=dev)
+    if want_state and SN is None:
+        SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
+    if want_state and convN is None:
+        convN = torch.empty((N, K - 1, dims.channels), dtype=x.dtype, device=dev)
+    need = prefill_workspace_size(N, T, x.dtype, dims)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check("gdn_chunk_prefill", lib().gdn_chunk_prefill(
+        ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
+        _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
+        _ptr(norm_w, "norm_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N, T,
+        _ptr(S0, "S0", torch.float32), _ptr(SN, "SN", torch.float32),
+        _ptr(conv0, "conv0", x.dtype), _ptr(convN, "convN", x.dtype), _ptr(out, "out", x.dtype),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
+        _ptr(dev_status, "dev_status", torch.int32), _stream()))
+    return out, SN, convN
+
+
+def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx=None,
+                out=None, dims: Dims | None = None):
+    """One token per sequence; conv_state and S are updated in place.  Returns out [B, Hv, d]."""
+    dims = dims or Dims()
+    dt = _act_dtype(x)
+    B = x.shape[0]
+    if out is None:
+        out = torch.empty((B, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
+    _check("gdn_decode_step", lib().gdn_decode_step(
+        ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype, False),
+        _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
+        _ptr(norm_w, "norm_w", x.dtype), _ptr(conv_state, "conv_state", x.dtype),
+        _ptr(S, "S", torch.float32), _ptr(slot_idx, "slot_idx", torch.int32), B,
+        _ptr(out, "out", x.dtype), _stream()))
+    return out
+
+
+def debug_wait_probe(dev_status, limit_us: int):
+    """Launch a kernel whose wait nothing satisfies; it gives up after limit_us."""
+    _check("gdn_debug_wait_probe", lib().gdn_debug_wait_probe(
+        _ptr(dev_status, "dev_status", torch.int32, False), int(limit_us), _stream()))
+
+
+class Trace:
+    """Per-launch device times of the library's kernels (CUDA events on the launch stream)."""
+
+    def __init__(self):
+        h = ctypes.c_void_p()
+        _check("gdn_trace_create", lib().gdn_trace_create(ctypes.byref(h)))
+        self._h = h
+
+    def __enter__(self):
+        lib().gdn_trace_attach(self._h)
+        return self
+
+    def __exit__(self, *exc):
+        lib().gdn_trace_attach(None)
+
+    def reset(self):
+        lib().gdn_trace_reset(self._h)
+
+    def records(self):
+        """[(kernel name, ms)] in launch order (synchronises on each end event)."""
+        out = []
+        for i in range(lib().gdn_trace_count(self._h)):
+            name, ms = ctypes.c_char_p(), ctypes.c_float()
+            _check("gdn_trace_get", lib().gdn_trace_get(self._h, i, ctypes.byref(name),
+                                                        ctypes.byref(ms)))
+            out.append((name.value.decode(), ms.value))
+        return out
+
+    def close(self):
+        if self._h:
+            lib().gdn_trace_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+__all__ = ["Dims", "GdnError", "lib", "conv1d_update", "gated_rmsnorm", "chunk_prefill",
+           "decode_step", "prefill_workspace_size", "conv_channels", "status_string", "Trace",
+           "debug_wait_probe", "EXPORTS", "LIB_PATH"]

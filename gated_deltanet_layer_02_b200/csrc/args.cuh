@@ -1,0 +1,72 @@
+// args.cuh -- argument blocks passed by value from the C-ABI layer to the kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct DecodeArgs {
+  const void* x;
+  const void* conv_w;
+  const float* beta;
+  const float* g;
+  const void* z;
+  const void* norm_w;
+  void* conv_state;
+  float* S;
+  const int32_t* slot_idx;
+  void* out;
+  int B, Hk, Hv;
+  float q_scale, l2_eps, norm_eps;
+};
+
+struct RecArgs {
+  const float* x;
+  const float* conv_w;
+  const float* beta;
+  const float* g;
+  const float* z;
+  const float* norm_w;
+  const int32_t* cu;
+  const float* S0;
+  float* SN;
+  const float* conv0;
+  float* out;
+  int N, Hk, Hv;
+  float q_scale, l2_eps, norm_eps;
+};
+
+struct ChunkInfo {
+  int n, t0, L, pad;
+};
+
+struct Workspace {
+  ChunkInfo* chunks;     // [NCmax]
+  int32_t* seq_first;    // [N+1] first chunk of each sequence (prefix sum), [N] = total
+  __nv_bfloat16* Qw;     // [NCmax][Hk][128][128]
+  __nv_bfloat16* Kw;     // [NCmax][Hk][128][128]
+  __nv_bfloat16* Ww;     // [NCmax][Hv][128][128]
+  __nv_bfloat16* Uw;     // [NCmax][Hv][128][128]  U~ from prep, overwritten with U by chain
+  __nv_bfloat16* Sw;     // [NCmax][Hv][128 (d_k)][128 (d_v)]  S^T entering each chunk
+  float* Gw;             // [NCmax][Hv][128]  cumulative log decay inside the chunk
+};
+
+struct PrefillArgs {
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* conv_w;
+  const float* beta;
+  const float* g;
+  const __nv_bfloat16* z;
+  const __nv_bfloat16* norm_w;
+  const int32_t* cu;
+  const float* S0;
+  float* SN;
+  const __nv_bfloat16* conv0;
+  __nv_bfloat16* out;
+  int32_t* status;
+  int N, T, Hk, Hv, nsplit;
+  float q_scale, l2_eps, norm_eps;
+  Workspace ws;
+};
+
+}  // namespace gdn

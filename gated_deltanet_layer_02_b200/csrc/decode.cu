@@ -1,0 +1,174 @@
+// decode.cu -- one decode token per sequence: conv-state shift + conv + SiLU, L2 norms of q and
+// k, one read-modify-write pass over the fp32 recurrent state, z-gated RMSNorm.
+//
+// Source: the recurrence of the hyper.ai Gated DeltaNet paragraph as read in gdn.h (beta gates
+// the update, kv_mem = alpha S k is the read-out of the stored knowledge), with the fp32 state
+// of the "Qwen3-Next" SGLang cookbook, section 3.2 (--mamba-ssm-dtype default).
+//
+// Per state row r (value index) of value head h, with alpha = exp(g), kq = k.q:
+//   kv  = alpha * (S_r . k)                 (kv_mem)
+//   u   = beta * (v_r - kv)
+//   o_r = alpha * (S_r . q) + u * kq        (= S'_r . q)
+//   S'_r = alpha * S_r + u * k
+// so each state element is read once and written once.  One CTA per (sequence, key head)
+// handles that key head's R = Hv/Hk value heads; each warp streams whole rows (a lane owns 4
+// consecutive columns, 512 contiguous bytes per warp load) with kRowBatch rows in flight, and
+// reduces the two dot products with warp shuffles.
+#include "args.cuh"
+#include "common.cuh"
+
+namespace gdn {
+
+constexpr int kDecodeThreads = 256;
+constexpr int kRowBatch = 8;
+constexpr int kMaxR = 8;
+
+
+template <typename T>
+__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
+  constexpr int d = kHeadDim;
+  const int b = blockIdx.x / a.Hk;
+  const int hk = blockIdx.x % a.Hk;
+  const int R = a.Hv / a.Hk;
+  const int Cc = (2 * a.Hk + a.Hv) * d;
+  const int slot = a.slot_idx ? __ldg(a.slot_idx + b) : b;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  __shared__ float y_s[(2 + kMaxR) * d];  // q | k | v_0..v_{R-1} after conv
+  __shared__ float o_s[kMaxR * d];
+  __shared__ float red_s[4];
+
+  const T* x = static_cast<const T*>(a.x) + (size_t)b * Cc;
+  const T* w = static_cast<const T*>(a.conv_w);
+  T* cs = static_cast<T*>(a.conv_state) + (size_t)slot * 3 * Cc;
+
+  // ---- conv + SiLU with in-place history shift: 2 channels per item
+  const int items = (2 + R) * d / 2;
+  for (int it = tid; it < items; it += kDecodeThreads) {
+    const int gch = it * 2;              // position inside y_s
+    const int grp = gch / d, off = gch % d;
+    int c;
+    if (grp == 0) c = hk * d + off;
+    else if (grp == 1) c = a.Hk * d + hk * d + off;
+    else c = 2 * a.Hk * d + (hk * R + grp - 2) * d + off;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float s0 = to_f(cs[c + e]), s1 = to_f(cs[Cc + c + e]), s2 = to_f(cs[2 * Cc + c + e]);
+      const T xt = x[c + e];
+      const T* wr = w + (size_t)(c + e) * 4;
+      const float acc = to_f(wr[0]) * s0 + to_f(wr[1]) * s1 + to_f(wr[2]) * s2 + to_f(wr[3]) * to_f(xt);
+      y_s[gch + e] = silu_f(acc);
+      cs[c + e] = from_f<T>(s1);
+      cs[Cc + c + e] = from_f<T>(s2);
+      cs[2 * Cc + c + e] = xt;
+    }
+  }
+  __syncthreads();
+  // ---- |q|^2, |k|^2, q.k
+  if (warp < 3) {
+    float acc = 0.f;
+    for (int i = lane; i < d; i += 32) {
+      const float qv = y_s[i], kv = y_s[d + i];
+      acc += warp == 0 ? qv * qv : (warp == 1 ? kv * kv : qv * kv);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) red_s[warp] = acc;
+  }
+  __syncthreads();
+  const float rq = a.q_scale * rsqrtf(red_s[0] + a.l2_eps);
+  const float rk = rsqrtf(red_s[1] + a.l2_eps);
+  const float kq = red_s[2] * rq * rk;
+  float kreg[4], qreg[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    kreg[j] = y_s[d + 4 * lane + j] * rk;
+    qreg[j] = y_s[4 * lane + j] * rq;
+  }
+
+  // ---- state pass: R*d rows split over the warps
+  const int rows_total = R * d;
+  const int rows_per_warp = rows_total / (kDecodeThreads / 32);
+  for (int r0 = warp * rows_per_warp; r0 < (warp + 1) * rows_per_warp; r0 += kRowBatch) {
+    float4 sv[kRowBatch];
+    float dk[kRowBatch], dq[kRowBatch];
+#pragma unroll
+    for (int i = 0; i < kRowBatch; ++i) {
+      const int gr = r0 + i, hr = gr / d, v = gr % d;
+      const int h = hk * R + hr;
+      const float4* p = reinterpret_cast<const float4*>(a.S + (((size_t)slot * a.Hv + h) * d + v) * d) + lane;
+      sv[i] = __ldcs(p);
+    }
+#pragma unroll
+    for (int i = 0; i < kRowBatch; ++i) {
+      dk[i] = sv[i].x * kreg[0] + sv[i].y * kreg[1] + sv[i].z * kreg[2] + sv[i].w * kreg[3];
+      dq[i] = sv[i].x * qreg[0] + sv[i].y * qreg[1] + sv[i].z * qreg[2] + sv[i].w * qreg[3];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int i = 0; i < kRowBatch; ++i) {
+        dk[i] += __shfl_xor_sync(0xffffffffu, dk[i], o);
+        dq[i] += __shfl_xor_sync(0xffffffffu, dq[i], o);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kRowBatch; ++i) {
+      const int gr = r0 + i, hr = gr / d, v = gr % d;
+      const int h = hk * R + hr;
+      const float alpha = expf(__ldg(a.g + (size_t)b * a.Hv + h));
+      const float beta = __ldg(a.beta + (size_t)b * a.Hv + h);
+      const float vv = y_s[(2 + hr) * d + v];
+      const float u = beta * (vv - alpha * dk[i]);
+      if (lane == 0) o_s[hr * d + v] = alpha * dq[i] + u * kq;
+      float4 nv;
+      nv.x = alpha * sv[i].x + u * kreg[0];
+      nv.y = alpha * sv[i].y + u * kreg[1];
+      nv.z = alpha * sv[i].z + u * kreg[2];
+      nv.w = alpha * sv[i].w + u * kreg[3];
+      float4* p = reinterpret_cast<float4*>(a.S + (((size_t)slot * a.Hv + h) * d + v) * d) + lane;
+      __stcs(p, nv);
+    }
+  }
+  __syncthreads();
+  // ---- gated RMSNorm (or plain output), one warp per value head
+  T* out = static_cast<T*>(a.out);
+  for (int hr = warp; hr < R; hr += kDecodeThreads / 32) {
+    const int h = hk * R + hr;
+    float ov[4], ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      ov[j] = o_s[hr * d + 4 * lane + j];
+      ss += ov[j] * ov[j];
+    }
+    if (a.z) {
+      ss = warp_sum(ss);
+      const float inv = rsqrtf(ss / d + a.norm_eps);
+      const T* zr = static_cast<const T*>(a.z) + ((size_t)b * a.Hv + h) * d;
+      const T* nw = static_cast<const T*>(a.norm_w);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = 4 * lane + j;
+        ov[j] = ov[j] * inv * (nw ? to_f(nw[c]) : 1.f) * silu_f(to_f(zr[c]));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) out[((size_t)b * a.Hv + h) * d + 4 * lane + j] = from_f<T>(ov[j]);
+  }
+}
+
+}  // namespace gdn
+
+namespace gdn_host {
+
+cudaError_t launch_decode(bool bf16, const gdn::DecodeArgs& a, cudaStream_t s) {
+  if (a.B == 0) return cudaSuccess;
+  trace_begin("decode_step", s);
+  if (bf16)
+    gdn::decode_kernel<__nv_bfloat16><<<a.B * a.Hk, gdn::kDecodeThreads, 0, s>>>(a);
+  else
+    gdn::decode_kernel<float><<<a.B * a.Hk, gdn::kDecodeThreads, 0, s>>>(a);
+  trace_end(s);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn_host

@@ -1,0 +1,176 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, a B200 (sm_100a) implementation of the Gated DeltaNet
+ * linear-attention layer of the Qwen3-Next hybrid stack.
+ *
+ * Sources for what is computed:
+ *   - layer constants: "Qwen3-Coder-Next" model card (llm-atlas), raw config.json fields
+ *     (linear_conv_kernel_dim 4, linear_num_key_heads 16, linear_num_value_heads 32,
+ *     linear_key_head_dim = linear_value_head_dim = 128, rms_norm_eps 1e-6, hidden_act silu);
+ *   - the token mixer: hyper.ai story on Qwen3-Next in Transformers, Gated DeltaNet paragraph
+ *     (QKV plus a Z projection, causal convolution for local context, beta gating the update
+ *     strength, kv_mem as the prior knowledge read from the recurrent state, linear cost through
+ *     a recurrent state update, zero-centred RMSNorm);
+ *   - state size independent of the sequence: Qwen3.5 teardown (rkmt.cn), section 3.2;
+ *   - fp32 recurrent state by default, chunked FLA kernels with chunk 64 as prior art:
+ *     "Qwen3-Next" SGLang cookbook, section 3.2 Configuration Tips.
+ * Per token t of a sequence (value head h reads key head h / (Hv/Hk)):
+ *   y     = silu(causal depthwise conv_K(x))          (x = [q | k | v] projections)
+ *   q     = q~ / sqrt(|q~|^2 + l2_eps) * q_scale,   k = k~ / sqrt(|k~|^2 + l2_eps)
+ *   S_t   = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   alpha_t = exp(g_t)
+ *   o_t   = S_t q_t
+ *   out_t = o_t / sqrt(mean(o_t^2) + norm_eps) * w * silu(z_t)       (when z is given)
+ *
+ * General rules for every call:
+ *   - Pointers are DEVICE pointers owned by the caller unless a comment says "host".  The
+ *     library allocates no device memory and keeps no global state between calls.
+ *   - Tensors are dense, row-major, contiguous and 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Return value: GDN_OK, or a negative gdn_status.  On argument errors nothing is launched
+ *     and no memory is touched.  GDN_ERR_CUDA reports a failed launch (cudaGetLastError).
+ *   - Supported shapes: head_dim 128, conv_kernel 4, num_v_heads a multiple of num_k_heads.
+ *     Other values return GDN_ERR_UNSUPPORTED.
+ *   - Activations use one dtype per call (gdn_dtype); the recurrent state is always fp32
+ *     [.., Hv, d_v, d_k] with row = value index.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+typedef enum gdn_status {
+  GDN_OK = 0,
+  GDN_ERR_INVALID_ARG = -1, /* null/misaligned pointer, negative size, bad cu_seqlens shape */
+  GDN_ERR_UNSUPPORTED = -2, /* shape or dtype this build does not implement */
+  GDN_ERR_CUDA = -3,        /* a CUDA runtime call or kernel launch failed */
+  GDN_ERR_TIMEOUT = -4,     /* written to dev_status by a device wait that ran out */
+  GDN_ERR_WORKSPACE = -5    /* workspace missing or smaller than *_workspace_size() */
+} gdn_status;
+
+typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Layer shape.  Qwen3-Next: {16, 32, 128, 4, 1.0f, 1e-6f, 1e-6f}. */
+typedef struct gdn_dims {
+  int32_t num_k_heads; /* Hk: query/key heads */
+  int32_t num_v_heads; /* Hv: value heads (state heads), multiple of Hk */
+  int32_t head_dim;    /* d = d_k = d_v (128) */
+  int32_t conv_kernel; /* K, causal conv width (4) */
+  float q_scale;       /* multiplies the L2-normalised q (1.0) */
+  float l2_eps;        /* inside the square root of the q/k L2 norm (1e-6) */
+  float norm_eps;      /* inside the square root of the gated RMSNorm (1e-6) */
+} gdn_dims;
+
+/* Conv channel count Cc = (2*Hk + Hv) * d, in the order [q (Hk*d) | k (Hk*d) | v (Hv*d)]. */
+int64_t gdn_conv_channels(const gdn_dims* dims);
+
+/* Human-readable text of a status code (static string, never NULL). */
+const char* gdn_status_string(int status);
+
+/*
+ * gdn_conv1d_update -- causal depthwise conv (width K, no bias) + SiLU over packed sequences.
+ * Source: the causal convolution of the hyper.ai Gated DeltaNet paragraph; width from
+ * linear_conv_kernel_dim in the Qwen3-Coder-Next raw config.json fields.
+ *   x          [T, Cc]       input rows of all sequences, packed
+ *   y          [T, Cc]       out: y[t,c] = silu(sum_i w[c,i] * x_{t-K+1+i}[c]); may not alias x
+ *   conv_w     [Cc, K]       tap K-1 multiplies the current token
+ *   cu_seqlens [N+1] int32   device; 0 = cu[0] <= cu[1] <= ... <= cu[N] = T
+ *   conv_state_in  [N, K-1, Cc] nullable (= zeros): row j holds x_{j-K+1} of the sequence
+ *   conv_state_out [N, K-1, Cc] nullable: last K-1 rows of [state_in ; x_seq]; may equal
+ *                  conv_state_in (in-place update).
+ * T = 1 per sequence is the decode-time update.
+ */
+int gdn_conv1d_update(const gdn_dims* dims, gdn_dtype dtype, const void* x, void* y,
+                      const void* conv_w, const int32_t* cu_seqlens, int32_t num_seqs,
+                      int32_t num_tokens, const void* conv_state_in, void* conv_state_out,
+                      void* stream);
+
+/*
+ * gdn_gated_rmsnorm -- y = o / sqrt(mean(o^2) + eps) * w * silu(z), per row of `dim`.
+ * Source: the z projection and zero-centred RMSNorm of the hyper.ai Gated DeltaNet
+ * paragraph; eps from rms_norm_eps (Qwen3-Coder-Next raw config.json fields).  `w` is the
+ * effective weight (a zero-centred parameterisation passes 1 + w); NULL means ones.
+ *   o, z, y [rows, dim] (y may equal o), w [dim]; dim a multiple of 8, at most 1024.
+ */
+int gdn_gated_rmsnorm(gdn_dtype dtype, const void* o, const void* z, const void* w, float eps,
+                      int32_t rows, int32_t dim, void* y, void* stream);
+
+/*
+ * gdn_chunk_prefill -- the whole layer over packed variable-length sequences, chunked.
+ * Source: the recurrence in the file header; chunked (WY / UT transform) evaluation as in the
+ * FLA kernels named in the "Qwen3-Next" SGLang cookbook, section 3.2 (this build uses its own
+ * chunk size).  bf16 runs on tcgen05 tensor cores; fp32 runs an fp32 SIMT recurrence.
+ *   x        [T, Cc]          pre-conv q|k|v projections
+ *   conv_w   [Cc, K]          nullable: conv + SiLU switched off (x used as is)
+ *   beta     [T, Hv] fp32     update strength
+ *   g        [T, Hv] fp32     log alpha (<= 0)
+ *   z        [T, Hv, d]       nullable: gated RMSNorm switched off (out = o)
+ *   norm_w   [d]              nullable: ones
+ *   cu_seqlens [N+1] int32    device, as for gdn_conv1d_update
+ *   S0       [N, Hv, d, d] fp32  nullable: zero initial states
+ *   SN       [N, Hv, d, d] fp32  nullable: final states (may equal S0)
+ *   conv0    [N, K-1, Cc]     nullable: zero conv history
+ *   convN    [N, K-1, Cc]     nullable: final conv history (may equal conv0)
+ *   out      [T, Hv, d]
+ *   workspace, workspace_bytes: device scratch of at least
+ *            gdn_chunk_prefill_workspace_size(dims, dtype, N, T) bytes, 256-byte aligned.
+ *   dev_status  int32, nullable: set to GDN_ERR_TIMEOUT if a device wait ran out (the caller
+ *            zeroes it and reads it after synchronising).
+ */
+size_t gdn_chunk_prefill_workspace_size(const gdn_dims* dims, gdn_dtype dtype, int32_t num_seqs,
+                                        int32_t num_tokens);
+int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
+                      const float* beta, const float* g, const void* z, const void* norm_w,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int32_t num_tokens,
+                      const float* S0, float* SN, const void* conv0, void* convN, void* out,
+                      void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * gdn_decode_step -- one token for each of B sequences; conv and recurrent state in place.
+ * Source: as gdn_chunk_prefill with T = 1 per sequence; states resident in a slot pool, fp32
+ * recurrent state as the "Qwen3-Next" SGLang cookbook's default --mamba-ssm-dtype.
+ *   x [B, Cc], beta/g [B, Hv] fp32, z [B, Hv, d] nullable, conv_w [Cc, K] (required),
+ *   norm_w [d] nullable, conv_state [slots, K-1, Cc] in/out, S [slots, Hv, d, d] fp32 in/out,
+ *   slot_idx [B] int32 device, nullable (= identity); slots of one call must be distinct.
+ *   out [B, Hv, d].
+ * One pass over the state: it is read once and written once.
+ */
+int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
+                    const float* beta, const float* g, const void* z, const void* norm_w,
+                    void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
+                    void* out, void* stream);
+
+/*
+ * Launch tracing (host-side measurement aid, not on the compute path).  While a trace is
+ * attached to the calling host thread, every kernel the library launches from that thread is
+ * bracketed by two CUDA events recorded on the launch stream.  After synchronising, read the
+ * per-launch device times.  A trace holds up to 4096 launches; further ones are not recorded.
+ */
+typedef struct gdn_trace gdn_trace;
+int gdn_trace_create(gdn_trace** out);         /* host object, owned by the caller */
+int gdn_trace_destroy(gdn_trace* trace);
+int gdn_trace_attach(gdn_trace* trace);        /* NULL detaches; per host thread */
+int gdn_trace_reset(gdn_trace* trace);
+int gdn_trace_count(const gdn_trace* trace);   /* launches recorded */
+/* name: static kernel name; ms: device time of launch i (synchronises on its end event). */
+int gdn_trace_get(gdn_trace* trace, int32_t i, const char** name, float* ms);
+
+/*
+ * gdn_debug_wait_probe -- test aid for the bounded device waits: launches one CTA that waits
+ * on an mbarrier nothing will complete, with the given limit in microseconds (<= 10^6), and
+ * writes GDN_ERR_TIMEOUT to dev_status when the wait gives up.  No fault, trap or hang.
+ */
+int gdn_debug_wait_probe(int32_t* dev_status, uint32_t limit_us, void* stream);
+
+int gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

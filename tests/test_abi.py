@@ -1,0 +1,140 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol include/gdn.h
+declares, and rejects bad arguments with the documented status before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_deltanet_layer_02_b200 as gdn
+from gated_deltanet_layer_02_b200 import build as gdn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    gdn_build.build()
+    return gdn.lib()
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "gdn.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(gdn.EXPORTS)
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.gdn_abi_version() == 1
+    for code, text in [(0, "ok"), (-1, "invalid argument"), (-2, "unsupported shape or dtype"),
+                       (-3, "CUDA error"), (-4, "device wait timed out"),
+                       (-5, "workspace too small"), (7, "unknown status")]:
+        assert gdn.status_string(code) == text
+
+
+def test_conv_channels(L):
+    assert gdn.conv_channels(gdn.Dims()) == 8192
+    assert gdn.conv_channels(gdn.Dims(2, 4)) == 1024
+    assert L.gdn_conv_channels(None) == -1
+
+
+P = ctypes.c_void_p
+A = P(1 << 20)          # an aligned fake address: never dereferenced on these paths
+MIS = P((1 << 20) + 8)  # misaligned
+
+
+def _prefill(L, dims, dtype=gdn.GDN_BF16, x=A, ws=A, ws_bytes=1 << 40, N=1, T=16, cu=A, out=A,
+             beta=A, g=A):
+    return L.gdn_chunk_prefill(dims, dtype, x, None, beta, g, None, None, cu, N, T, None, None,
+                               None, None, out, ws, ws_bytes, None, None)
+
+
+def test_prefill_argument_errors(L):
+    d = gdn.Dims()
+    assert _prefill(L, None) == gdn.GDN_ERR_INVALID_ARG
+    assert _prefill(L, ctypes.byref(gdn.Dims(head_dim=64))) == gdn.GDN_ERR_UNSUPPORTED
+    assert _prefill(L, ctypes.byref(gdn.Dims(conv_kernel=3))) == gdn.GDN_ERR_UNSUPPORTED
+    assert _prefill(L, ctypes.byref(gdn.Dims(16, 24))) == gdn.GDN_ERR_INVALID_ARG   # 24 % 16
+    assert _prefill(L, ctypes.byref(gdn.Dims(8, 32))) == gdn.GDN_ERR_UNSUPPORTED    # bf16 ratio 4
+    assert _prefill(L, ctypes.byref(d), dtype=5) == gdn.GDN_ERR_UNSUPPORTED
+    assert _prefill(L, ctypes.byref(d), x=MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert _prefill(L, ctypes.byref(d), x=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _prefill(L, ctypes.byref(d), cu=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _prefill(L, ctypes.byref(d), N=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert _prefill(L, ctypes.byref(d), N=0) == gdn.GDN_ERR_INVALID_ARG           # tokens, no seqs
+    assert _prefill(L, ctypes.byref(d), ws=None) == gdn.GDN_ERR_WORKSPACE
+    assert _prefill(L, ctypes.byref(d), ws_bytes=1024) == gdn.GDN_ERR_WORKSPACE
+    assert _prefill(L, ctypes.byref(d), ws=P((1 << 20) + 16)) == gdn.GDN_ERR_INVALID_ARG
+    bad = gdn.Dims()
+    bad.l2_eps = -1.0
+    assert _prefill(L, ctypes.byref(bad)) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_workspace_size(L):
+    d = ctypes.byref(gdn.Dims())
+    f = L.gdn_chunk_prefill_workspace_size
+    assert f(None, 1, 1, 10) == 0
+    assert f(d, 0, -1, 10) == 0
+    assert f(d, gdn.GDN_F32, 1, 4096) == 256
+    small, big = f(d, 1, 1, 4096), f(d, 1, 1, 8192)
+    assert 0 < small < big
+    assert f(d, 1, 8, 4096) > small      # more sequences -> more partial chunks
+
+
+def test_other_entry_points_reject_bad_arguments(L):
+    d = ctypes.byref(gdn.Dims())
+    assert L.gdn_conv1d_update(None, 1, A, A, A, A, 1, 4, None, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_conv1d_update(d, 1, A, A, A, None, 1, 4, None, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_conv1d_update(d, 1, A, A, A, A, 1, 4, MIS, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_conv1d_update(d, 1, A, A, A, A, 1, -4, None, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_gated_rmsnorm(1, A, A, None, 1e-6, 4, 12, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_gated_rmsnorm(1, A, A, None, 1e-6, 4, 2048, A, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_gated_rmsnorm(1, A, None, None, 1e-6, 4, 128, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_gated_rmsnorm(1, A, A, None, -1.0, 4, 128, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_gated_rmsnorm(3, A, A, None, 1e-6, 4, 128, A, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, A, None, -1, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_step(d, 1, A, None, A, A, None, None, A, A, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, MIS, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_step(ctypes.byref(gdn.Dims(1, 16)), 1, A, A, A, A, None, None, A, A, None,
+                             4, A, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_debug_wait_probe(None, 10, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_debug_wait_probe(A, 10_000_000, None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_zero_size_calls_launch_nothing(L):
+    d = ctypes.byref(gdn.Dims())
+    # no sequences, no tokens: valid and a no-op
+    assert L.gdn_chunk_prefill(d, 1, None, None, None, None, None, None, None, 0, 0, None, None,
+                               None, None, None, A, 1 << 30, None, None) == gdn.GDN_OK
+    assert L.gdn_decode_step(d, 1, None, None, None, None, None, None, None, None, None, 0, None,
+                             None) == gdn.GDN_OK
+    assert L.gdn_gated_rmsnorm(1, None, None, None, 1e-6, 0, 128, None, None) == gdn.GDN_OK
+
+
+def test_trace_object_lifecycle(L):
+    h = P()
+    assert L.gdn_trace_create(ctypes.byref(h)) == gdn.GDN_OK
+    assert L.gdn_trace_count(h) == 0
+    assert L.gdn_trace_attach(h) == gdn.GDN_OK
+    assert L.gdn_trace_attach(None) == gdn.GDN_OK
+    assert L.gdn_trace_get(h, 0, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_trace_reset(h) == gdn.GDN_OK
+    assert L.gdn_trace_destroy(h) == gdn.GDN_OK
+    assert L.gdn_trace_create(None) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 8192, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        gdn.conv1d_update(x, torch.zeros(8192, 4, dtype=torch.bfloat16),
+                          torch.tensor([0, 4], dtype=torch.int32))

@@ -1,0 +1,71 @@
+"""GPU parity on the five workload configurations at full size (the launch configuration the
+benchmark times), against the fp64 oracle on the same seeded inputs.
+
+  tiny fp32 T=128 (Hk=2, Hv=4, conv/norm off)   max-abs <= 1e-4 on outputs and final state
+  T=4096 prefill, Qwen3-Next layer shape         max-abs/rms <= 2e-2
+  8-sequence packed varlen prefill, S0 ~ N(0,.1) max-abs/rms <= 2e-2, final states returned
+  decode, 256 sequences x 64 steps               outputs every step, states after step 64
+  T=262144 prefill, slow decay                   last 4096 outputs and the final state
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import gated_deltanet_layer_02_b200 as gdn
+from gated_deltanet_layer_02_b200 import inputs
+from gpu_util import (assert_close, dev, dims_of, ensure_built, gpu_prefill, np64,
+                      oracle_dims_of, oracle_prefill)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2])
+def test_prefill_config(idx):
+    w = inputs.CONFIGS[idx]
+    inp = inputs.prefill_inputs(w, inputs.config_seed(idx))
+    out, SN, convN = gpu_prefill(w, inp)
+    ref_o, ref_S, ref_c = oracle_prefill(w, inp)
+    e_o = assert_close(out, ref_o, w.dtype, f"{w.name}: out")
+    e_s = assert_close(SN, ref_S, w.dtype, f"{w.name}: final state")
+    np.testing.assert_array_equal(np64(convN), ref_c)
+    print(f"{w.name}: out err {e_o:.3g}, state err {e_s:.3g}")
+
+
+@pytest.mark.slow
+def test_long_context_config():
+    w = inputs.CONFIGS[4]
+    inp = inputs.prefill_inputs(w, inputs.config_seed(4))
+    out, SN, _ = gpu_prefill(w, inp, want_state=True)
+    T = w.tokens
+    tail = out[T - 4096:].cpu()
+    del out
+    torch.cuda.empty_cache()
+    ref_o, ref_S, _ = oracle_prefill(w, inp, out_t0=T - 4096)
+    e_o = assert_close(tail, ref_o, w.dtype, "T=262144: last 4096 outputs")
+    e_s = assert_close(SN, ref_S, w.dtype, "T=262144: final state")
+    print(f"{w.name}: out err {e_o:.3g}, state err {e_s:.3g}")
+
+
+def test_decode_config():
+    ensure_built()
+    w = inputs.CONFIGS[3]
+    seed = inputs.config_seed(3)
+    st = inputs.decode_state(w, seed)
+    S_d, cs_d = dev(st["S"]), dev(st["conv_state"])
+    S_ref = st["S"].double().numpy().copy()
+    cs_ref = st["conv_state"].double().numpy().copy()
+    cw, nw = dev(st["conv_w"]), dev(st["norm_w"])
+    dims, od = dims_of(w), oracle_dims_of(w)
+    worst = 0.0
+    for step in range(w.steps):
+        s = inputs.decode_step_inputs(w, seed, step)
+        out = gdn.decode_step(dev(s["x"]), dev(s["beta"]), dev(s["g"]), cs_d, S_d, cw,
+                              z=dev(s["z"]), norm_w=nw, dims=dims)
+        torch.cuda.synchronize()
+        ref = oracle.decode_step(od, s["x"], s["beta"], s["g"], cs_ref, S_ref,
+                                 conv_w=st["conv_w"], z=s["z"], norm_w=st["norm_w"])
+        worst = max(worst, assert_close(out, ref, w.dtype, f"decode out step {step}"))
+    e_s = assert_close(S_d, S_ref, w.dtype, "decode state after 64 steps")
+    np.testing.assert_array_equal(np64(cs_d), cs_ref)
+    print(f"decode: worst out err {worst:.3g}, state err {e_s:.3g}")

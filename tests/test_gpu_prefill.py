@@ -1,0 +1,100 @@
+"""GPU parity of gdn_chunk_prefill against the fp64 oracle on small and edge-case inputs:
+ragged tails around the 128-token chunk, sequences shorter than the conv window, empty
+sequences, initial states, conv/norm switched off, every chain split, determinism."""
+import numpy as np
+import pytest
+import torch
+
+import gated_deltanet_layer_02_b200 as gdn
+from gated_deltanet_layer_02_b200 import inputs
+from gpu_util import assert_close, gpu_prefill, np64, oracle_prefill
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(w, inp, what):
+    out, SN, convN = gpu_prefill(w, inp)
+    ref_o, ref_S, ref_c = oracle_prefill(w, inp)
+    e1 = assert_close(out, ref_o, w.dtype, f"{what}: out")
+    e2 = assert_close(SN, ref_S, w.dtype, f"{what}: final state")
+    np.testing.assert_array_equal(np64(convN), ref_c)
+    return e1, e2
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 63, 64, 65, 127, 128, 129, 300])
+def test_bf16_single_sequence_lengths(T):
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(T,))
+    _check(w, inputs.prefill_inputs(w, 500 + T), f"T={T}")
+
+
+@pytest.mark.parametrize("T", [1, 3, 129, 300])
+def test_f32_single_sequence_lengths(T):
+    w = inputs.custom(2, 4, 128, torch.float32, lengths=(T,))
+    _check(w, inputs.prefill_inputs(w, 600 + T), f"f32 T={T}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_varlen_with_states_and_empty_sequences(dtype):
+    w = inputs.custom(2, 4, 128, dtype, lengths=(1, 0, 130, 2, 257, 0, 64), s0_std=0.1)
+    _check(w, inputs.prefill_inputs(w, 700, with_conv0=True), "varlen")
+
+
+@pytest.mark.parametrize("conv,norm", [(False, True), (True, False), (False, False)])
+def test_bf16_conv_and_norm_switches(conv, norm):
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(200,), conv=conv, norm=norm)
+    _check(w, inputs.prefill_inputs(w, 800 + 2 * conv + norm), f"conv={conv} norm={norm}")
+
+
+@pytest.mark.parametrize("nseq", [1, 20, 40])
+def test_bf16_every_chain_split(nseq):
+    # N*Hv units decide the d_v split of the chain kernel: 4 -> 4 blocks, 80 -> 2, 160 -> 1
+    lengths = tuple(int(v) for v in np.random.default_rng(900 + nseq).integers(1, 300, nseq))
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=lengths, s0_std=0.1)
+    _check(w, inputs.prefill_inputs(w, 900 + nseq), f"nseq={nseq}")
+
+
+def test_bf16_long_memory_gates():
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(1000,), g_dist="uniform", g_low=-0.05,
+                      s0_std=0.1)
+    _check(w, inputs.prefill_inputs(w, 950), "slow decay")
+
+
+def test_bf16_state_in_place_and_deterministic():
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(77, 300), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 960, with_conv0=True)
+    a = gpu_prefill(w, inp)
+    b = gpu_prefill(w, inp)
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+    # S0 == SN and conv0 == convN (in-place state update)
+    S = inp["S0"].cuda()
+    c = inp["conv0"].cuda()
+    out, _, _ = gdn.chunk_prefill(inp["x"].cuda(), inp["beta"].cuda(), inp["g"].cuda(),
+                                  inp["cu_seqlens"].cuda(), conv_w=inp["conv_w"].cuda(),
+                                  z=inp["z"].cuda(), norm_w=inp["norm_w"].cuda(), S0=S, SN=S,
+                                  conv0=c, convN=c, dims=gdn.Dims(2, 4))
+    torch.cuda.synchronize()
+    assert torch.equal(out, a[0])
+    assert torch.equal(S, a[1])
+    assert torch.equal(c, a[2])
+
+
+def test_split_prefill_matches_whole():
+    """prefill(0..T) == prefill(0..T1) then prefill(T1..T) with the carried states."""
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(390,), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 970, with_conv0=True)
+    full = gpu_prefill(w, inp)
+    T1 = 200
+    first = {k: v for k, v in inp.items()}
+    second = {k: v for k, v in inp.items()}
+    for k in ("x", "beta", "g", "z"):
+        first[k], second[k] = inp[k][:T1], inp[k][T1:]
+    first["cu_seqlens"] = inputs.cu_seqlens_of([T1])
+    second["cu_seqlens"] = inputs.cu_seqlens_of([390 - T1])
+    a = gpu_prefill(w, first)
+    second["S0"], second["conv0"] = a[1].cpu(), a[2].cpu()
+    b = gpu_prefill(w, second)
+    ref_o, ref_S, _ = oracle_prefill(w, inp)
+    assert_close(torch.cat([a[0], b[0]]), ref_o, w.dtype, "split out")
+    assert_close(b[1], ref_S, w.dtype, "split state")
+    assert torch.equal(b[2], full[2])

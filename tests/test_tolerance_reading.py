@@ -1,0 +1,28 @@
+"""Why the bf16 parity bar is the relative RMS error (CPU only).
+
+The workload statement asks for agreement "within 2e-2 relative-to-RMS" for bf16 activations.
+Read as max|gpu - oracle| / rms(oracle), the bar would reject even the exact result rounded once
+to bf16, because the z-gated RMSNorm output is heavy-tailed (elements reach 10-15x its RMS and
+bf16 keeps 8 significant bits).  Read as ||gpu - oracle||_2 / ||oracle||_2 it is met by that
+rounding with a wide margin.  The tests use the second reading.
+"""
+import numpy as np
+import torch
+
+import oracle
+from gated_deltanet_layer_02_b200 import inputs
+
+
+def test_bf16_rounding_of_exact_output_breaks_max_abs_reading_only():
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300,))
+    inp = inputs.prefill_inputs(w, 800)
+    ref, _, _ = oracle.prefill(oracle.Dims(2, 4), inp["x"], inp["beta"], inp["g"],
+                               inp["cu_seqlens"], conv_w=inp["conv_w"], z=inp["z"],
+                               norm_w=inp["norm_w"], want_state=False)
+    rounded = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+    rms = np.sqrt(np.mean(ref ** 2))
+    max_abs_reading = np.max(np.abs(rounded - ref)) / rms
+    rel_rms_reading = np.sqrt(np.mean((rounded - ref) ** 2)) / rms
+    assert max_abs_reading > 2e-2          # the exact answer in bf16 "fails"
+    assert rel_rms_reading < 2e-3          # and sits 10x inside the relative RMS bar
+    assert np.max(np.abs(ref)) > 10 * rms  # because the normalised output is heavy-tailed
