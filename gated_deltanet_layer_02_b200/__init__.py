@@ -29,7 +29,11 @@ EXPORTS = (
     "gdn_gated_rmsnorm", "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill",
     "gdn_decode_step", "gdn_trace_create", "gdn_trace_destroy", "gdn_trace_attach",
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
+    "gdn_chunk_prefill_static_ws",
 )
+
+#: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
+STATIC_WORKSPACE_BYTES = 64 << 20
 
 
 class GdnError(RuntimeError):
@@ -89,6 +93,8 @@ def lib():
             L.gdn_trace_get.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_char_p),
                                         ctypes.POINTER(ctypes.c_float)]
             L.gdn_debug_wait_probe.argtypes = [vp, ctypes.c_uint32, vp]
+            L.gdn_chunk_prefill_static_ws.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                                      i32, i32, vp, vp, vp, vp, vp, vp, vp]
             for name in EXPORTS:  # every declared symbol must resolve
                 getattr(L, name)
             _lib = L
@@ -205,6 +211,37 @@ def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=N
     return out, SN, convN
 
 
+def chunk_prefill_static_ws(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None,
+                            SN=None, conv0=None, convN=None, out=None, dev_status=None,
+                            want_state=True, dims: Dims | None = None):
+    """chunk_prefill without a caller workspace: the library's own 64 MiB device scratch is used.
+
+    For callers that cannot allocate device memory.  Calls on one device share that scratch, so
+    they must not overlap on the GPU.  Sizes needing more scratch raise GdnError
+    (GDN_ERR_WORKSPACE).  Returns (out, SN, convN) like chunk_prefill.
+    """
+    dims = dims or Dims()
+    dt = _act_dtype(x)
+    T = x.shape[0]
+    N = cu_seqlens.numel() - 1
+    Hv, d, K = dims.num_v_heads, dims.head_dim, dims.conv_kernel
+    dev = x.device
+    if out is None:
+        out = torch.empty((T, Hv, d), dtype=x.dtype, device=dev)
+    if want_state and SN is None:
+        SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
+    if want_state and convN is None:
+        convN = torch.empty((N, K - 1, dims.channels), dtype=x.dtype, device=dev)
+    _check("gdn_chunk_prefill_static_ws", lib().gdn_chunk_prefill_static_ws(
+        ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
+        _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
+        _ptr(norm_w, "norm_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N, T,
+        _ptr(S0, "S0", torch.float32), _ptr(SN, "SN", torch.float32),
+        _ptr(conv0, "conv0", x.dtype), _ptr(convN, "convN", x.dtype), _ptr(out, "out", x.dtype),
+        _ptr(dev_status, "dev_status", torch.int32), _stream()))
+    return out, SN, convN
+
+
 def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx=None,
                 out=None, dims: Dims | None = None):
     """One token per sequence; conv_state and S are updated in place.  Returns out [B, Hv, d]."""
@@ -269,5 +306,6 @@ class Trace:
 
 
 __all__ = ["Dims", "GdnError", "lib", "conv1d_update", "gated_rmsnorm", "chunk_prefill",
+           "chunk_prefill_static_ws", "STATIC_WORKSPACE_BYTES",
            "decode_step", "prefill_workspace_size", "conv_channels", "status_string", "Trace",
            "debug_wait_probe", "EXPORTS", "LIB_PATH"]

@@ -146,6 +146,34 @@ int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const 
                     void* out, void* stream);
 
 /*
+ * gdn_chunk_prefill_static_ws -- gdn_chunk_prefill for callers that cannot allocate device
+ * memory.  No counterpart on the source pages: this is a deployment aid of this library.
+ * Some callers have no way to obtain a device workspace: extensions loaded into a host
+ * framework that owns every device allocation and lends none to plugins, C programs without a
+ * caching allocator, and latency-critical loops that must not pay the implicit device
+ * synchronisation of cudaMalloc/cudaFree.  This entry point takes the same arguments as
+ * gdn_chunk_prefill minus workspace/workspace_bytes and allocates nothing: its scratch is a
+ * file-scope device array of GDN_STATIC_WORKSPACE_BYTES (64 MiB) inside libgdn.so, which every
+ * GPU that loads the library holds until the process exits.
+ *   - Sizes whose gdn_chunk_prefill_workspace_size() exceeds GDN_STATIC_WORKSPACE_BYTES return
+ *     GDN_ERR_WORKSPACE and launch nothing (for the Qwen3-Next shape, one sequence of up to
+ *     1,791 tokens, or fewer tokens spread over more sequences).
+ *   - The first call on each device looks the array's device address up (cudaGetSymbolAddress,
+ *     with that device current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents (nothing in it
+ *     needs to start at zero).  Calls that overlap on the GPU (different streams, or different
+ *     host threads on one device) race on it and must be serialised by the caller.
+ * Other arguments, results and status codes are those of gdn_chunk_prefill.
+ */
+#define GDN_STATIC_WORKSPACE_BYTES (64u << 20)
+int gdn_chunk_prefill_static_ws(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                                const void* conv_w, const float* beta, const float* g,
+                                const void* z, const void* norm_w, const int32_t* cu_seqlens,
+                                int32_t num_seqs, int32_t num_tokens, const float* S0, float* SN,
+                                const void* conv0, void* convN, void* out, int32_t* dev_status,
+                                void* stream);
+
+/*
  * Launch tracing (host-side measurement aid, not on the compute path).  While a trace is
  * attached to the calling host thread, every kernel the library launches from that thread is
  * bracketed by two CUDA events recorded on the launch stream.  After synchronising, read the

@@ -138,3 +138,19 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(ValueError, match="CUDA"):
         gdn.conv1d_update(x, torch.zeros(8192, 4, dtype=torch.bfloat16),
                           torch.tensor([0, 4], dtype=torch.int32))
+
+
+def test_static_workspace_entry_point_rejects_oversized_calls(L):
+    """Sizes whose scratch exceeds the library's static array are refused before any launch."""
+    d = ctypes.byref(gdn.Dims())
+    f = L.gdn_chunk_prefill_workspace_size
+    assert f(d, 1, 1, 1791) <= gdn.STATIC_WORKSPACE_BYTES < f(d, 1, 1, 1792)
+    args = (d, 1, A, None, A, A, None, None, A)
+    tail = (None, None, None, None, A, None, None)
+    assert L.gdn_chunk_prefill_static_ws(*args, 1, 1792, *tail) == gdn.GDN_ERR_WORKSPACE
+    assert L.gdn_chunk_prefill_static_ws(*args, 64, 64, *tail) == gdn.GDN_ERR_WORKSPACE
+    # invalid shapes keep the regular entry point's status codes
+    assert L.gdn_chunk_prefill_static_ws(None, 1, A, None, A, A, None, None, A, 1, 16,
+                                         *tail) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_chunk_prefill_static_ws(ctypes.byref(gdn.Dims(head_dim=64)), 1, A, None, A, A,
+                                         None, None, A, 1, 16, *tail) == gdn.GDN_ERR_UNSUPPORTED
