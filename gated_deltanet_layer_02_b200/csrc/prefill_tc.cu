@@ -75,53 +75,188 @@ __global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Wor
 }
 
 
+// --------------------------------------------------------------------------------- q/k/v
+// One CTA per (chunk, 128-channel group of the conv input): causal conv (width 4) + SiLU, and
+// for q and k the L2 norm of every (token, head) row.  128 threads: 16 column vectors x 8 runs
+// of 16 tokens; the 16 threads of a row share a half-warp, so the norm is a 4-step shuffle.
+// Outputs are bf16 [128][128] tiles per (chunk, head): Q -> Qw, K -> Kw, V -> Uw (V is read by
+// gdn_prep, which overwrites the same tile with U~).  Rows past the chunk's length are zero.
+__device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// silu(x) = x * sigmoid(x), sigmoid(x) = (1 + tanh(x / 2)) / 2: one transcendental per element.
+__device__ __forceinline__ float silu_fast(float x) {
+  const float h = 0.5f * x;
+  return fmaf(h, tanh_approx(h), h);
+}
+
+__global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a) {
+  const int c = blockIdx.x, grp = blockIdx.y;
+  if (c >= a.ws.seq_first[a.N]) return;
+  const ChunkInfo ci = a.ws.chunks[c];
+  const int tid = threadIdx.x, vec = tid & 15, run = tid >> 4;
+  const int Hk = a.Hk, Hv = a.Hv;
+  const int Cc = (2 * Hk + Hv) * kD;
+  const int kind = grp < Hk ? 0 : (grp < 2 * Hk ? 1 : 2);
+  const int head = kind == 0 ? grp : (kind == 1 ? grp - Hk : grp - 2 * Hk);
+  const int ch = grp * kD + vec * 8;
+  __nv_bfloat16* dst = (kind == 0 ? a.ws.Qw + ((size_t)c * Hk + head) * kC * kD
+                      : kind == 1 ? a.ws.Kw + ((size_t)c * Hk + head) * kC * kD
+                                  : a.ws.Uw + ((size_t)c * Hv + head) * kC * kD) + vec * 8;
+  const int seq_start = __ldg(a.cu + ci.n);
+  float2 wv[4][4];  // taps x channel pairs
+  if (a.conv_w) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      uint2 u = *reinterpret_cast<const uint2*>(a.conv_w + (size_t)(ch + e) * 4);
+      const __nv_bfloat162* hw = reinterpret_cast<const __nv_bfloat162*>(&u);
+      const float2 f0 = __bfloat1622float2(hw[0]), f1 = __bfloat1622float2(hw[1]);
+      const float t[4] = {f0.x, f0.y, f1.x, f1.y};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (e & 1) wv[k][e >> 1].y = t[k]; else wv[k][e >> 1].x = t[k];
+      }
+    }
+  }
+  const int i0 = run * 16;
+  float2 hst[3][4];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const int t = ci.t0 + i0 - 3 + j;
+    float v8[8];
+    if (i0 >= ci.L) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v8[e] = 0.f;
+    } else if (t >= seq_start) {
+      load8(a.x + (size_t)t * Cc + ch, v8);
+    } else if (a.conv0) {
+      load8(a.conv0 + ((size_t)ci.n * 3 + 3 + (t - seq_start)) * Cc + ch, v8);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v8[e] = 0.f;
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) hst[j][p] = make_float2(v8[2 * p], v8[2 * p + 1]);
+  }
+  const float sc_mul = kind == 0 ? a.q_scale : 1.0f;
+  constexpr int kPF = 4;
+#pragma unroll 1
+  for (int i8 = 0; i8 < 16; i8 += kPF) {
+    uint4 raw[kPF];
+#pragma unroll
+    for (int u = 0; u < kPF; ++u) {
+      const int i = i0 + i8 + u;
+      raw[u] = (i < ci.L) ? __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)(ci.t0 + i) * Cc + ch))
+                          : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kPF; ++u) {
+      const int i = i0 + i8 + u;
+      float xv[8], y[8];
+      unpack8(raw[u], xv);
+      if (a.conv_w) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 xp = make_float2(xv[2 * p], xv[2 * p + 1]);
+          float2 acc = __fmul2_rn(wv[3][p], xp);
+          acc = __ffma2_rn(wv[2][p], hst[2][p], acc);
+          acc = __ffma2_rn(wv[1][p], hst[1][p], acc);
+          acc = __ffma2_rn(wv[0][p], hst[0][p], acc);
+          y[2 * p] = silu_fast(acc.x);
+          y[2 * p + 1] = silu_fast(acc.y);
+          hst[0][p] = hst[1][p];
+          hst[1][p] = hst[2][p];
+          hst[2][p] = xp;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = xv[e];
+      }
+      if (kind < 2) {
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss += y[e] * y[e];
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float sc = sc_mul * rsqrtf(ss + a.l2_eps);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] *= sc;
+      }
+      if (i >= ci.L) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = 0.f;
+      }
+      store8(dst + (size_t)i * kD, y);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------- prep
+// One CTA per (chunk, value head), 8 warps, two CTAs per SM.  K and V arrive by TMA from the
+// tiles gdn_qkv wrote.  Gates -> K K^T (tcgen05) -> A -> two 64x64 forward substitutions (CUDA
+// cores) -> Y = N T_h, Z' = T_h Y diag(beta) (tcgen05) -> T diag(beta) -> W and U~ (tcgen05).
 // smem map (bytes from the 1024-aligned base)
-constexpr uint32_t kPrepKs = 0;
-constexpr uint32_t kPrepV0 = 32768;
-constexpr uint32_t kPrepV1 = 65536;
-constexpr uint32_t kPrepR1 = 98304;    // A^T blocks (fp32) -> T_h^T (bf16) -> T diag(beta)
-constexpr uint32_t kPrepR2 = 131072;   // N (16 KB) + Y' (8 KB) -> K^ = diag(e^G) K
-constexpr uint32_t kPrepEnd = 163840;
-constexpr uint32_t kPrepSmem = kPrepEnd + 1024 + 4096;
-// TMEM columns
-constexpr uint32_t kColGram = 0, kColY = 128, kColZ = 192, kColW = 256, kColU = 384;
+constexpr uint32_t kPrepKs = 0;        // K (TMA) -> K^ = diag(e^G) K, in place
+constexpr uint32_t kPrepR1 = 32768;    // A^T blocks (fp32) -> T_h^T (bf16) -> T diag(beta)
+constexpr uint32_t kPrepR2 = 65536;    // N (16 KB) + Y' (8 KB) -> V (TMA)
+constexpr uint32_t kPrepEnd = 98304;
+constexpr uint32_t kPrepSmem = kPrepEnd + 1024 + 1536;
+// TMEM columns (256 allocated)
+constexpr uint32_t kColGram = 0, kColY = 128, kColZ = 192, kColW = 0, kColU = 128;
 
 __device__ __forceinline__ void zero_row_chunk(uint8_t* tile, uint32_t row, uint32_t chunk) {
   *reinterpret_cast<uint4*>(tile + sw128_off(row, chunk)) = make_uint4(0, 0, 0, 0);
 }
 
-__global__ void __launch_bounds__(256, 1) gdn_prep_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
+                                                          const __grid_constant__ CUtensorMap mapK,
+                                                          const __grid_constant__ CUtensorMap mapV) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  float* G_s = reinterpret_cast<float*>(sm + kPrepEnd);        // [2][128]
-  float* B_s = G_s + 2 * kC;                                    // [2][128]
-  float* wt_s = B_s + 2 * kC;                                   // [8] warp totals
-  uint64_t* bar = reinterpret_cast<uint64_t*>(wt_s + 8);        // [1]
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
-  int* abort_s = reinterpret_cast<int*>(tslot + 1);
+  float* G_s = reinterpret_cast<float*>(sm + kPrepEnd);        // [128]
+  float* B_s = G_s + kC;                                        // [128]
+  float* wt_s = B_s + kC;                                       // [4] warp totals
+  uint64_t* bar_k = reinterpret_cast<uint64_t*>(wt_s + 8);
+  uint64_t* bar_v = bar_k + 1;
+  uint64_t* bar = bar_k + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_k + 3);
 
   const int c = blockIdx.x;
-  const int hk = blockIdx.y;
+  const int h = blockIdx.y;
   const int total_chunks = a.ws.seq_first[a.N];
   if (c >= total_chunks) return;
   const ChunkInfo ci = a.ws.chunks[c];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int Hk = a.Hk, Hv = a.Hv;
-  const int Cc = (2 * Hk + Hv) * kD;
-  const int seq_start = __ldg(a.cu + ci.n);
+  const int quarter = warp & 3, wg = warp >> 2;
+  const int Hv = a.Hv;
+  const int hk = h / (Hv / a.Hk);
 
   if (tid == 0) {
+    mbar_init(bar_k, 1);
+    mbar_init(bar_v, 1);
     mbar_init(bar, 1);
     fence_barrier_init();
-    *abort_s = 0;
+    const int rowK = (c * a.Hk + hk) * kC;
+    mbar_arrive_expect_tx(bar_k, 2 * kTile);
+    tma_load_2d(sm + kPrepKs, &mapK, bar_k, 0, rowK);
+    tma_load_2d(sm + kPrepKs + kTile, &mapK, bar_k, 64, rowK);
   }
-  if (warp == 0) tmem_alloc(tslot, 512);
-  // ---------------- gates: G = inclusive cumsum of g inside the chunk, beta (2 value heads)
-  {
-    const int r = warp >> 2, i = (warp & 3) * 32 + lane;
-    const int h = hk * 2 + r;
+  if (warp == 0) tmem_alloc(tslot, 256);
+  // ---------------- gates: G = inclusive cumsum of g inside the chunk, beta
+  if (warp < 4) {
+    const int i = warp * 32 + lane;
     const bool valid = i < ci.L;
     float gv = valid ? __ldg(a.g + (size_t)(ci.t0 + i) * Hv + h) : 0.f;
     const float bv = valid ? __ldg(a.beta + (size_t)(ci.t0 + i) * Hv + h) : 0.f;
@@ -131,173 +266,121 @@ __global__ void __launch_bounds__(256, 1) gdn_prep_kernel(PrefillArgs a) {
       if (lane >= o) gv += y;
     }
     if (lane == 31) wt_s[warp] = gv;
-    B_s[r * kC + i] = bv;
-    __syncthreads();
+    B_s[i] = bv;
+    G_s[i] = gv;  // warp-local prefix; completed below
+  }
+  __syncthreads();
+  if (warp < 4) {
+    const int i = warp * 32 + lane;
     float pre = 0.f;
-    for (int w = r * 4; w < warp; ++w) pre += wt_s[w];
-    gv += pre;
-    G_s[r * kC + i] = gv;
+    for (int w = 0; w < warp; ++w) pre += wt_s[w];
+    const float gv = G_s[i] + pre;
+    G_s[i] = gv;
     a.ws.Gw[((size_t)c * Hv + h) * kC + i] = gv;
   }
-  // ---------------- conv + SiLU + L2 norms -> Q, K (global), K, V0, V1 (smem operands)
-  {
-    const int run = tid >> 6, cvec = tid & 63, grp = cvec >> 4, vec = cvec & 15;
-    int ch;
-    if (grp == 0) ch = hk * kD;
-    else if (grp == 1) ch = Hk * kD + hk * kD;
-    else ch = 2 * Hk * kD + (hk * 2 + grp - 2) * kD;
-    ch += vec * 8;
-    float wv[4][8];
-    if (a.conv_w) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        uint2 u = *reinterpret_cast<const uint2*>(a.conv_w + (size_t)(ch + e) * 4);
-        const __nv_bfloat162* hw = reinterpret_cast<const __nv_bfloat162*>(&u);
-        float2 f0 = __bfloat1622float2(hw[0]), f1 = __bfloat1622float2(hw[1]);
-        wv[0][e] = f0.x; wv[1][e] = f0.y; wv[2][e] = f1.x; wv[3][e] = f1.y;
-      }
-    }
-    const int i0 = run * 32;
-    float hst[3][8];
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      const int t = ci.t0 + i0 - 3 + j;
-      if (i0 >= ci.L) {  // the whole run is padding: nothing to read
-#pragma unroll
-        for (int e = 0; e < 8; ++e) hst[j][e] = 0.f;
-      } else if (t >= seq_start) {
-        load8(a.x + (size_t)t * Cc + ch, hst[j]);
-      } else if (a.conv0) {
-        load8(a.conv0 + ((size_t)ci.n * 3 + 3 + (t - seq_start)) * Cc + ch, hst[j]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) hst[j][e] = 0.f;
-      }
-    }
-    uint8_t* vtile = sm + (grp == 2 ? kPrepV0 : kPrepV1);
-    const size_t qk_base = ((size_t)c * Hk + hk) * kC * kD;
-    for (int ii = 0; ii < 32; ++ii) {
-      const int i = i0 + ii;
-      const bool valid = i < ci.L;
-      float y[8];
-      if (valid) {
-        float xv[8];
-        load8(a.x + (size_t)(ci.t0 + i) * Cc + ch, xv);
-        if (a.conv_w) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float acc = wv[0][e] * hst[0][e] + wv[1][e] * hst[1][e] + wv[2][e] * hst[2][e] +
-                              wv[3][e] * xv[e];
-            y[e] = acc / (1.0f + __expf(-acc));
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = xv[e];
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          hst[0][e] = hst[1][e];
-          hst[1][e] = hst[2][e];
-          hst[2][e] = xv[e];
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = 0.f;
-      }
-      float ss = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ss += y[e] * y[e];
-#pragma unroll
-      for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      if (grp < 2) {
-        const float sc = (grp == 0 ? a.q_scale : 1.0f) * rsqrtf(ss + a.l2_eps);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = valid ? y[e] * sc : 0.f;
-        __nv_bfloat16* dst = (grp == 0 ? a.ws.Qw : a.ws.Kw) + qk_base + (size_t)i * kD + vec * 8;
-        store8(dst, y);
-        if (grp == 1) st_row8_bf16(sm + kPrepKs, kTile, i, vec, y);
-      } else {
-        st_row8_bf16(vtile, kTile, i, vec, y);
-      }
-    }
-  }
-  fence_proxy_async_smem();
   __syncthreads();
+  tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t sKs = smem_u32(sm + kPrepKs);
+  const uint32_t lane_addr = tmem_at(tmem, quarter * 32, 0);
   uint32_t phase = 0;
+  bool ok = true;
   // ---------------- gram K K^T
   if (tid == 0) {
+    ok = mbar_wait(bar_k, 0);
     tc_fence_after();
+    if (ok) {
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_bf16(tmem + kColGram, desc_kmajor(sKs, kk, kTile), desc_kmajor(sKs, kk, kTile),
-               idesc_bf16(128, 128, false, false), kk > 0);
-    mma_commit(bar);
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16(tmem + kColGram, desc_kmajor(sKs, kk, kTile), desc_kmajor(sKs, kk, kTile),
+                 idesc_bf16(128, 128, false, false), kk > 0);
+      mma_commit(bar);
+    }
   }
-  bool ok = mbar_wait(bar, phase);
+  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(bar, phase);
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-
-  for (int r = 0; r < 2; ++r) {
-    const int h = hk * 2 + r;
-    const float* Gr = G_s + r * kC;
-    const float* Br = B_s + r * kC;
-    float* AT = reinterpret_cast<float*>(sm + kPrepR1);    // [2][64][64]
-    uint8_t* Nt = sm + kPrepR2;                            // [128][64] bf16 tile
-    uint8_t* Yt = sm + kPrepR2 + kTile;                    // [64][64] bf16 tile
-    // ---- A from the gram: thread row i, columns [half*64, half*64+64)
-    {
-      const int i = (warp & 3) * 32 + lane, half = warp >> 2;
-      const float Gi = Gr[i], bi = Br[i];
-      const uint32_t taddr = tmem_at(tmem, (warp & 3) * 32, kColGram + half * 64);
+  // ---------------- A from the gram: thread row i, column half wg
+  {
+    const int i = quarter * 32 + lane, half = wg;
+    const float Gi = G_s[i], bi = B_s[i];
+    float* ATh = reinterpret_cast<float*>(sm + kPrepR1) + half * 4096;
+    uint8_t* Nt = sm + kPrepR2;
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+    for (int cc = 0; cc < 2; ++cc) {
+      const int j0 = half * 64 + cc * 32;
+      // warp-uniform: does any row of this warp have j < i inside this column chunk?
+      const bool any_lower = j0 < quarter * 32 + 31;
+      const bool needed = ((i >> 6) == half) || (half == 0);
+      float av[32];
+      if (any_lower) {
         float v[32];
-        tmem_ld32(taddr + cc * 32, v);
+        tmem_ld32(lane_addr + kColGram + j0, v);
         tmem_ld_wait();
-        const int j0 = half * 64 + cc * 32;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int j = j0 + e;
-          v[e] = (j < i) ? bi * __expf(Gi - Gr[j]) * v[e] : 0.f;
+          av[e] = (j < i) ? bi * __expf(Gi - G_s[j]) * v[e] : 0.f;
         }
-        if ((i >> 6) == half) {
-          // diagonal block: store transposed, AT[b][jj][ii]
-          float* dst = AT + half * 4096;
+      } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) dst[((j0 + e) & 63) * 64 + (i & 63)] = v[e];
-        } else if (half == 0) {
+        for (int e = 0; e < 32; ++e) av[e] = 0.f;
+      }
+      if (needed) {
+        if ((i >> 6) == half) {
+          // diagonal block: transposed, ATh[jj][ii]
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ATh[((j0 + e) & 63) * 64 + (i & 63)] = av[e];
+        } else {
           // lower-left block (i >= 64, j < 64) -> N (bf16, K-major)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) st_row8_bf16(Nt, kTile, i, (j0 >> 3) + q, v + 8 * q);
+          for (int q = 0; q < 4; ++q) st_row8_bf16(Nt, kTile, i, (j0 >> 3) + q, av + 8 * q);
         }
       }
-      if (i < 64 && half == 0) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) zero_row_chunk(Nt, i, q);
-      }
     }
-    tc_fence_before();
-    __syncthreads();
-    // ---- two 64x64 unit-lower inverses by forward substitution (column per thread)
+    if (i < 64 && half == 0) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) zero_row_chunk(Nt, i, q);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  {
+    // ---- two 64x64 unit-lower inverses by forward substitution (threads 0..127: one column
+    // each).  Columns 32..63 are zero above their diagonal, so those warps skip ii < 32.
+    const int sb = (tid >> 6) & 1, sn = tid & 63;
     float acc[64];
-    const int sb = tid >> 6, sn = tid & 63;
     if (tid < 128) {
 #pragma unroll
       for (int rr = 0; rr < 64; ++rr) acc[rr] = (rr == sn) ? 1.f : 0.f;
-      const float* ATb = AT + sb * 4096;
+      const float* ATb = reinterpret_cast<const float*>(sm + kPrepR1) + sb * 4096;
+      const bool upper_cols = sn >= 32;  // warp-uniform
 #pragma unroll
       for (int ii = 0; ii < 63; ++ii) {
+        if (ii < 32 && upper_cols) continue;
         const float ti = acc[ii];
+        const float2 t2 = make_float2(-ti, -ti);
 #pragma unroll
         for (int r4 = (ii + 1) & ~3; r4 < 64; r4 += 4) {
           const float4 av = *reinterpret_cast<const float4*>(ATb + ii * 64 + r4);
-          if (r4 + 0 > ii) acc[r4 + 0] -= av.x * ti;
-          if (r4 + 1 > ii) acc[r4 + 1] -= av.y * ti;
-          if (r4 + 2 > ii) acc[r4 + 2] -= av.z * ti;
-          if (r4 + 3 > ii) acc[r4 + 3] -= av.w * ti;
+          if (r4 > ii) {
+            const float2 lo =
+                __ffma2_rn(make_float2(av.x, av.y), t2, make_float2(acc[r4], acc[r4 + 1]));
+            acc[r4] = lo.x;
+            acc[r4 + 1] = lo.y;
+          } else if (r4 + 1 > ii) {
+            acc[r4 + 1] -= av.y * ti;
+          }
+          if (r4 + 2 > ii) {
+            const float2 hi =
+                __ffma2_rn(make_float2(av.z, av.w), t2, make_float2(acc[r4 + 2], acc[r4 + 3]));
+            acc[r4 + 2] = hi.x;
+            acc[r4 + 3] = hi.y;
+          } else if (r4 + 3 > ii) {
+            acc[r4 + 3] -= av.w * ti;
+          }
         }
       }
     }
@@ -318,7 +401,7 @@ __global__ void __launch_bounds__(256, 1) gdn_prep_kernel(PrefillArgs a) {
     // ---- Y = N T_h (M=128, N=64, K=64)
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t sN = smem_u32(Nt), sT = smem_u32(TT);
+      const uint32_t sN = smem_u32(sm + kPrepR2), sT = smem_u32(TT);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + kColY, desc_kmajor(sN, kk, kTile), desc_kmajor(sT, kk, kTile),
@@ -330,13 +413,14 @@ __global__ void __launch_bounds__(256, 1) gdn_prep_kernel(PrefillArgs a) {
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
     // ---- Y' = Y diag(beta) restricted to rows 64..127, cols 0..63 -> bf16 [64][64]
-    if ((warp & 3) >= 2) {
-      const int j = (warp & 3) * 32 + lane, half = warp >> 2;
+    if (quarter >= 2) {
+      const int j = quarter * 32 + lane, half = wg;
       float v[32];
-      tmem_ld32(tmem_at(tmem, (warp & 3) * 32, kColY + half * 32), v);
+      tmem_ld32(lane_addr + kColY + half * 32, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] *= Br[half * 32 + e];
+      for (int e = 0; e < 32; ++e) v[e] *= B_s[half * 32 + e];
+      uint8_t* Yt = sm + kPrepR2 + kTile;
 #pragma unroll
       for (int q = 0; q < 4; ++q) st_row8_bf16(Yt, kTile, j - 64, half * 4 + q, v + 8 * q);
     }
@@ -346,7 +430,7 @@ __global__ void __launch_bounds__(256, 1) gdn_prep_kernel(PrefillArgs a) {
     // ---- Z' = T_h Y' (M=128, N=64, K=64 over rows 64..127 of T_h)
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t sT = smem_u32(TT), sY = smem_u32(Yt);
+      const uint32_t sT = smem_u32(TT), sY = smem_u32(sm + kPrepR2 + kTile);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16(tmem + kColZ, desc_mnmajor(sT + 8192, kk, kTile), desc_mnmajor(sY, kk, kTile),
@@ -357,13 +441,18 @@ __global__ void __launch_bounds__(256, 1) gdn_prep_kernel(PrefillArgs a) {
     phase ^= 1;
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
-    // ---- T diag(beta) (bf16, K-major [i][j]) into R1; K^ = diag(e^G) K into R2
+    // ---- V into R2 (N and Y' are consumed) while T diag(beta) and K^ are built
+    if (tid == 0) {
+      const int rowV = (c * Hv + h) * kC;
+      mbar_arrive_expect_tx(bar_v, 2 * kTile);
+      tma_load_2d(sm + kPrepR2, &mapV, bar_v, 0, rowV);
+      tma_load_2d(sm + kPrepR2 + kTile, &mapV, bar_v, 64, rowV);
+    }
     uint8_t* TB = sm + kPrepR1;
-    uint8_t* Kh = sm + kPrepR2;
     if (tid < 128) {
       // diagonal blocks from the column owners: element (sb*64+rr, sb*64+sn)
       const int col = sb * 64 + sn;
-      const float bcol = Br[col];
+      const float bcol = B_s[col];
 #pragma unroll
       for (int rr = 0; rr < 64; ++rr) {
         const int row = sb * 64 + rr;
@@ -376,87 +465,88 @@ __global__ void __launch_bounds__(256, 1) gdn_prep_kernel(PrefillArgs a) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) zero_row_chunk(TB + kTile, row, q);
     }
-    if ((warp & 3) >= 2) {
-      // lower-left block: -Z'
-      const int i = (warp & 3) * 32 + lane, half = warp >> 2;
-      float v[32];
-      tmem_ld32(tmem_at(tmem, (warp & 3) * 32, kColZ + half * 32), v);
-      tmem_ld_wait();
+  }
+  if (quarter >= 2) {
+    // lower-left block: -Z'
+    const int i = quarter * 32 + lane, half = wg;
+    float v[32];
+    tmem_ld32(lane_addr + kColZ + half * 32, v);
+    tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = -v[e];
+    for (int e = 0; e < 32; ++e) v[e] = -v[e];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) st_row8_bf16(TB, kTile, i, half * 4 + q, v + 8 * q);
-    }
-    {
-      // K^ rows: thread pair per row, 8 chunks each; the swizzled position is the same
-      const int row = tid >> 1, part = tid & 1;
-      const float gam = __expf(Gr[row]);
+    for (int q = 0; q < 4; ++q) st_row8_bf16(sm + kPrepR1, kTile, i, half * 4 + q, v + 8 * q);
+  }
+  {
+    // K^ = diag(e^G) K in place: thread pair per row, 8 chunks each
+    const int row = tid >> 1, part = tid & 1;
+    const float gam = __expf(G_s[row]);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int chunk16 = part * 8 + q;
-        const uint32_t off = (chunk16 >> 3) * kTile + sw128_off(row, chunk16 & 7);
-        uint4 u = *reinterpret_cast<const uint4*>(sm + kPrepKs + off);
-        __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
+    for (int q = 0; q < 8; ++q) {
+      const int chunk16 = part * 8 + q;
+      const uint32_t off = (chunk16 >> 3) * kTile + sw128_off(row, chunk16 & 7);
+      uint4 u = *reinterpret_cast<const uint4*>(sm + kPrepKs + off);
+      __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float2 f = __bfloat1622float2(hv[e]);
-          hv[e] = __floats2bfloat162_rn(f.x * gam, f.y * gam);
-        }
-        *reinterpret_cast<uint4*>(Kh + off) = u;
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hv[e]);
+        hv[e] = __floats2bfloat162_rn(f.x * gam, f.y * gam);
       }
+      *reinterpret_cast<uint4*>(sm + kPrepKs + off) = u;
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- W = T diag(beta) K^,  U~ = T diag(beta) V
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sTB = smem_u32(TB), sK = smem_u32(Kh),
-                     sV = smem_u32(sm + (r == 0 ? kPrepV0 : kPrepV1));
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---- W = T diag(beta) K^,  U~ = T diag(beta) V
+  if (tid == 0) {
+    ok = mbar_wait(bar_v, 0);
+    tc_fence_after();
+    if (ok) {
+      const uint32_t sTB = smem_u32(sm + kPrepR1), sK = smem_u32(sm + kPrepKs),
+                     sV = smem_u32(sm + kPrepR2);
+      constexpr uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        mma_bf16(tmem + kColW, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sK, kk, kTile),
-                 idesc_bf16(128, 128, false, true), kk > 0);
-        mma_bf16(tmem + kColU, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sV, kk, kTile),
-                 idesc_bf16(128, 128, false, true), kk > 0);
+        mma_bf16(tmem + kColW, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sK, kk, kTile), id, kk > 0);
+        mma_bf16(tmem + kColU, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sV, kk, kTile), id, kk > 0);
       }
       mma_commit(bar);
     }
-    ok = mbar_wait(bar, phase);
-    phase ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
-    tc_fence_after();
-    // ---- W, U~ -> workspace (bf16 row-major)
-    {
-      const int i = (warp & 3) * 32 + lane, half = warp >> 2;
-      const size_t base = (((size_t)c * Hv + h) * kC + i) * kD + half * 64;
+  }
+  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(bar, phase);
+  phase ^= 1;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  // ---- W, U~ -> workspace (bf16 row-major; U~ replaces V): thread row i, column half wg
+  {
+    const int i = quarter * 32 + lane, half = wg;
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        __nv_bfloat16* dst = (m == 0 ? a.ws.Ww : a.ws.Uw) + base;
-        const uint32_t col = (m == 0 ? kColW : kColU) + half * 64;
+    for (int m = 0; m < 2; ++m) {
+      __nv_bfloat16* dst = (m == 0 ? a.ws.Ww : a.ws.Uw) +
+                           (((size_t)c * Hv + h) * kC + i) * kD + half * 64;
+      const uint32_t col = (m == 0 ? kColW : kColU) + half * 64;
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          float v[32];
-          tmem_ld32(tmem_at(tmem, (warp & 3) * 32, col + cc * 32), v);
-          tmem_ld_wait();
+      for (int cc = 0; cc < 2; ++cc) {
+        float v[32];
+        tmem_ld32(lane_addr + col + cc * 32, v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float w8[8];
+        for (int q = 0; q < 4; ++q) {
+          float w8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = v[8 * q + e];
-            store8(dst + cc * 32 + 8 * q, w8);
-          }
+          for (int e = 0; e < 8; ++e) w8[e] = v[8 * q + e];
+          store8(dst + cc * 32 + 8 * q, w8);
         }
       }
     }
-    tc_fence_before();
-    __syncthreads();
   }
 done:
   if (tid == 0 && !ok) report_status(a.status, GDN_ERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(*tslot, 512);
+  if (warp == 0) tmem_dealloc(*tslot, 256);
 }
 
 // --------------------------------------------------------------------------------- chain
@@ -542,24 +632,28 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
   int failed = 0;
   uint8_t* SB = sm + Cfg::kSB;
   uint8_t* UB = sm + Cfg::kUB;
+  // per-token inputs of a chunk (row = tid): U~ slice (packed bf16), G_i, G_last
+  constexpr int kVec = DV / 8;
+  uint4 ut_cur[kVec], ut_nxt[kVec];
+  float Gi_cur = 0.f, Gl_cur = 0.f, Gi_nxt = 0.f, Gl_nxt = 0.f;
+  auto load_chunk_rows = [&](int ci, uint4 (&ut)[kVec], float& Gi, float& Gl) {
+    const int c = first + ci;
+    const float* Gc = a.ws.Gw + ((size_t)c * a.Hv + h) * kC;
+    Gi = Gc[tid];
+    Gl = Gc[kC - 1];
+    const uint4* src = reinterpret_cast<const uint4*>(
+        a.ws.Uw + (((size_t)c * a.Hv + h) * kC + tid) * kD + v0);
+#pragma unroll
+    for (int q = 0; q < kVec; ++q) ut[q] = src[q];
+  };
+  if (nch > 0) load_chunk_rows(0, ut_cur, Gi_cur, Gl_cur);
   for (int ci = 0; ci < nch; ++ci) {
     const int c = first + ci, stage = ci & 1;
     if (tid == 0 && ci + 1 < nch) issue_tma(ci + 1, stage ^ 1);
-    // per-token inputs of this chunk (row i = tid)
-    const float* Gc = a.ws.Gw + ((size_t)c * a.Hv + h) * kC;
-    const float Gi = Gc[tid], Glast = Gc[kC - 1];
     __nv_bfloat16* Urow = a.ws.Uw + (((size_t)c * a.Hv + h) * kC + tid) * kD + v0;
-    float ut[DV];
-#pragma unroll
-    for (int q = 0; q < DV / 8; ++q) {
-      float t8[8];
-      load8(Urow + 8 * q, t8);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ut[8 * q + e] = t8[e];
-    }
     // ---- S_b (bf16) -> SB operand and workspace; S^T *= e^(G_last)
     {
-      const float gam = __expf(Glast);
+      const float gam = __expf(Gl_cur);
       __nv_bfloat16* Srow = a.ws.Sw + (((size_t)c * a.Hv + h) * kD + k_row) * kD + v0;
 #pragma unroll
       for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
@@ -600,13 +694,15 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
       }
     }
     if ((failed = __syncthreads_or(!ok))) break;
+    // next chunk's rows travel while the MMA runs
+    if (ci + 1 < nch) load_chunk_rows(ci + 1, ut_nxt, Gi_nxt, Gl_nxt);
     ok = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1;
     if ((failed = __syncthreads_or(!ok))) break;
     tc_fence_after();
     // ---- U = U~ - X -> workspace; U^ = diag(e^(G_L - G)) U -> UB operand
     {
-      const float dec = __expf(Glast - Gi);
+      const float dec = __expf(Gl_cur - Gi_cur);
 #pragma unroll
       for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
         float v[32];
@@ -615,14 +711,19 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           if (cc * 32 + 8 * q < DV) {
+            const int vq = (cc * 32 + 8 * q) >> 3;
+            const __nv_bfloat162* uh = reinterpret_cast<const __nv_bfloat162*>(&ut_cur[vq]);
             float u8[8], h8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              u8[e] = ut[cc * 32 + 8 * q + e] - v[8 * q + e];
-              h8[e] = u8[e] * dec;
+            for (int e2 = 0; e2 < 4; ++e2) {
+              const float2 f = __bfloat1622float2(uh[e2]);
+              u8[2 * e2] = f.x - v[8 * q + 2 * e2];
+              u8[2 * e2 + 1] = f.y - v[8 * q + 2 * e2 + 1];
             }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) h8[e] = u8[e] * dec;
             store8(Urow + cc * 32 + 8 * q, u8);
-            st_row8_bf16(UB, kTile, tid, (cc * 32 + 8 * q) >> 3, h8);
+            st_row8_bf16(UB, kTile, tid, vq, h8);
           }
         }
       }
@@ -644,6 +745,10 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
     mma_phase ^= 1;
     if ((failed = __syncthreads_or(!ok))) break;
     tc_fence_after();
+#pragma unroll
+    for (int q = 0; q < kVec; ++q) ut_cur[q] = ut_nxt[q];
+    Gi_cur = Gi_nxt;
+    Gl_cur = Gl_nxt;
   }
   if (!failed && a.SN) {
     const size_t sbase = ((size_t)n * a.Hv + h) * kD * kD;
@@ -664,16 +769,20 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
 }
 
 // ----------------------------------------------------------------------------------- out
-constexpr uint32_t kOutQ = 0, kOutK = 32768, kOutS = 65536, kOutU = 98304, kOutP = 131072;
-constexpr uint32_t kOutEnd = 163840;
-constexpr uint32_t kOutSmem = kOutEnd + 1024 + 1024;
+// One CTA per (chunk, key head), 8 warps.  Warp w reads TMEM lanes 32*(w%4).. (token rows) and
+// handles the column half w/4 of every 128-wide row, so each thread owns 64 values of a row.
+// P of both value heads is built from one Q K^T; S^T and U of the second value head are loaded
+// by TMA while the first head's epilogue runs; z is prefetched into registers.
+constexpr uint32_t kOutQ = 0, kOutK = 32768, kOutS = 65536, kOutU = 98304, kOutP0 = 131072,
+                   kOutP1 = 163840;
+constexpr uint32_t kOutEnd = 196608;
+constexpr uint32_t kOutSmem = kOutEnd + 1024 + 4096;
 constexpr uint32_t kColQK = 0, kColYo = 128, kColPU = 256;
+constexpr int kOutThreads = 256;
 
-__global__ void __launch_bounds__(128, 1) gdn_out_kernel(PrefillArgs a,
-                                                         const __grid_constant__ CUtensorMap mapQ,
-                                                         const __grid_constant__ CUtensorMap mapK,
-                                                         const __grid_constant__ CUtensorMap mapS,
-                                                         const __grid_constant__ CUtensorMap mapU) {
+__global__ void __launch_bounds__(kOutThreads, 1) gdn_out_kernel(
+    PrefillArgs a, const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+    const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapU) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
@@ -681,13 +790,18 @@ __global__ void __launch_bounds__(128, 1) gdn_out_kernel(PrefillArgs a,
   uint64_t* bar_su = bar_qk + 1;
   uint64_t* bar_mma = bar_qk + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_qk + 3);
-  float* G_s = reinterpret_cast<float*>(sm + kOutEnd + 64);   // [128]
+  float* G_s = reinterpret_cast<float*>(sm + kOutEnd + 64);   // [2][128]
+  float* red_s = G_s + 2 * kC;                                // [2][128] partial sums of squares
+  float* w_s = red_s + 2 * kC;                                // [128] norm weight
 
   const int c = blockIdx.x, hk = blockIdx.y;
   const int total_chunks = a.ws.seq_first[a.N];
   if (c >= total_chunks) return;
   const ChunkInfo ci = a.ws.chunks[c];
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int i = quarter * 32 + lane;  // token row of this thread
+  const bool valid = i < ci.L;
   const int Hv = a.Hv;
   if (tid == 0) {
     mbar_init(bar_qk, 1);
@@ -696,10 +810,6 @@ __global__ void __launch_bounds__(128, 1) gdn_out_kernel(PrefillArgs a,
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(tslot, 512);
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tslot;
-  const uint32_t lane_addr = tmem_at(tmem, warp * 32, 0);
   auto load_su = [&](int r) {
     const int row = ((c * Hv) + hk * 2 + r) * kC;
     mbar_arrive_expect_tx(bar_su, 4 * kTile);
@@ -717,8 +827,26 @@ __global__ void __launch_bounds__(128, 1) gdn_out_kernel(PrefillArgs a,
     tma_load_2d(sm + kOutK + kTile, &mapK, bar_qk, 64, row);
     load_su(0);
   }
+  // gates of both value heads, norm weight
+  G_s[tid] = a.ws.Gw[((size_t)c * Hv + hk * 2 + (tid >> 7)) * kC + (tid & 127)];
+  if (tid < kD) w_s[tid] = a.norm_w ? __bfloat162float(a.norm_w[tid]) : 1.f;
+  // z of the first value head: this thread's 64 values, prefetched
+  uint4 zreg[8];
+  auto load_z = [&](int r) {
+    if (a.z && valid) {
+      const uint4* zp = reinterpret_cast<const uint4*>(
+          a.z + ((size_t)(ci.t0 + i) * Hv + hk * 2 + r) * kD + half * 64);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) zreg[q] = __ldg(zp + q);
+    }
+  };
+  load_z(0);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t lane_addr = tmem_at(tmem, quarter * 32, 0);
   const uint32_t sQ = smem_u32(sm + kOutQ), sK = smem_u32(sm + kOutK),
-                 sS = smem_u32(sm + kOutS), sU = smem_u32(sm + kOutU), sP = smem_u32(sm + kOutP);
+                 sS = smem_u32(sm + kOutS), sU = smem_u32(sm + kOutU);
   bool ok = true;
   uint32_t mma_phase = 0;
   if (tid == 0) {
@@ -737,34 +865,43 @@ __global__ void __launch_bounds__(128, 1) gdn_out_kernel(PrefillArgs a,
   mma_phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  for (int r = 0; r < 2; ++r) {
-    const int h = hk * 2 + r;
-    const int i = tid;
-    G_s[i] = a.ws.Gw[((size_t)c * Hv + h) * kC + i];
-    __syncthreads();
-    const float Gi = G_s[i];
-    // ---- P (bf16, K-major) from Q K^T
+  // ---- P_r = mask(e^(G_i - G_j)) * (Q K^T), both value heads, bf16 K-major
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      float v[32];
-      tmem_ld32(lane_addr + kColQK + cc * 32, v);
+  for (int cc = 0; cc < 2; ++cc) {
+    const int j0 = half * 64 + cc * 32;
+    // warp-uniform: every row of this warp is above the chunk (all of P is masked there)
+    const bool any_lower = j0 <= quarter * 32 + 31;
+    float v[32];
+    if (any_lower) {
+      tmem_ld32(lane_addr + kColQK + j0, v);
       tmem_ld_wait();
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const float* Gr = G_s + r * kC;
+      const float Gi = Gr[i];
+      float p[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const int j = cc * 32 + e;
-        v[e] = (j <= i) ? __expf(Gi - G_s[j]) * v[e] : 0.f;
+        const int j = j0 + e;
+        p[e] = (any_lower && j <= i) ? __expf(Gi - Gr[j]) * v[e] : 0.f;
       }
+      uint8_t* P = sm + (r == 0 ? kOutP0 : kOutP1);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) st_row8_bf16(sm + kOutP, kTile, i, cc * 4 + q, v + 8 * q);
+      for (int q = 0; q < 4; ++q) st_row8_bf16(P, kTile, i, half * 8 + cc * 4 + q, p + 8 * q);
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  for (int r = 0; r < 2; ++r) {
+    const int h = hk * 2 + r;
     // ---- Y = Q S^T ; O_intra = P U
     if (tid == 0) {
       ok = mbar_wait(bar_su, r & 1);
       tc_fence_after();
       if (ok) {
+        const uint32_t sP = smem_u32(sm + (r == 0 ? kOutP0 : kOutP1));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           mma_bf16(tmem + kColYo, desc_kmajor(sQ, kk, kTile), desc_mnmajor(sS, kk, kTile),
@@ -782,50 +919,47 @@ __global__ void __launch_bounds__(128, 1) gdn_out_kernel(PrefillArgs a,
     tc_fence_after();
     if (tid == 0 && r == 0) load_su(1);  // S and U buffers are free again
     // ---- epilogue: o = e^G Y + P U, gated RMSNorm, bf16 out
-    const float eg = __expf(Gi);
-    const bool valid = i < ci.L;
-    const size_t orow = ((size_t)(ci.t0 + i) * Hv + h) * kD;
-    float inv = 1.f;
+    const float eg = __expf(G_s[r * kC + i]);
+    float o[64];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      float y[32], pu[32];
+      tmem_ld32(lane_addr + kColYo + half * 64 + cc * 32, y);
+      tmem_ld32(lane_addr + kColPU + half * 64 + cc * 32, pu);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[cc * 32 + e] = eg * y[e] + pu[e];
+    }
     if (a.z) {
       float ss = 0.f;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float y[32], p[32];
-        tmem_ld32(lane_addr + kColYo + cc * 32, y);
-        tmem_ld32(lane_addr + kColPU + cc * 32, p);
-        tmem_ld_wait();
+      for (int e = 0; e < 64; ++e) ss += o[e] * o[e];
+      red_s[half * kC + i] = ss;
+      __syncthreads();
+      const float inv = rsqrtf((red_s[i] + red_s[kC + i]) / kD + a.norm_eps);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float o = eg * y[e] + p[e];
-          ss += o * o;
-        }
-      }
-      inv = rsqrtf(ss / kD + a.norm_eps);
-    }
+      for (int q = 0; q < 8; ++q) {
+        const __nv_bfloat162* zh = reinterpret_cast<const __nv_bfloat162*>(&zreg[q]);
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      float y[32], p[32];
-      tmem_ld32(lane_addr + kColYo + cc * 32, y);
-      tmem_ld32(lane_addr + kColPU + cc * 32, p);
-      tmem_ld_wait();
-      if (valid) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float o8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o8[e] = eg * y[8 * q + e] + p[8 * q + e];
-          if (a.z) {
-            float z8[8], w8[8];
-            load8(a.z + orow + cc * 32 + 8 * q, z8);
-            if (a.norm_w) load8(a.norm_w + cc * 32 + 8 * q, w8);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              o8[e] = o8[e] * inv * (a.norm_w ? w8[e] : 1.f) * (z8[e] / (1.f + __expf(-z8[e])));
-          }
-          store8(a.out + orow + cc * 32 + 8 * q, o8);
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float2 zf = __bfloat1622float2(zh[e2]);
+          const int e = q * 8 + e2 * 2;
+          o[e] = o[e] * inv * w_s[half * 64 + e] * silu_fast(zf.x);
+          o[e + 1] = o[e + 1] * inv * w_s[half * 64 + e + 1] * silu_fast(zf.y);
         }
       }
     }
+    if (valid) {
+      __nv_bfloat16* dst = a.out + ((size_t)(ci.t0 + i) * Hv + h) * kD + half * 64;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float o8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o8[e] = o[q * 8 + e];
+        store8(dst + q * 8, o8);
+      }
+    }
+    if (r == 0) load_z(1);
     tc_fence_before();
     __syncthreads();
   }
@@ -954,8 +1088,12 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const dim3 grid_chunks((unsigned)(a.T / kC + a.N), a.Hk);
   if (a.T > 0) {
+    trace_begin("gdn_qkv", s);
+    gdn::gdn_qkv_kernel<<<dim3(grid_chunks.x, 2 * a.Hk + a.Hv), 128, 0, s>>>(a);
+    trace_end(s);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     trace_begin("gdn_prep", s);
-    gdn::gdn_prep_kernel<<<grid_chunks, 256, gdn::kPrepSmem, s>>>(a);
+    gdn::gdn_prep_kernel<<<dim3(grid_chunks.x, a.Hv), 256, gdn::kPrepSmem, s>>>(a, mK, mU);
     trace_end(s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -967,7 +1105,7 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   if (e != cudaSuccess) return e;
   if (a.T > 0) {
     trace_begin("gdn_out", s);
-    gdn::gdn_out_kernel<<<grid_chunks, 128, gdn::kOutSmem, s>>>(a, mQ, mK, mS, mU);
+    gdn::gdn_out_kernel<<<grid_chunks, gdn::kOutThreads, gdn::kOutSmem, s>>>(a, mQ, mK, mS, mU);
     trace_end(s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
