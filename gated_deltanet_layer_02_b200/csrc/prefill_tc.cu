@@ -769,32 +769,44 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
 }
 
 // ----------------------------------------------------------------------------------- out
-// One CTA per (chunk, key head), 8 warps.  Warp w reads TMEM lanes 32*(w%4).. (token rows) and
-// handles the column half w/4 of every 128-wide row, so each thread owns 64 values of a row.
-// P of both value heads is built from one Q K^T; S^T and U of the second value head are loaded
-// by TMA while the first head's epilogue runs; z is prefetched into registers.
-constexpr uint32_t kOutQ = 0, kOutK = 32768, kOutS = 65536, kOutU = 98304, kOutP0 = 131072,
-                   kOutP1 = 163840;
-constexpr uint32_t kOutEnd = 196608;
+// One CTA per (chunk, value head), 8 warps, two CTAs per SM.  Warp w reads TMEM lanes
+// 32*(w%4).. (token rows) and handles the column half w/4 of each 128-wide row.
+//   Q K^T (tcgen05, both operands from smem) -> P = mask(e^(G_i - G_j)) * Q K^T and
+//   Q^ = diag(e^G) Q, both written to TMEM as bf16 A operands -> O = Q^ S^T + P U accumulated
+//   in one TMEM region (A from TMEM, B from smem) -> z-gated RMSNorm -> bf16 output.
+// S^T is loaded into K's buffer once the gram has consumed K.
+constexpr uint32_t kOutQ = 0, kOutKS = 32768, kOutU = 65536;
+constexpr uint32_t kOutEnd = 98304;
 constexpr uint32_t kOutSmem = kOutEnd + 1024 + 4096;
-constexpr uint32_t kColQK = 0, kColYo = 128, kColPU = 256;
+constexpr uint32_t kColQK = 0, kColP = 0, kColQh = 64, kColO = 128;  // 256 TMEM columns
 constexpr int kOutThreads = 256;
 
-__global__ void __launch_bounds__(kOutThreads, 1) gdn_out_kernel(
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
     PrefillArgs a, const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
     const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapU) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bar_qk = reinterpret_cast<uint64_t*>(sm + kOutEnd);
-  uint64_t* bar_su = bar_qk + 1;
-  uint64_t* bar_mma = bar_qk + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_qk + 3);
-  float* G_s = reinterpret_cast<float*>(sm + kOutEnd + 64);   // [2][128]
-  float* red_s = G_s + 2 * kC;                                // [2][128] partial sums of squares
+  uint64_t* bar_s = bar_qk + 1;
+  uint64_t* bar_u = bar_qk + 2;
+  uint64_t* bar_mma = bar_qk + 3;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_qk + 4);
+  float* G_s = reinterpret_cast<float*>(sm + kOutEnd + 64);   // [128]
+  float* red_s = G_s + kC;                                    // [2][128] partial sums of squares
   float* w_s = red_s + 2 * kC;                                // [128] norm weight
 
-  const int c = blockIdx.x, hk = blockIdx.y;
+  const int c = blockIdx.x, h = blockIdx.y;
   const int total_chunks = a.ws.seq_first[a.N];
   if (c >= total_chunks) return;
   const ChunkInfo ci = a.ws.chunks[c];
@@ -803,59 +815,48 @@ __global__ void __launch_bounds__(kOutThreads, 1) gdn_out_kernel(
   const int i = quarter * 32 + lane;  // token row of this thread
   const bool valid = i < ci.L;
   const int Hv = a.Hv;
+  const int hk = h / (Hv / a.Hk);
   if (tid == 0) {
     mbar_init(bar_qk, 1);
-    mbar_init(bar_su, 1);
+    mbar_init(bar_s, 1);
+    mbar_init(bar_u, 1);
     mbar_init(bar_mma, 1);
     fence_barrier_init();
-  }
-  if (warp == 0) tmem_alloc(tslot, 512);
-  auto load_su = [&](int r) {
-    const int row = ((c * Hv) + hk * 2 + r) * kC;
-    mbar_arrive_expect_tx(bar_su, 4 * kTile);
-    tma_load_2d(sm + kOutS, &mapS, bar_su, 0, row);
-    tma_load_2d(sm + kOutS + kTile, &mapS, bar_su, 64, row);
-    tma_load_2d(sm + kOutU, &mapU, bar_su, 0, row);
-    tma_load_2d(sm + kOutU + kTile, &mapU, bar_su, 64, row);
-  };
-  if (tid == 0) {
-    const int row = (c * a.Hk + hk) * kC;
+    const int rowQK = (c * a.Hk + hk) * kC, rowV = (c * Hv + h) * kC;
     mbar_arrive_expect_tx(bar_qk, 4 * kTile);
-    tma_load_2d(sm + kOutQ, &mapQ, bar_qk, 0, row);
-    tma_load_2d(sm + kOutQ + kTile, &mapQ, bar_qk, 64, row);
-    tma_load_2d(sm + kOutK, &mapK, bar_qk, 0, row);
-    tma_load_2d(sm + kOutK + kTile, &mapK, bar_qk, 64, row);
-    load_su(0);
+    tma_load_2d(sm + kOutQ, &mapQ, bar_qk, 0, rowQK);
+    tma_load_2d(sm + kOutQ + kTile, &mapQ, bar_qk, 64, rowQK);
+    tma_load_2d(sm + kOutKS, &mapK, bar_qk, 0, rowQK);
+    tma_load_2d(sm + kOutKS + kTile, &mapK, bar_qk, 64, rowQK);
+    mbar_arrive_expect_tx(bar_u, 2 * kTile);
+    tma_load_2d(sm + kOutU, &mapU, bar_u, 0, rowV);
+    tma_load_2d(sm + kOutU + kTile, &mapU, bar_u, 64, rowV);
   }
-  // gates of both value heads, norm weight
-  G_s[tid] = a.ws.Gw[((size_t)c * Hv + hk * 2 + (tid >> 7)) * kC + (tid & 127)];
-  if (tid < kD) w_s[tid] = a.norm_w ? __bfloat162float(a.norm_w[tid]) : 1.f;
-  // z of the first value head: this thread's 64 values, prefetched
+  if (warp == 0) tmem_alloc(tslot, 256);
+  if (tid < kC) G_s[tid] = a.ws.Gw[((size_t)c * Hv + h) * kC + tid];
+  else w_s[tid - kC] = a.norm_w ? __bfloat162float(a.norm_w[tid - kC]) : 1.f;
   uint4 zreg[8];
-  auto load_z = [&](int r) {
-    if (a.z && valid) {
-      const uint4* zp = reinterpret_cast<const uint4*>(
-          a.z + ((size_t)(ci.t0 + i) * Hv + hk * 2 + r) * kD + half * 64);
+  if (a.z && valid) {
+    const uint4* zp = reinterpret_cast<const uint4*>(a.z + ((size_t)(ci.t0 + i) * Hv + h) * kD +
+                                                     half * 64);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) zreg[q] = __ldg(zp + q);
-    }
-  };
-  load_z(0);
+    for (int q = 0; q < 8; ++q) zreg[q] = __ldg(zp + q);
+  }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t lane_addr = tmem_at(tmem, quarter * 32, 0);
-  const uint32_t sQ = smem_u32(sm + kOutQ), sK = smem_u32(sm + kOutK),
-                 sS = smem_u32(sm + kOutS), sU = smem_u32(sm + kOutU);
+  const uint32_t sQ = smem_u32(sm + kOutQ), sKS = smem_u32(sm + kOutKS), sU = smem_u32(sm + kOutU);
   bool ok = true;
   uint32_t mma_phase = 0;
+  // ---- Q K^T
   if (tid == 0) {
     ok = mbar_wait(bar_qk, 0);
     tc_fence_after();
     if (ok) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + kColQK, desc_kmajor(sQ, kk, kTile), desc_kmajor(sK, kk, kTile),
+        mma_bf16(tmem + kColQK, desc_kmajor(sQ, kk, kTile), desc_kmajor(sKS, kk, kTile),
                  idesc_bf16(128, 128, false, false), kk > 0);
       mma_commit(bar_mma);
     }
@@ -865,70 +866,86 @@ __global__ void __launch_bounds__(kOutThreads, 1) gdn_out_kernel(
   mma_phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  // ---- P_r = mask(e^(G_i - G_j)) * (Q K^T), both value heads, bf16 K-major
-#pragma unroll
-  for (int cc = 0; cc < 2; ++cc) {
-    const int j0 = half * 64 + cc * 32;
-    // warp-uniform: every row of this warp is above the chunk (all of P is masked there)
-    const bool any_lower = j0 <= quarter * 32 + 31;
-    float v[32];
-    if (any_lower) {
-      tmem_ld32(lane_addr + kColQK + j0, v);
-      tmem_ld_wait();
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const float* Gr = G_s + r * kC;
-      const float Gi = Gr[i];
-      float p[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int j = j0 + e;
-        p[e] = (any_lower && j <= i) ? __expf(Gi - Gr[j]) * v[e] : 0.f;
-      }
-      uint8_t* P = sm + (r == 0 ? kOutP0 : kOutP1);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) st_row8_bf16(P, kTile, i, half * 8 + cc * 4 + q, p + 8 * q);
-    }
+  if (tid == 0) {  // K is consumed: S^T of this chunk and value head into the same buffer
+    const int rowS = (c * Hv + h) * kC;
+    mbar_arrive_expect_tx(bar_s, 2 * kTile);
+    tma_load_2d(sm + kOutKS, &mapS, bar_s, 0, rowS);
+    tma_load_2d(sm + kOutKS + kTile, &mapS, bar_s, 64, rowS);
   }
-  fence_proxy_async_smem();
+  {
+    // ---- P row half and Q^ row half, packed bf16 pairs in registers
+    const float Gi = G_s[i];
+    uint32_t pp[32], qq[32];
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int j0 = half * 64 + cc * 32;
+      const bool any_lower = j0 <= quarter * 32 + 31;  // warp-uniform
+      float v[32];
+      if (any_lower) {
+        tmem_ld32(lane_addr + kColQK + j0, v);
+        tmem_ld_wait();
+      }
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const int j = j0 + e;
+        const float p0 = (any_lower && j <= i) ? __expf(Gi - G_s[j]) * v[e] : 0.f;
+        const float p1 = (any_lower && j + 1 <= i) ? __expf(Gi - G_s[j + 1]) * v[e + 1] : 0.f;
+        pp[cc * 16 + e / 2] = pack_bf16x2(p0, p1);
+      }
+    }
+    const float eg = __expf(Gi);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int chunk16 = half * 8 + q;
+      const uint4 u = *reinterpret_cast<const uint4*>(sm + kOutQ + (chunk16 >> 3) * kTile +
+                                                      sw128_off(i, chunk16 & 7));
+      const __nv_bfloat162* hq = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hq[e]);
+        qq[q * 4 + e] = pack_bf16x2(f.x * eg, f.y * eg);
+      }
+    }
+    // every thread has read its gram columns: the gram region may now take P and Q^
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    tmem_st32(lane_addr + kColP + half * 32, *reinterpret_cast<float(*)[32]>(pp));
+    tmem_st32(lane_addr + kColQh + half * 32, *reinterpret_cast<float(*)[32]>(qq));
+    tmem_st_wait();
+  }
   tc_fence_before();
   __syncthreads();
-  for (int r = 0; r < 2; ++r) {
-    const int h = hk * 2 + r;
-    // ---- Y = Q S^T ; O_intra = P U
-    if (tid == 0) {
-      ok = mbar_wait(bar_su, r & 1);
-      tc_fence_after();
-      if (ok) {
-        const uint32_t sP = smem_u32(sm + (r == 0 ? kOutP0 : kOutP1));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          mma_bf16(tmem + kColYo, desc_kmajor(sQ, kk, kTile), desc_mnmajor(sS, kk, kTile),
-                   idesc_bf16(128, 128, false, true), kk > 0);
-          mma_bf16(tmem + kColPU, desc_kmajor(sP, kk, kTile), desc_mnmajor(sU, kk, kTile),
-                   idesc_bf16(128, 128, false, true), kk > 0);
-        }
-        mma_commit(bar_mma);
-      }
-    }
-    if (__syncthreads_or(!ok)) goto done;
-    ok = mbar_wait(bar_mma, mma_phase);
-    mma_phase ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
+  // ---- O = Q^ S^T + P U   (A operands from TMEM)
+  if (tid == 0) {
+    ok = mbar_wait(bar_s, 0) && mbar_wait(bar_u, 0);
     tc_fence_after();
-    if (tid == 0 && r == 0) load_su(1);  // S and U buffers are free again
-    // ---- epilogue: o = e^G Y + P U, gated RMSNorm, bf16 out
-    const float eg = __expf(G_s[r * kC + i]);
+    if (ok) {
+      constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ts(tmem + kColO, tmem + kColQh + kk * 8, desc_mnmajor(sKS, kk, kTile), id, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, desc_mnmajor(sU, kk, kTile), id, 1);
+      mma_commit(bar_mma);
+    }
+  }
+  if (__syncthreads_or(!ok)) goto done;
+  ok = mbar_wait(bar_mma, mma_phase);
+  mma_phase ^= 1;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  {
+    // ---- epilogue: gated RMSNorm, bf16 out
     float o[64];
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
-      float y[32], pu[32];
-      tmem_ld32(lane_addr + kColYo + half * 64 + cc * 32, y);
-      tmem_ld32(lane_addr + kColPU + half * 64 + cc * 32, pu);
+      float y[32];
+      tmem_ld32(lane_addr + kColO + half * 64 + cc * 32, y);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) o[cc * 32 + e] = eg * y[e] + pu[e];
+      for (int e = 0; e < 32; ++e) o[cc * 32 + e] = y[e];
     }
     if (a.z) {
       float ss = 0.f;
@@ -959,15 +976,12 @@ __global__ void __launch_bounds__(kOutThreads, 1) gdn_out_kernel(
         store8(dst + q * 8, o8);
       }
     }
-    if (r == 0) load_z(1);
-    tc_fence_before();
-    __syncthreads();
   }
 done:
   if (tid == 0 && !ok) report_status(a.status, GDN_ERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 512);
+  if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 }  // namespace gdn
@@ -1105,7 +1119,8 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   if (e != cudaSuccess) return e;
   if (a.T > 0) {
     trace_begin("gdn_out", s);
-    gdn::gdn_out_kernel<<<grid_chunks, gdn::kOutThreads, gdn::kOutSmem, s>>>(a, mQ, mK, mS, mU);
+    gdn::gdn_out_kernel<<<dim3(grid_chunks.x, a.Hv), gdn::kOutThreads, gdn::kOutSmem, s>>>(
+        a, mQ, mK, mS, mU);
     trace_end(s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
