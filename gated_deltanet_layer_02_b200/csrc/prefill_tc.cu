@@ -76,11 +76,6 @@ __global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Wor
 
 
 // --------------------------------------------------------------------------------- q/k/v
-// One CTA per (chunk, 128-channel group of the conv input): causal conv (width 4) + SiLU, and
-// for q and k the L2 norm of every (token, head) row.  128 threads: 16 column vectors x 8 runs
-// of 16 tokens; the 16 threads of a row share a half-warp, so the norm is a 4-step shuffle.
-// Outputs are bf16 [128][128] tiles per (chunk, head): Q -> Qw, K -> Kw, V -> Uw (V is read by
-// gdn_prep, which overwrites the same tile with U~).  Rows past the chunk's length are zero.
 __device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -101,8 +96,25 @@ __device__ __forceinline__ float silu_fast(float x) {
   return fmaf(h, tanh_approx(h), h);
 }
 
-__global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a) {
-  const int c = blockIdx.x, grp = blockIdx.y;
+// One CTA per (chunk, 128-channel group of the conv input): causal conv (width 4) + SiLU, and
+// for q and k the L2 norm of every (token, head) row.  The chunk's input rows, with the 3
+// preceding rows, arrive by TMA as two [131][64] boxes (128-byte swizzle); for the first chunk
+// of a sequence the 3 preceding rows are replaced by the caller's conv state (or zeros).
+// 128 threads: 16 column vectors x 8 runs of 16 tokens; the 16 threads of a row share a
+// half-warp, so the norm is a 4-step shuffle.  Outputs are bf16 [128][128] tiles per (chunk,
+// head): Q -> Qw, K -> Kw, V -> Uw (read by gdn_prep, which overwrites it with U~).  Rows past
+// the chunk's length are written as zeros.
+constexpr int kXRows = kC + 3;
+constexpr uint32_t kXBox = 17408;  // one [131][64] bf16 box, rounded up to 1024 bytes
+constexpr uint32_t kQkvSmem = 2 * kXBox + 1024 + 64;
+
+__global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
+                                                         const __grid_constant__ CUtensorMap mapX) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 2 * kXBox);
+  const int grp = blockIdx.x, c = blockIdx.y;
   if (c >= a.ws.seq_first[a.N]) return;
   const ChunkInfo ci = a.ws.chunks[c];
   const int tid = threadIdx.x, vec = tid & 15, run = tid >> 4;
@@ -111,10 +123,18 @@ __global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a) {
   const int kind = grp < Hk ? 0 : (grp < 2 * Hk ? 1 : 2);
   const int head = kind == 0 ? grp : (kind == 1 ? grp - Hk : grp - 2 * Hk);
   const int ch = grp * kD + vec * 8;
+  const int seq_start = __ldg(a.cu + ci.n);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(bar, 2 * kXRows * 128);
+    tma_load_2d(sm, &mapX, bar, grp * kD, ci.t0 - 3);
+    tma_load_2d(sm + kXBox, &mapX, bar, grp * kD + 64, ci.t0 - 3);
+  }
+  __syncthreads();  // the barrier is initialised before any thread waits on it
   __nv_bfloat16* dst = (kind == 0 ? a.ws.Qw + ((size_t)c * Hk + head) * kC * kD
                       : kind == 1 ? a.ws.Kw + ((size_t)c * Hk + head) * kC * kD
                                   : a.ws.Uw + ((size_t)c * Hv + head) * kC * kD) + vec * 8;
-  const int seq_start = __ldg(a.cu + ci.n);
   float2 wv[4][4];  // taps x channel pairs
   if (a.conv_w) {
 #pragma unroll
@@ -129,76 +149,72 @@ __global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a) {
       }
     }
   }
+  uint8_t* box = sm + (vec >> 3) * kXBox;
+  const uint32_t chunk = vec & 7;
+  auto row_ptr = [&](int r) { return reinterpret_cast<uint4*>(box + sw128_off(r, chunk)); };
+  const bool ok = mbar_wait(bar, 0);
+  if (!ok) {
+    if (tid == 0) report_status(a.status, GDN_ERR_TIMEOUT);
+    return;
+  }
+  // first chunk of a sequence: the 3 rows before it come from the conv state (or are zero)
+  if (ci.t0 == seq_start && run == 0) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (a.conv0) v = *reinterpret_cast<const uint4*>(a.conv0 + ((size_t)ci.n * 3 + j) * Cc + ch);
+      *row_ptr(j) = v;
+    }
+  }
+  __syncthreads();
   const int i0 = run * 16;
   float2 hst[3][4];
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
-    const int t = ci.t0 + i0 - 3 + j;
     float v8[8];
-    if (i0 >= ci.L) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v8[e] = 0.f;
-    } else if (t >= seq_start) {
-      load8(a.x + (size_t)t * Cc + ch, v8);
-    } else if (a.conv0) {
-      load8(a.conv0 + ((size_t)ci.n * 3 + 3 + (t - seq_start)) * Cc + ch, v8);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v8[e] = 0.f;
-    }
+    unpack8(*row_ptr(i0 + j), v8);
 #pragma unroll
     for (int p = 0; p < 4; ++p) hst[j][p] = make_float2(v8[2 * p], v8[2 * p + 1]);
   }
   const float sc_mul = kind == 0 ? a.q_scale : 1.0f;
-  constexpr int kPF = 4;
-#pragma unroll 1
-  for (int i8 = 0; i8 < 16; i8 += kPF) {
-    uint4 raw[kPF];
+#pragma unroll 4
+  for (int u = 0; u < 16; ++u) {
+    const int i = i0 + u;
+    float xv[8], y[8];
+    unpack8(*row_ptr(i + 3), xv);
+    if (a.conv_w) {
 #pragma unroll
-    for (int u = 0; u < kPF; ++u) {
-      const int i = i0 + i8 + u;
-      raw[u] = (i < ci.L) ? __ldg(reinterpret_cast<const uint4*>(a.x + (size_t)(ci.t0 + i) * Cc + ch))
-                          : make_uint4(0, 0, 0, 0);
+      for (int p = 0; p < 4; ++p) {
+        const float2 xp = make_float2(xv[2 * p], xv[2 * p + 1]);
+        float2 acc = __fmul2_rn(wv[3][p], xp);
+        acc = __ffma2_rn(wv[2][p], hst[2][p], acc);
+        acc = __ffma2_rn(wv[1][p], hst[1][p], acc);
+        acc = __ffma2_rn(wv[0][p], hst[0][p], acc);
+        y[2 * p] = silu_fast(acc.x);
+        y[2 * p + 1] = silu_fast(acc.y);
+        hst[0][p] = hst[1][p];
+        hst[1][p] = hst[2][p];
+        hst[2][p] = xp;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = xv[e];
     }
+    if (kind < 2) {
+      float ss = 0.f;
 #pragma unroll
-    for (int u = 0; u < kPF; ++u) {
-      const int i = i0 + i8 + u;
-      float xv[8], y[8];
-      unpack8(raw[u], xv);
-      if (a.conv_w) {
+      for (int e = 0; e < 8; ++e) ss += y[e] * y[e];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 xp = make_float2(xv[2 * p], xv[2 * p + 1]);
-          float2 acc = __fmul2_rn(wv[3][p], xp);
-          acc = __ffma2_rn(wv[2][p], hst[2][p], acc);
-          acc = __ffma2_rn(wv[1][p], hst[1][p], acc);
-          acc = __ffma2_rn(wv[0][p], hst[0][p], acc);
-          y[2 * p] = silu_fast(acc.x);
-          y[2 * p + 1] = silu_fast(acc.y);
-          hst[0][p] = hst[1][p];
-          hst[1][p] = hst[2][p];
-          hst[2][p] = xp;
-        }
-      } else {
+      for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float sc = sc_mul * rsqrtf(ss + a.l2_eps);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = xv[e];
-      }
-      if (kind < 2) {
-        float ss = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss += y[e] * y[e];
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float sc = sc_mul * rsqrtf(ss + a.l2_eps);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] *= sc;
-      }
-      if (i >= ci.L) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = 0.f;
-      }
-      store8(dst + (size_t)i * kD, y);
+      for (int e = 0; e < 8; ++e) y[e] *= sc;
     }
+    if (i >= ci.L) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = 0.f;
+    }
+    store8(dst + (size_t)i * kD, y);
   }
 }
 
@@ -1043,6 +1059,19 @@ static bool make_map(CUtensorMap* m, const void* base, size_t rows) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over the conv input x [T][Cc] bf16: box [128 + 3 rows][64 cols], 128-byte swizzle.
+static bool make_map_x(CUtensorMap* m, const void* base, int T, int Cc) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)Cc, (cuuint64_t)T};
+  cuuint64_t strides[1] = {(cuuint64_t)Cc * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)gdn::kXRows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DV>
 static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW,
                                 const CUtensorMap& mK, cudaStream_t s) {
@@ -1079,7 +1108,9 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   a.ws.Sw = reinterpret_cast<__nv_bfloat16*>(w + l.Sw);
   a.ws.Gw = reinterpret_cast<float*>(w + l.Gw);
   const size_t NC = (size_t)a.T / kC + (size_t)a.N + 1;
-  CUtensorMap mQ, mK, mW, mU, mS;
+  CUtensorMap mQ, mK, mW, mU, mS, mX;
+  const int Cc = (2 * a.Hk + a.Hv) * kD;
+  if (a.T > 0 && !make_map_x(&mX, a.x, a.T, Cc)) return cudaErrorInvalidValue;
   if (!make_map(&mQ, a.ws.Qw, NC * a.Hk * kC) || !make_map(&mK, a.ws.Kw, NC * a.Hk * kC) ||
       !make_map(&mW, a.ws.Ww, NC * a.Hv * kC) || !make_map(&mU, a.ws.Uw, NC * a.Hv * kC) ||
       !make_map(&mS, a.ws.Sw, NC * a.Hv * kC))
@@ -1092,6 +1123,9 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gdn::gdn_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                gdn::kOutSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn::gdn_qkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               gdn::kQkvSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -1103,7 +1137,7 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   const dim3 grid_chunks((unsigned)(a.T / kC + a.N), a.Hk);
   if (a.T > 0) {
     trace_begin("gdn_qkv", s);
-    gdn::gdn_qkv_kernel<<<dim3(grid_chunks.x, 2 * a.Hk + a.Hv), 128, 0, s>>>(a);
+    gdn::gdn_qkv_kernel<<<dim3(2 * a.Hk + a.Hv, grid_chunks.x), 128, gdn::kQkvSmem, s>>>(a, mX);
     trace_end(s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     trace_begin("gdn_prep", s);
