@@ -227,7 +227,7 @@ constexpr uint32_t kPrepKs = 0;        // K (TMA) -> K^ = diag(e^G) K, in place
 constexpr uint32_t kPrepR1 = 32768;    // A^T blocks (fp32) -> T_h^T (bf16) -> T diag(beta)
 constexpr uint32_t kPrepR2 = 65536;    // N (16 KB) + Y' (8 KB) -> V (TMA)
 constexpr uint32_t kPrepEnd = 98304;
-constexpr uint32_t kPrepSmem = kPrepEnd + 1024 + 1536;
+constexpr uint32_t kPrepSmem = kPrepEnd + 1024 + 2048;
 // TMEM columns (256 allocated)
 constexpr uint32_t kColGram = 0, kColY = 128, kColZ = 192, kColW = 0, kColU = 128;
 
@@ -237,14 +237,16 @@ __device__ __forceinline__ void zero_row_chunk(uint8_t* tile, uint32_t row, uint
 
 __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
                                                           const __grid_constant__ CUtensorMap mapK,
-                                                          const __grid_constant__ CUtensorMap mapV) {
+                                                          const __grid_constant__ CUtensorMap mapV,
+                                                          const __grid_constant__ CUtensorMap mapW) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   float* G_s = reinterpret_cast<float*>(sm + kPrepEnd);        // [128]
   float* B_s = G_s + kC;                                        // [128]
   float* wt_s = B_s + kC;                                       // [4] warp totals
-  uint64_t* bar_k = reinterpret_cast<uint64_t*>(wt_s + 8);
+  float* F_s = wt_s + 8;                                        // [128] column factors
+  uint64_t* bar_k = reinterpret_cast<uint64_t*>(F_s + kC);
   uint64_t* bar_v = bar_k + 1;
   uint64_t* bar = bar_k + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_k + 3);
@@ -295,6 +297,9 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
     a.ws.Gw[((size_t)c * Hv + h) * kC + i] = gv;
   }
   __syncthreads();
+  // column factors exp(G_m - G_j), m = last column of j's 32-column chunk (exponent <= 0)
+  if (tid < kC) F_s[tid] = __expf(G_s[tid | 31] - G_s[tid]);
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t sKs = smem_u32(sm + kPrepKs);
@@ -329,9 +334,18 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
       const int j0 = half * 64 + cc * 32;
       // warp-uniform: does any row of this warp have j < i inside this column chunk?
       const bool any_lower = j0 < quarter * 32 + 31;
+      const bool all_lower = j0 + 31 < quarter * 32;    // warp-uniform: every j < every i
       const bool needed = ((i >> 6) == half) || (half == 0);
       float av[32];
-      if (any_lower) {
+      if (all_lower) {
+        // exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31: both exponents <= 0
+        float v[32];
+        tmem_ld32(lane_addr + kColGram + j0, v);
+        const float rf = bi * __expf(Gi - G_s[j0 + 31]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) av[e] = rf * F_s[j0 + e] * v[e];
+      } else if (any_lower) {
         float v[32];
         tmem_ld32(lane_addr + kColGram + j0, v);
         tmem_ld_wait();
@@ -535,13 +549,12 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  // ---- W, U~ -> workspace (bf16 row-major; U~ replaces V): thread row i, column half wg
+  // ---- W, U~ -> bf16 swizzled tiles in smem (R1, R2 are free) -> TMA stores (U~ replaces V)
   {
     const int i = quarter * 32 + lane, half = wg;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      __nv_bfloat16* dst = (m == 0 ? a.ws.Ww : a.ws.Uw) +
-                           (((size_t)c * Hv + h) * kC + i) * kD + half * 64;
+      uint8_t* tile = sm + (m == 0 ? kPrepR1 : kPrepR2);
       const uint32_t col = (m == 0 ? kColW : kColU) + half * 64;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -549,14 +562,20 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
         tmem_ld32(lane_addr + col + cc * 32, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float w8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = v[8 * q + e];
-          store8(dst + cc * 32 + 8 * q, w8);
-        }
+        for (int q = 0; q < 4; ++q) st_row8_bf16(tile, kTile, i, half * 8 + cc * 4 + q, v + 8 * q);
       }
     }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    const int row = (c * Hv + h) * kC;
+    tma_store_2d(&mapW, sm + kPrepR1, 0, row);
+    tma_store_2d(&mapW, sm + kPrepR1 + kTile, 64, row);
+    tma_store_2d(&mapV, sm + kPrepR2, 0, row);
+    tma_store_2d(&mapV, sm + kPrepR2 + kTile, 64, row);
+    bulk_commit();
+    bulk_wait_all();
   }
 done:
   if (tid == 0 && !ok) report_status(a.status, GDN_ERR_TIMEOUT);
@@ -821,6 +840,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
   float* G_s = reinterpret_cast<float*>(sm + kOutEnd + 64);   // [128]
   float* red_s = G_s + kC;                                    // [2][128] partial sums of squares
   float* w_s = red_s + 2 * kC;                                // [128] norm weight
+  float* F_s = w_s + kC;                                      // [128] column factors
 
   const int c = blockIdx.x, h = blockIdx.y;
   const int total_chunks = a.ws.seq_first[a.N];
@@ -860,6 +880,9 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
   }
   __syncthreads();
   tc_fence_after();
+  // column factors exp(G_m - G_j), m = last column of j's 32-column chunk (exponent <= 0);
+  // read after the barriers of the gram wait below
+  if (tid < kC) F_s[tid] = __expf(G_s[tid | 31] - G_s[tid]);
   const uint32_t tmem = *tslot;
   const uint32_t lane_addr = tmem_at(tmem, quarter * 32, 0);
   const uint32_t sQ = smem_u32(sm + kOutQ), sKS = smem_u32(sm + kOutKS), sU = smem_u32(sm + kOutU);
@@ -896,17 +919,27 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
     for (int cc = 0; cc < 2; ++cc) {
       const int j0 = half * 64 + cc * 32;
       const bool any_lower = j0 <= quarter * 32 + 31;  // warp-uniform
+      const bool all_lower = j0 + 31 < quarter * 32;   // warp-uniform: every j < every i
       float v[32];
       if (any_lower) {
         tmem_ld32(lane_addr + kColQK + j0, v);
         tmem_ld_wait();
       }
+      if (all_lower) {
+        // exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31: both exponents <= 0
+        const float rf = __expf(Gi - G_s[j0 + 31]);
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        const int j = j0 + e;
-        const float p0 = (any_lower && j <= i) ? __expf(Gi - G_s[j]) * v[e] : 0.f;
-        const float p1 = (any_lower && j + 1 <= i) ? __expf(Gi - G_s[j + 1]) * v[e + 1] : 0.f;
-        pp[cc * 16 + e / 2] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < 32; e += 2)
+          pp[cc * 16 + e / 2] =
+              pack_bf16x2(rf * F_s[j0 + e] * v[e], rf * F_s[j0 + e + 1] * v[e + 1]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int j = j0 + e;
+          const float p0 = (any_lower && j <= i) ? __expf(Gi - G_s[j]) * v[e] : 0.f;
+          const float p1 = (any_lower && j + 1 <= i) ? __expf(Gi - G_s[j + 1]) * v[e + 1] : 0.f;
+          pp[cc * 16 + e / 2] = pack_bf16x2(p0, p1);
+        }
       }
     }
     const float eg = __expf(Gi);
@@ -1141,7 +1174,7 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     trace_end(s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     trace_begin("gdn_prep", s);
-    gdn::gdn_prep_kernel<<<dim3(grid_chunks.x, a.Hv), 256, gdn::kPrepSmem, s>>>(a, mK, mU);
+    gdn::gdn_prep_kernel<<<dim3(grid_chunks.x, a.Hv), 256, gdn::kPrepSmem, s>>>(a, mK, mU, mW);
     trace_end(s);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
