@@ -685,33 +685,33 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
   for (int ci = 0; ci < nch; ++ci) {
     const int c = first + ci, stage = ci & 1;
     if (tid == 0 && ci + 1 < nch) issue_tma(ci + 1, stage ^ 1);
-    __nv_bfloat16* Urow = a.ws.Uw + (((size_t)c * a.Hv + h) * kC + tid) * kD + v0;
-    // ---- S_b (bf16) -> SB operand and workspace; S^T *= e^(G_last)
-    {
-      const float gam = __expf(Gl_cur);
-      __nv_bfloat16* Srow = a.ws.Sw + (((size_t)c * a.Hv + h) * kD + k_row) * kD + v0;
+    // ---- S_b (bf16) -> SB operand (the only step X waits for).  With DV <= 64 the rest of the
+    // S bookkeeping runs while X is computed; DV = 128 keeps it here (register budget).
+    constexpr bool kOverlap = DV <= 64;
+    const float gam = __expf(Gl_cur);
+    __nv_bfloat16* Srow = a.ws.Sw + (((size_t)c * a.Hv + h) * kD + k_row) * kD + v0;
+    float sreg[(DV + 31) / 32][32];
 #pragma unroll
-      for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
-        float v[32];
-        tmem_ld32(lane_addr + colS + cc * 32, v);
-        tmem_ld_wait();
+    for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
+      tmem_ld32(lane_addr + colS + cc * 32, sreg[cc]);
+      tmem_ld_wait();
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (cc * 32 + 8 * q < DV) st_row8_bf16(SB, kTile, k_row, (cc * 32 + 8 * q) >> 3, sreg[cc] + 8 * q);
+      if constexpr (!kOverlap) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          if (cc * 32 + 8 * q < DV) {
-            const int ch = (cc * 32 + 8 * q) >> 3;
-            st_row8_bf16(SB, kTile, k_row, ch, v + 8 * q);
-            float w8[8];
+          float w8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = v[8 * q + e];
-            store8(Srow + cc * 32 + 8 * q, w8);
-          }
+          for (int e = 0; e < 8; ++e) w8[e] = sreg[cc][8 * q + e];
+          store8(Srow + cc * 32 + 8 * q, w8);
         }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] *= gam;
-        tmem_st32(lane_addr + colS + cc * 32, v);
+        for (int e = 0; e < 32; ++e) sreg[cc][e] *= gam;
+        tmem_st32(lane_addr + colS + cc * 32, sreg[cc]);
       }
-      tmem_st_wait();
     }
+    if constexpr (!kOverlap) tmem_st_wait();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -728,14 +728,34 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
         mma_commit(bar_mma);
       }
     }
-    if ((failed = __syncthreads_or(!ok))) break;
-    // next chunk's rows travel while the MMA runs
+    // while X runs: S_c to the workspace, S^T *= e^(G_last) in TMEM, next chunk's rows
+    if constexpr (kOverlap) {
+#pragma unroll
+      for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (cc * 32 + 8 * q < DV) {
+            float w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w8[e] = sreg[cc][8 * q + e];
+            store8(Srow + cc * 32 + 8 * q, w8);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sreg[cc][e] *= gam;
+        tmem_st32(lane_addr + colS + cc * 32, sreg[cc]);
+      }
+      tmem_st_wait();
+    }
     if (ci + 1 < nch) load_chunk_rows(ci + 1, ut_nxt, Gi_nxt, Gl_nxt);
+    if ((failed = __syncthreads_or(!ok))) break;
     ok = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1;
     if ((failed = __syncthreads_or(!ok))) break;
     tc_fence_after();
-    // ---- U = U~ - X -> workspace; U^ = diag(e^(G_L - G)) U -> UB operand
+    // ---- U = U~ - X; U^ = diag(e^(G_L - G)) U -> UB operand (U to the workspace afterwards)
+    float ureg[kOverlap ? DV : 8];
+    __nv_bfloat16* Urow = a.ws.Uw + (((size_t)c * a.Hv + h) * kC + tid) * kD + v0;
     {
       const float dec = __expf(Gl_cur - Gi_cur);
 #pragma unroll
@@ -748,7 +768,8 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
           if (cc * 32 + 8 * q < DV) {
             const int vq = (cc * 32 + 8 * q) >> 3;
             const __nv_bfloat162* uh = reinterpret_cast<const __nv_bfloat162*>(&ut_cur[vq]);
-            float u8[8], h8[8];
+            float* u8 = kOverlap ? ureg + vq * 8 : ureg;
+            float h8[8];
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
               const float2 f = __bfloat1622float2(uh[e2]);
@@ -757,8 +778,13 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) h8[e] = u8[e] * dec;
-            store8(Urow + cc * 32 + 8 * q, u8);
             st_row8_bf16(UB, kTile, tid, vq, h8);
+            if constexpr (!kOverlap) {
+              float w8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) w8[e] = u8[e];
+              store8(Urow + vq * 8, w8);
+            }
           }
         }
       }
@@ -775,6 +801,16 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
         mma_bf16(tmem + colS, desc_mnmajor(sK, kk, kTile), desc_mnmajor(sU, kk, kTile),
                  idesc_bf16(128, DV, true, true), 1);
       mma_commit(bar_mma);
+    }
+    // while the state update runs: U to the workspace
+    if constexpr (kOverlap) {
+#pragma unroll
+      for (int q = 0; q < DV / 8; ++q) {
+        float u8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) u8[e] = ureg[q * 8 + e];
+        store8(Urow + q * 8, u8);
+      }
     }
     ok = mbar_wait(bar_mma, mma_phase);
     mma_phase ^= 1;
