@@ -325,6 +325,20 @@ def dist_on():
     return torch.distributed.is_available() and torch.distributed.is_initialized()
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum over ranks of per-rank times: the slowest rank sets the job's time."""
+    if not dist_on():
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def job_tokens_per_s(world, tokens_per_rank, ms):
+    """Whole-job throughput of weak-scaled replicas: all ranks' tokens over the slowest time."""
+    return world * tokens_per_rank / (ms * 1e-3)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -356,14 +370,10 @@ def main():
     import gated_deltanet_layer_02_b200 as gdn
 
     step_ms, recs, clocks, (e2e_ms, h2d, d2h), eager_ms = bench_prefill(args, w, seed, dev, gdn)
-    ms = statistics.mean(step_ms)
-    if dist_on():
-        t = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([statistics.mean(step_ms), e2e_ms], dev)
     n = world
     T = w.tokens
-    value = n * T / (ms * 1e-3)
+    value = job_tokens_per_s(n, T, ms)
     peaks, peak_src = load_peaks()
 
     # per-kernel breakdown of the timed steps
@@ -402,11 +412,12 @@ def main():
 
     dec_ms, dec_bytes, dec_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev, gdn,
                                               args.decode_steps)
-    dec_gbs = dec_bytes / (dec_ms * 1e-3) / 1e9
+    dec_ms = max_over_ranks([dec_ms], dev)[0]
+    dec_gbs = n * dec_bytes / (dec_ms * 1e-3) / 1e9
     decode = {"workload": inputs.CONFIGS[3].name, "value": dec_gbs, "unit": "GB/s",
               "ms_per_step": dec_ms, "steps": args.decode_steps,
-              "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
-                           "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
+              "roofline": {"bound": "hbm", "achieved": dec_gbs / n, "peak": peaks["hbm_gbs"],
+                           "unit": "GB/s", "frac": dec_gbs / n / peaks["hbm_gbs"],
                            "traffic": ncu_traffic("decode_step"),
                            "peak_source": f"{peak_src} (copy)"},
               "clocks": dec_clk}
@@ -426,7 +437,7 @@ def main():
                    "launch": "CUDA graph replay of the whole step",
                    "chunk": CHUNK, "heads": [w.num_k_heads, w.num_v_heads], "head_dim": 128},
         "roofline": roof, "step_roofline": step_roof, "kernels": kern,
-        "e2e": {"value": n * T / (e2e_ms * 1e-3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+        "e2e": {"value": job_tokens_per_s(n, T, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": len(recs), "eager_ms_per_step": eager_ms,
         "clocks": clocks, "decode": decode, "cpu_baseline": cpu,
