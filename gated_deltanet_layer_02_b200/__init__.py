@@ -29,7 +29,7 @@ EXPORTS = (
     "gdn_gated_rmsnorm", "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill",
     "gdn_decode_step", "gdn_trace_create", "gdn_trace_destroy", "gdn_trace_attach",
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
-    "gdn_chunk_prefill_static_ws",
+    "gdn_chunk_prefill_static_ws", "gdn_trace_span",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
@@ -92,6 +92,8 @@ def lib():
             L.gdn_trace_count.argtypes = [vp]
             L.gdn_trace_get.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_char_p),
                                         ctypes.POINTER(ctypes.c_float)]
+            L.gdn_trace_span.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_float),
+                                         ctypes.POINTER(ctypes.c_float)]
             L.gdn_debug_wait_probe.argtypes = [vp, ctypes.c_uint32, vp]
             L.gdn_chunk_prefill_static_ws.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
                                                       i32, i32, vp, vp, vp, vp, vp, vp, vp]
@@ -291,6 +293,17 @@ class Trace:
             _check("gdn_trace_get", lib().gdn_trace_get(self._h, i, ctypes.byref(name),
                                                         ctypes.byref(ms)))
             out.append((name.value.decode(), ms.value))
+        return out
+
+    def timeline(self):
+        """[(kernel name, start ms, end ms)] relative to the start of the first launch."""
+        out = []
+        for i in range(lib().gdn_trace_count(self._h)):
+            name, a, b = ctypes.c_char_p(), ctypes.c_float(), ctypes.c_float()
+            _check("gdn_trace_get", lib().gdn_trace_get(self._h, i, ctypes.byref(name), None))
+            _check("gdn_trace_span", lib().gdn_trace_span(self._h, i, ctypes.byref(a),
+                                                          ctypes.byref(b)))
+            out.append((name.value.decode(), a.value, b.value))
         return out
 
     def close(self):

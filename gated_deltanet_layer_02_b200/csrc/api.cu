@@ -323,6 +323,18 @@ int gdn_trace_get(gdn_trace* trace, int32_t i, const char** name, float* ms) {
   return GDN_OK;
 }
 
+int gdn_trace_span(gdn_trace* trace, int32_t i, float* start_ms, float* end_ms) {
+  if (!trace || i < 0 || i >= trace->used || !start_ms || !end_ms) return GDN_ERR_INVALID_ARG;
+  auto& r0 = trace->recs[0];
+  auto& r = trace->recs[i];
+  if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventSynchronize(r0.stop) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  if (cudaEventElapsedTime(start_ms, r0.start, r.start) != cudaSuccess ||
+      cudaEventElapsedTime(end_ms, r0.start, r.stop) != cudaSuccess)
+    return GDN_ERR_CUDA;
+  return GDN_OK;
+}
+
 int gdn_debug_wait_probe(int32_t* dev_status, uint32_t limit_us, void* stream) {
   if (!dev_status || limit_us > 1000000u) return GDN_ERR_INVALID_ARG;
   gdn_host::trace_begin("wait_probe", static_cast<cudaStream_t>(stream));

@@ -67,6 +67,12 @@ struct PrefillArgs {
   int N, T, Hk, Hv, nsplit;
   float q_scale, l2_eps, norm_eps;
   Workspace ws;
+  // chunk range [c0, c1) of this launch (global chunk indices of the chunk table); a sequence
+  // that crosses c0 enters with the fp32 state in carry_in, one that crosses c1 leaves it in
+  // carry_out ([Hv][d_v][d_k] each: at most one sequence crosses any chunk boundary)
+  int c0, c1;
+  const float* carry_in;
+  float* carry_out;
 };
 
 }  // namespace gdn

@@ -28,6 +28,9 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <cstdlib>
+
 namespace gdn {
 
 constexpr int kC = 128;  // chunk length (tokens)
@@ -114,7 +117,7 @@ __global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 2 * kXBox);
-  const int grp = blockIdx.x, c = blockIdx.y;
+  const int grp = blockIdx.x, c = a.c0 + blockIdx.y;
   if (c >= a.ws.seq_first[a.N]) return;
   const ChunkInfo ci = a.ws.chunks[c];
   const int tid = threadIdx.x, vec = tid & 15, run = tid >> 4;
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   uint64_t* bar = bar_k + 2;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_k + 3);
 
-  const int c = blockIdx.x;
+  const int c = a.c0 + blockIdx.x;
   const int h = blockIdx.y;
   const int total_chunks = a.ws.seq_first[a.N];
   if (c >= total_chunks) return;
@@ -575,7 +578,7 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
     tma_store_2d(&mapV, sm + kPrepR2, 0, row);
     tma_store_2d(&mapV, sm + kPrepR2 + kTile, 64, row);
     bulk_commit();
-    bulk_wait_all();
+    bulk_wait_reads();  // the writes complete before the kernel is seen to end
   }
 done:
   if (tid == 0 && !ok) report_status(a.status, GDN_ERR_TIMEOUT);
@@ -585,31 +588,37 @@ done:
 }
 
 // --------------------------------------------------------------------------------- chain
-struct ChainMaps {
-  CUtensorMap W, K;
-};
-
+// One CTA per (sequence, value head, d_v block).  Thread t owns TMEM lane t % 128 (d_k row of S^T,
+// token row of X) and, with 256 threads (d_v blocks of 64 or 128), the column half t / 128.  A launch covers the chunks of its sequence inside [c0, c1): the state
+// enters from S0 (or zero) when the sequence starts there, else from carry_in, and leaves to SN
+// when the sequence ends there, else to carry_out.  Shared memory: W tile(s), one K tile and one
+// bf16 operand tile that holds S_b^T for X and then U^ for the state update (X has consumed S_b
+// by the time U^ is written).  It stays near 100 KB so that a prep or out CTA fits beside it.
 template <int DV>
 struct ChainCfg {
+  static_assert(DV == 32 || DV == 64 || DV == 128, "d_v block");
+  static constexpr int kThreads = DV >= 64 ? 256 : 128;
+  static constexpr int kCPT = DV * 128 / kThreads;              // value columns per thread
   static constexpr uint32_t kOpTiles = DV > 64 ? 2 : 1;         // 64-col tiles of S_b / U^
-  static constexpr uint32_t kStage = 2 * 2 * kTile;             // W + K tiles
-  static constexpr uint32_t kSB = 2 * kStage;                   // after two stages
-  static constexpr uint32_t kUB = kSB + kOpTiles * kTile;
-  static constexpr uint32_t kEnd = kUB + kOpTiles * kTile;
+  static constexpr uint32_t kWStages = DV > 64 ? 1 : 2;         // W tiles in flight
+  static constexpr uint32_t kK = kWStages * 2 * kTile;          // K tile pair
+  static constexpr uint32_t kOp = kK + 2 * kTile;               // S_b^T, then U^
+  static constexpr uint32_t kEnd = kOp + kOpTiles * kTile;
   static constexpr uint32_t kSmem = kEnd + 1024 + 256;
-  static constexpr uint32_t kTmemCols = DV < 32 ? 64 : 2 * DV;  // S^T | X
+  static constexpr uint32_t kTmemCols = 2 * DV;                 // S^T | X
 };
 
 template <int DV>
-__global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
+__global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(PrefillArgs a,
                                                            const __grid_constant__ CUtensorMap mapW,
                                                            const __grid_constant__ CUtensorMap mapK) {
   using Cfg = ChainCfg<DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(sm + Cfg::kEnd);  // [2]
-  uint64_t* bar_mma = bar_tma + 2;
+  uint64_t* bar_w = reinterpret_cast<uint64_t*>(sm + Cfg::kEnd);  // [kWStages]
+  uint64_t* bar_k = bar_w + 2;
+  uint64_t* bar_mma = bar_k + 1;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_mma + 1);
 
   const int nsplit = a.nsplit;
@@ -617,14 +626,21 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
   const int h = (blockIdx.x / nsplit) % a.Hv;
   const int n = blockIdx.x / (nsplit * a.Hv);
   const int hk = h / (a.Hv / a.Hk);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int first = a.ws.seq_first[n];
-  const int nch = a.ws.seq_first[n + 1] - first;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int s_first = a.ws.seq_first[n], s_end = a.ws.seq_first[n + 1];
+  const int first = max(s_first, a.c0);
+  const int nch = min(s_end, a.c1) - first;
+  // an empty sequence belongs to the launch whose range holds its position in the chunk table
+  const bool mine = nch > 0 || (s_first == s_end && a.c0 <= s_first && s_first < a.c1);
+  if (!mine) return;  // uniform over the CTA, before any barrier or TMEM is set up
+  const bool from_carry = s_first < a.c0;
+  const bool to_carry = s_end > a.c1;
   const int v0 = blk * DV;
 
   if (tid == 0) {
-    mbar_init(bar_tma, 1);
-    mbar_init(bar_tma + 1, 1);
+    mbar_init(bar_w, 1);
+    mbar_init(bar_w + 1, 1);
+    mbar_init(bar_k, 1);
     mbar_init(bar_mma, 1);
     fence_barrier_init();
   }
@@ -633,82 +649,105 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t colS = 0, colX = Cfg::kTmemCols / 2;
-  const uint32_t lane_addr = tmem_at(tmem, warp * 32, 0);
-  const int k_row = tid;  // TMEM lane = d_k index for S^T, = token index for X
+  constexpr int kCPT = Cfg::kCPT, kGroups = kCPT / 32;
+  const uint32_t lane_addr = tmem_at(tmem, (warp & 3) * 32, 0);
+  const int k_row = tid & 127;  // TMEM lane = d_k index for S^T, = token index for X
+  const int cs = (tid >> 7) * kCPT;  // first column of this thread inside the d_v block
+  const size_t sbase = ((size_t)n * a.Hv + h) * kD * kD;
 
-  // ---- S^T initial value: lane k, column v
+  // ---- S^T initial value: lane k, column v  (state layout [v][k])
   {
-    const size_t sbase = ((size_t)n * a.Hv + h) * kD * kD;
+    const float* src = from_carry ? a.carry_in + (size_t)h * kD * kD
+                                  : (a.S0 ? a.S0 + sbase : nullptr);
 #pragma unroll
-    for (int cc = 0; cc < DV / 32 + (DV < 32 ? 1 : 0); ++cc) {
+    for (int gi = 0; gi < kGroups; ++gi) {
       float v[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const int vv = v0 + cc * 32 + e;
-        v[e] = (a.S0 && cc * 32 + e < DV) ? a.S0[sbase + (size_t)vv * kD + k_row] : 0.f;
+        const int vv = v0 + cs + gi * 32 + e;
+        v[e] = src ? src[(size_t)vv * kD + k_row] : 0.f;
       }
-      tmem_st32(lane_addr + colS + cc * 32, v);
+      tmem_st32(lane_addr + colS + cs + gi * 32, v);
     }
     tmem_st_wait();
   }
-  auto issue_tma = [&](int ci, int stage) {
+  auto issue_w = [&](int ci) {
     const int c = first + ci;
-    uint8_t* st = sm + stage * Cfg::kStage;
-    mbar_arrive_expect_tx(bar_tma + stage, 4 * kTile);
-    const int rowW = (c * a.Hv + h) * kC, rowK = (c * a.Hk + hk) * kC;
-    tma_load_2d(st, &mapW, bar_tma + stage, 0, rowW);
-    tma_load_2d(st + kTile, &mapW, bar_tma + stage, 64, rowW);
-    tma_load_2d(st + 2 * kTile, &mapK, bar_tma + stage, 0, rowK);
-    tma_load_2d(st + 3 * kTile, &mapK, bar_tma + stage, 64, rowK);
+    const int st = Cfg::kWStages == 1 ? 0 : (ci & 1);
+    uint8_t* dst = sm + st * 2 * kTile;
+    mbar_arrive_expect_tx(bar_w + st, 2 * kTile);
+    const int row = (c * a.Hv + h) * kC;
+    tma_load_2d(dst, &mapW, bar_w + st, 0, row);
+    tma_load_2d(dst + kTile, &mapW, bar_w + st, 64, row);
   };
-  if (tid == 0 && nch > 0) issue_tma(0, 0);
+  auto issue_k = [&](int ci) {
+    const int c = first + ci;
+    uint8_t* dst = sm + Cfg::kK;
+    mbar_arrive_expect_tx(bar_k, 2 * kTile);
+    const int row = (c * a.Hk + hk) * kC;
+    tma_load_2d(dst, &mapK, bar_k, 0, row);
+    tma_load_2d(dst + kTile, &mapK, bar_k, 64, row);
+  };
+  // thread 0's count of loads issued and waited for, to drain them after a failed wait
+  int w_issued = 0, w_done = 0, k_issued = 0, k_done = 0;
+  bool mma_pending = false;
+  if (tid == 0 && nch > 0) {
+    issue_w(0);
+    issue_k(0);
+    w_issued = k_issued = 1;
+  }
   uint32_t mma_phase = 0;
   bool ok = true;
   int failed = 0;
-  uint8_t* SB = sm + Cfg::kSB;
-  uint8_t* UB = sm + Cfg::kUB;
-  // per-token inputs of a chunk (row = tid): U~ slice (packed bf16), G_i, G_last
-  constexpr int kVec = DV / 8;
+  uint8_t* OP = sm + Cfg::kOp;
+  // per-token inputs of a chunk (row = k_row): U~ slice (packed bf16), G_i, G_last
+  constexpr int kVec = kCPT / 8;
   uint4 ut_cur[kVec], ut_nxt[kVec];
   float Gi_cur = 0.f, Gl_cur = 0.f, Gi_nxt = 0.f, Gl_nxt = 0.f;
   auto load_chunk_rows = [&](int ci, uint4 (&ut)[kVec], float& Gi, float& Gl) {
     const int c = first + ci;
     const float* Gc = a.ws.Gw + ((size_t)c * a.Hv + h) * kC;
-    Gi = Gc[tid];
+    Gi = Gc[k_row];
     Gl = Gc[kC - 1];
     const uint4* src = reinterpret_cast<const uint4*>(
-        a.ws.Uw + (((size_t)c * a.Hv + h) * kC + tid) * kD + v0);
+        a.ws.Uw + (((size_t)c * a.Hv + h) * kC + k_row) * kD + v0 + cs);
 #pragma unroll
     for (int q = 0; q < kVec; ++q) ut[q] = src[q];
   };
   if (nch > 0) load_chunk_rows(0, ut_cur, Gi_cur, Gl_cur);
   for (int ci = 0; ci < nch; ++ci) {
-    const int c = first + ci, stage = ci & 1;
-    if (tid == 0 && ci + 1 < nch) issue_tma(ci + 1, stage ^ 1);
-    // ---- S_b (bf16) -> SB operand (the only step X waits for).  With DV <= 64 the rest of the
-    // S bookkeeping runs while X is computed; DV = 128 keeps it here (register budget).
-    constexpr bool kOverlap = DV <= 64;
+    const int c = first + ci;
+    const int wst = Cfg::kWStages == 1 ? 0 : (ci & 1);
+    const uint32_t wphase = Cfg::kWStages == 1 ? (ci & 1) : ((ci >> 1) & 1);
+    if (Cfg::kWStages == 2 && tid == 0 && ci + 1 < nch) {
+      issue_w(ci + 1);
+      ++w_issued;
+    }
+    // ---- S_b (bf16) -> operand tile (the only step X waits for).  With 32 columns per
+    // thread the rest of the S bookkeeping runs while X is computed; with 64 it stays here
+    // (register budget).
+    constexpr bool kOverlap = kCPT <= 32;
     const float gam = __expf(Gl_cur);
-    __nv_bfloat16* Srow = a.ws.Sw + (((size_t)c * a.Hv + h) * kD + k_row) * kD + v0;
-    float sreg[(DV + 31) / 32][32];
+    __nv_bfloat16* Srow = a.ws.Sw + (((size_t)c * a.Hv + h) * kD + k_row) * kD + v0 + cs;
+    float sreg[kGroups][32];
 #pragma unroll
-    for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
-      tmem_ld32(lane_addr + colS + cc * 32, sreg[cc]);
+    for (int gi = 0; gi < kGroups; ++gi) {
+      tmem_ld32(lane_addr + colS + cs + gi * 32, sreg[gi]);
       tmem_ld_wait();
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        if (cc * 32 + 8 * q < DV) st_row8_bf16(SB, kTile, k_row, (cc * 32 + 8 * q) >> 3, sreg[cc] + 8 * q);
+        st_row8_bf16(OP, kTile, k_row, (cs + gi * 32 + 8 * q) >> 3, sreg[gi] + 8 * q);
       if constexpr (!kOverlap) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float w8[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = sreg[cc][8 * q + e];
-          store8(Srow + cc * 32 + 8 * q, w8);
+          for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
+          store8(Srow + gi * 32 + 8 * q, w8);
         }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sreg[cc][e] *= gam;
-        tmem_st32(lane_addr + colS + cc * 32, sreg[cc]);
+        for (int e = 0; e < 32; ++e) sreg[gi][e] *= gam;
+        tmem_st32(lane_addr + colS + cs + gi * 32, sreg[gi]);
       }
     }
     if constexpr (!kOverlap) tmem_st_wait();
@@ -717,74 +756,78 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
     __syncthreads();
     // ---- X = W S_b^T  (M = 128 tokens, N = DV, K = d_k)
     if (tid == 0) {
-      ok = mbar_wait(bar_tma + stage, (ci >> 1) & 1);
+      ok = mbar_wait(bar_w + wst, wphase);
       tc_fence_after();
       if (ok) {
-        const uint32_t sW = smem_u32(sm + stage * Cfg::kStage), sS = smem_u32(SB);
+        ++w_done;
+        const uint32_t sW = smem_u32(sm + wst * 2 * kTile), sS = smem_u32(OP);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + colX, desc_kmajor(sW, kk, kTile), desc_mnmajor(sS, kk, kTile),
                    idesc_bf16(128, DV, false, true), kk > 0);
         mma_commit(bar_mma);
+        mma_pending = true;
       }
     }
     // while X runs: S_c to the workspace, S^T *= e^(G_last) in TMEM, next chunk's rows
     if constexpr (kOverlap) {
 #pragma unroll
-      for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
+      for (int gi = 0; gi < kGroups; ++gi) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          if (cc * 32 + 8 * q < DV) {
-            float w8[8];
+          float w8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = sreg[cc][8 * q + e];
-            store8(Srow + cc * 32 + 8 * q, w8);
-          }
+          for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
+          store8(Srow + gi * 32 + 8 * q, w8);
         }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sreg[cc][e] *= gam;
-        tmem_st32(lane_addr + colS + cc * 32, sreg[cc]);
+        for (int e = 0; e < 32; ++e) sreg[gi][e] *= gam;
+        tmem_st32(lane_addr + colS + cs + gi * 32, sreg[gi]);
       }
       tmem_st_wait();
     }
     if (ci + 1 < nch) load_chunk_rows(ci + 1, ut_nxt, Gi_nxt, Gl_nxt);
     if ((failed = __syncthreads_or(!ok))) break;
     ok = mbar_wait(bar_mma, mma_phase);
-    mma_phase ^= 1;
     if ((failed = __syncthreads_or(!ok))) break;
+    mma_phase ^= 1;
+    mma_pending = false;
     tc_fence_after();
-    // ---- U = U~ - X; U^ = diag(e^(G_L - G)) U -> UB operand (U to the workspace afterwards)
-    float ureg[kOverlap ? DV : 8];
-    __nv_bfloat16* Urow = a.ws.Uw + (((size_t)c * a.Hv + h) * kC + tid) * kD + v0;
+    // X has consumed W (single W buffer: the next chunk's W may come in now)
+    if (Cfg::kWStages == 1 && tid == 0 && ci + 1 < nch) {
+      issue_w(ci + 1);
+      ++w_issued;
+    }
+    // ---- U = U~ - X; U^ = diag(e^(G_L - G)) U -> operand tile (U to the workspace afterwards)
+    float ureg[kOverlap ? kCPT : 8];
+    __nv_bfloat16* Urow = a.ws.Uw + (((size_t)c * a.Hv + h) * kC + k_row) * kD + v0 + cs;
     {
       const float dec = __expf(Gl_cur - Gi_cur);
 #pragma unroll
-      for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
+      for (int gi = 0; gi < kGroups; ++gi) {
         float v[32];
-        tmem_ld32(lane_addr + colX + cc * 32, v);
+        tmem_ld32(lane_addr + colX + cs + gi * 32, v);
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          if (cc * 32 + 8 * q < DV) {
-            const int vq = (cc * 32 + 8 * q) >> 3;
-            const __nv_bfloat162* uh = reinterpret_cast<const __nv_bfloat162*>(&ut_cur[vq]);
-            float* u8 = kOverlap ? ureg + vq * 8 : ureg;
-            float h8[8];
+          const int vq = (gi * 32 + 8 * q) >> 3;  // 8-column group inside this thread's slice
+          const __nv_bfloat162* uh = reinterpret_cast<const __nv_bfloat162*>(&ut_cur[vq]);
+          float* u8 = kOverlap ? ureg + vq * 8 : ureg;
+          float h8[8];
 #pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-              const float2 f = __bfloat1622float2(uh[e2]);
-              u8[2 * e2] = f.x - v[8 * q + 2 * e2];
-              u8[2 * e2 + 1] = f.y - v[8 * q + 2 * e2 + 1];
-            }
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = __bfloat1622float2(uh[e2]);
+            u8[2 * e2] = f.x - v[8 * q + 2 * e2];
+            u8[2 * e2 + 1] = f.y - v[8 * q + 2 * e2 + 1];
+          }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) h8[e] = u8[e] * dec;
-            st_row8_bf16(UB, kTile, tid, vq, h8);
-            if constexpr (!kOverlap) {
-              float w8[8];
+          for (int e = 0; e < 8; ++e) h8[e] = u8[e] * dec;
+          st_row8_bf16(OP, kTile, k_row, (cs >> 3) + vq, h8);
+          if constexpr (!kOverlap) {
+            float w8[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) w8[e] = u8[e];
-              store8(Urow + vq * 8, w8);
-            }
+            for (int e = 0; e < 8; ++e) w8[e] = u8[e];
+            store8(Urow + vq * 8, w8);
           }
         }
       }
@@ -794,46 +837,66 @@ __global__ void __launch_bounds__(128, 1) gdn_chain_kernel(PrefillArgs a,
     __syncthreads();
     // ---- S^T += K^T U^  (M = d_k, N = DV, K = tokens)
     if (tid == 0) {
+      ok = mbar_wait(bar_k, ci & 1);
       tc_fence_after();
-      const uint32_t sK = smem_u32(sm + stage * Cfg::kStage + 2 * kTile), sU = smem_u32(UB);
+      if (ok) {
+        ++k_done;
+        const uint32_t sK = smem_u32(sm + Cfg::kK), sU = smem_u32(OP);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + colS, desc_mnmajor(sK, kk, kTile), desc_mnmajor(sU, kk, kTile),
-                 idesc_bf16(128, DV, true, true), 1);
-      mma_commit(bar_mma);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + colS, desc_mnmajor(sK, kk, kTile), desc_mnmajor(sU, kk, kTile),
+                   idesc_bf16(128, DV, true, true), 1);
+        mma_commit(bar_mma);
+        mma_pending = true;
+      }
     }
     // while the state update runs: U to the workspace
     if constexpr (kOverlap) {
 #pragma unroll
-      for (int q = 0; q < DV / 8; ++q) {
+      for (int q = 0; q < kCPT / 8; ++q) {
         float u8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) u8[e] = ureg[q * 8 + e];
         store8(Urow + q * 8, u8);
       }
     }
-    ok = mbar_wait(bar_mma, mma_phase);
-    mma_phase ^= 1;
     if ((failed = __syncthreads_or(!ok))) break;
+    ok = mbar_wait(bar_mma, mma_phase);
+    if ((failed = __syncthreads_or(!ok))) break;
+    mma_phase ^= 1;
+    mma_pending = false;
     tc_fence_after();
+    // the update has consumed K and the operand tile
+    if (tid == 0 && ci + 1 < nch) {
+      issue_k(ci + 1);
+      ++k_issued;
+    }
 #pragma unroll
     for (int q = 0; q < kVec; ++q) ut_cur[q] = ut_nxt[q];
     Gi_cur = Gi_nxt;
     Gl_cur = Gl_nxt;
   }
-  if (!failed && a.SN) {
-    const size_t sbase = ((size_t)n * a.Hv + h) * kD * kD;
+  float* dst = to_carry ? a.carry_out + (size_t)h * kD * kD : (a.SN ? a.SN + sbase : nullptr);
+  if (!failed && dst) {
 #pragma unroll
-    for (int cc = 0; cc < (DV + 31) / 32; ++cc) {
+    for (int gi = 0; gi < kGroups; ++gi) {
       float v[32];
-      tmem_ld32(lane_addr + colS + cc * 32, v);
+      tmem_ld32(lane_addr + colS + cs + gi * 32, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (cc * 32 + e < DV) a.SN[sbase + (size_t)(v0 + cc * 32 + e) * kD + k_row] = v[e];
+      for (int e = 0; e < 32; ++e) dst[(size_t)(v0 + cs + gi * 32 + e) * kD + k_row] = v[e];
     }
   }
-  if (tid == 0 && failed) report_status(a.status, GDN_ERR_TIMEOUT);
+  if (failed && tid == 0) {
+    report_status(a.status, GDN_ERR_TIMEOUT);
+    // give loads and products still in flight a bounded time to land before the CTA's shared
+    // memory and TMEM are released
+    for (int j = w_done; j < w_issued; ++j)
+      mbar_wait(bar_w + (Cfg::kWStages == 1 ? 0 : (j & 1)),
+                Cfg::kWStages == 1 ? (j & 1) : ((j >> 1) & 1));
+    for (int j = k_done; j < k_issued; ++j) mbar_wait(bar_k, j & 1);
+    if (mma_pending) mbar_wait(bar_mma, mma_phase);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, Cfg::kTmemCols);
@@ -878,7 +941,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
   float* w_s = red_s + 2 * kC;                                // [128] norm weight
   float* F_s = w_s + kC;                                      // [128] column factors
 
-  const int c = blockIdx.x, h = blockIdx.y;
+  const int c = a.c0 + blockIdx.x, h = blockIdx.y;
   const int total_chunks = a.ws.seq_first[a.N];
   if (c >= total_chunks) return;
   const ChunkInfo ci = a.ws.chunks[c];
@@ -1079,14 +1142,47 @@ using gdn::kD;
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+static int env_int(const char* name, int dflt) {
+  const char* v = getenv(name);
+  if (!v || !*v) return dflt;
+  char* end = nullptr;
+  const long x = strtol(v, &end, 10);
+  return (end && *end == 0 && x >= 0 && x < (1 << 20)) ? (int)x : dflt;
+}
+
+// Software pipeline over the chunk table.  The chunk range [0, NCmax) (NCmax = T/128 + N, an
+// upper bound on the chunks the table can hold) is cut into `nseg` segments of `seg` chunks.
+// Segment k's q/k/v + prep run while the chain works on segment k-1 and out on segment k-2, so
+// the sequential chain overlaps the parallel kernels instead of following them.  The parallel
+// kernels already fill every SM (two CTAs each, bound by shared memory), so the overlap only
+// pays where the chain is long: by default the table is cut only from 512 chunks on, into
+// segments of 64.  GDN_SEGMENT_CHUNKS=<n> sets the segment length (a value at or above the
+// chunk count gives a single launch of each kernel).
+struct SegPlan {
+  int nseg, seg;
+};
+
+static SegPlan seg_plan(int N, int T) {
+  const int NC = T / kC + N;
+  if (T == 0 || NC <= 1) return {1, NC > 0 ? NC : 1};
+  int target = env_int("GDN_SEGMENT_CHUNKS", 0);
+  if (target <= 0) target = NC >= 512 ? 64 : NC;
+  int nseg = (NC + target - 1) / target;
+  if (nseg < 1) nseg = 1;
+  const int seg = (NC + nseg - 1) / nseg;
+  nseg = (NC + seg - 1) / seg;
+  return {nseg, seg};
+}
+
 struct WsLayout {
-  size_t chunks, seq_first, Qw, Kw, Ww, Uw, Sw, Gw, total;
+  size_t chunks, seq_first, Qw, Kw, Ww, Uw, Sw, Gw, carry, total;
 };
 
 static WsLayout ws_layout(int N, int T, int Hk, int Hv) {
   const size_t NC = (size_t)T / kC + (size_t)N + 1;
   const size_t tile = (size_t)kC * kD * 2;
-  WsLayout l;
+  const SegPlan p = seg_plan(N, T);
+  WsLayout l{};
   size_t o = 0;
   l.chunks = o; o = align_up(o + NC * sizeof(gdn::ChunkInfo), 1024);
   l.seq_first = o; o = align_up(o + (size_t)(N + 1) * 4, 1024);
@@ -1096,6 +1192,8 @@ static WsLayout ws_layout(int N, int T, int Hk, int Hv) {
   l.Uw = o; o = align_up(o + NC * Hv * tile, 1024);
   l.Sw = o; o = align_up(o + NC * Hv * tile, 1024);
   l.Gw = o; o = align_up(o + NC * Hv * kC * 4, 1024);
+  // one fp32 [Hv][d][d] state per segment boundary (at most one sequence crosses each)
+  l.carry = o; o = align_up(o + (size_t)(p.nseg - 1) * Hv * kD * kD * 4, 1024);
   l.total = o;
   return l;
 }
@@ -1153,20 +1251,67 @@ static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW
     attr = true;
   }
   trace_begin("gdn_chain", s);
-  gdn::gdn_chain_kernel<DV><<<a.N * a.Hv * a.nsplit, 128, Cfg::kSmem, s>>>(a, mW, mK);
+  gdn::gdn_chain_kernel<DV><<<a.N * a.Hv * a.nsplit, Cfg::kThreads, Cfg::kSmem, s>>>(a, mW, mK);
   trace_end(s);
   return cudaGetLastError();
 }
 
 int choose_nsplit(int N, int Hv) {
+  const int forced = env_int("GDN_CHAIN_SPLIT", 0);
+  if (forced == 1 || forced == 2 || forced == 4) return forced;
   const int units = N * Hv;
   if (units >= 148) return 1;
   if (units * 2 >= 148) return 2;
   return 4;
 }
 
+// Helper streams of the pipeline, per device and host thread (a capture on one thread never
+// sees another thread's launches).  Consecutive segments alternate between two front streams
+// (q/k/v + prep) and two out streams, so that the next segment's CTAs fill the SMs while the
+// last wave of the previous one drains.  The chain stream gets the highest priority: it is the
+// critical path, and its CTAs should take a free SM slot before the next prep or out CTA.
+struct PipeStreams {
+  static constexpr int kWays = 2;
+  bool ready = false;
+  cudaStream_t P[kWays] = {}, O[kWays] = {}, C = nullptr;
+  cudaEvent_t fork = nullptr, evP = nullptr, evC = nullptr;
+  cudaEvent_t join[2 * kWays + 1] = {};
+};
+
+static cudaError_t pipe_streams(PipeStreams** out) {
+  constexpr int kMaxDev = 64;
+  static thread_local PipeStreams t_pipe[kMaxDev];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  PipeStreams& ps = t_pipe[dev];
+  if (!ps.ready) {
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+    for (int i = 0; i < PipeStreams::kWays; ++i)
+      if ((e = cudaStreamCreateWithPriority(&ps.P[i], cudaStreamNonBlocking, least)) !=
+              cudaSuccess ||
+          (e = cudaStreamCreateWithPriority(&ps.O[i], cudaStreamNonBlocking, least)) !=
+              cudaSuccess)
+        return e;
+    if ((e = cudaStreamCreateWithPriority(&ps.C, cudaStreamNonBlocking, greatest)) != cudaSuccess)
+      return e;
+    if ((e = cudaEventCreateWithFlags(&ps.fork, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&ps.evP, cudaEventDisableTiming)) != cudaSuccess ||
+        (e = cudaEventCreateWithFlags(&ps.evC, cudaEventDisableTiming)) != cudaSuccess)
+      return e;
+    for (cudaEvent_t& ev : ps.join)
+      if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    ps.ready = true;
+  }
+  *out = &ps;
+  return cudaSuccess;
+}
+
 cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t s) {
   const WsLayout l = ws_layout(a.N, a.T, a.Hk, a.Hv);
+  const SegPlan plan = seg_plan(a.N, a.T);
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a.ws.chunks = reinterpret_cast<gdn::ChunkInfo*>(w + l.chunks);
   a.ws.seq_first = reinterpret_cast<int32_t*>(w + l.seq_first);
@@ -1176,6 +1321,8 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   a.ws.Uw = reinterpret_cast<__nv_bfloat16*>(w + l.Uw);
   a.ws.Sw = reinterpret_cast<__nv_bfloat16*>(w + l.Sw);
   a.ws.Gw = reinterpret_cast<float*>(w + l.Gw);
+  float* carry = reinterpret_cast<float*>(w + l.carry);
+  const size_t carry_stride = (size_t)a.Hv * kD * kD;
   const size_t NC = (size_t)a.T / kC + (size_t)a.N + 1;
   CUtensorMap mQ, mK, mW, mU, mS, mX;
   const int Cc = (2 * a.Hk + a.Hv) * kD;
@@ -1203,30 +1350,79 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   gdn::chunk_schedule_kernel<<<1, 1024, 0, s>>>(a.cu, a.N, a.ws);
   trace_end(s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const dim3 grid_chunks((unsigned)(a.T / kC + a.N), a.Hk);
-  if (a.T > 0) {
-    trace_begin("gdn_qkv", s);
-    gdn::gdn_qkv_kernel<<<dim3(2 * a.Hk + a.Hv, grid_chunks.x), 128, gdn::kQkvSmem, s>>>(a, mX);
-    trace_end(s);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    trace_begin("gdn_prep", s);
-    gdn::gdn_prep_kernel<<<dim3(grid_chunks.x, a.Hv), 256, gdn::kPrepSmem, s>>>(a, mK, mU, mW);
-    trace_end(s);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // one segment's kernels on the given streams
+  auto launch_parallel_front = [&](const gdn::PrefillArgs& sa, cudaStream_t st) -> cudaError_t {
+    const unsigned nc = (unsigned)(sa.c1 - sa.c0);
+    trace_begin("gdn_qkv", st);
+    gdn::gdn_qkv_kernel<<<dim3(2 * sa.Hk + sa.Hv, nc), 128, gdn::kQkvSmem, st>>>(sa, mX);
+    trace_end(st);
+    cudaError_t e2 = cudaGetLastError();
+    if (e2 != cudaSuccess) return e2;
+    trace_begin("gdn_prep", st);
+    gdn::gdn_prep_kernel<<<dim3(nc, sa.Hv), 256, gdn::kPrepSmem, st>>>(sa, mK, mU, mW);
+    trace_end(st);
+    return cudaGetLastError();
+  };
+  auto launch_chain_any = [&](gdn::PrefillArgs sa, cudaStream_t st) -> cudaError_t {
+    switch (sa.nsplit) {
+      case 4: return launch_chain<32>(sa, mW, mK, st);
+      case 2: return launch_chain<64>(sa, mW, mK, st);
+      default: sa.nsplit = 1; return launch_chain<128>(sa, mW, mK, st);
+    }
+  };
+  auto launch_out = [&](const gdn::PrefillArgs& sa, cudaStream_t st) -> cudaError_t {
+    trace_begin("gdn_out", st);
+    gdn::gdn_out_kernel<<<dim3((unsigned)(sa.c1 - sa.c0), sa.Hv), gdn::kOutThreads, gdn::kOutSmem,
+                          st>>>(sa, mQ, mK, mS, mU);
+    trace_end(st);
+    return cudaGetLastError();
+  };
+
+  const int NCmax = a.T / kC + a.N;
+  if (plan.nseg <= 1) {
+    a.c0 = 0;
+    a.c1 = NCmax;
+    a.carry_in = nullptr;
+    a.carry_out = nullptr;
+    if (a.T > 0 && (e = launch_parallel_front(a, s)) != cudaSuccess) return e;
+    if ((e = launch_chain_any(a, s)) != cudaSuccess) return e;
+    if (a.T > 0 && (e = launch_out(a, s)) != cudaSuccess) return e;
+    return cudaSuccess;
   }
-  switch (a.nsplit) {
-    case 4: e = launch_chain<32>(a, mW, mK, s); break;
-    case 2: e = launch_chain<64>(a, mW, mK, s); break;
-    default: a.nsplit = 1; e = launch_chain<128>(a, mW, mK, s); break;
+
+  PipeStreams* ps = nullptr;
+  if ((e = pipe_streams(&ps)) != cudaSuccess) return e;
+  constexpr int W = PipeStreams::kWays;
+  cudaStream_t all[2 * W + 1] = {ps->C};
+  for (int i = 0; i < W; ++i) {
+    all[1 + i] = ps->P[i];
+    all[1 + W + i] = ps->O[i];
   }
-  if (e != cudaSuccess) return e;
-  if (a.T > 0) {
-    trace_begin("gdn_out", s);
-    gdn::gdn_out_kernel<<<dim3(grid_chunks.x, a.Hv), gdn::kOutThreads, gdn::kOutSmem, s>>>(
-        a, mQ, mK, mS, mU);
-    trace_end(s);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // fork: the helper streams start after everything already queued on s (the chunk table)
+  if ((e = cudaEventRecord(ps->fork, s)) != cudaSuccess) return e;
+  for (cudaStream_t st : all)
+    if ((e = cudaStreamWaitEvent(st, ps->fork, 0)) != cudaSuccess) return e;
+  for (int k = 0; k < plan.nseg; ++k) {
+    gdn::PrefillArgs sa = a;
+    sa.c0 = k * plan.seg;
+    sa.c1 = std::min(NCmax, (k + 1) * plan.seg);
+    sa.carry_in = k > 0 ? carry + (size_t)(k - 1) * carry_stride : nullptr;
+    sa.carry_out = k + 1 < plan.nseg ? carry + (size_t)k * carry_stride : nullptr;
+    cudaStream_t P = ps->P[k % W], O = ps->O[k % W];
+    if ((e = launch_parallel_front(sa, P)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ps->evP, P)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(ps->C, ps->evP, 0)) != cudaSuccess) return e;
+    if ((e = launch_chain_any(sa, ps->C)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ps->evC, ps->C)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(O, ps->evC, 0)) != cudaSuccess) return e;
+    if ((e = launch_out(sa, O)) != cudaSuccess) return e;
   }
+  // join: s continues after every helper stream
+  for (int i = 0; i < 2 * W + 1; ++i)
+    if ((e = cudaEventRecord(ps->join[i], all[i])) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(s, ps->join[i], 0)) != cudaSuccess)
+      return e;
   return cudaSuccess;
 }
 

@@ -187,6 +187,9 @@ int gdn_trace_reset(gdn_trace* trace);
 int gdn_trace_count(const gdn_trace* trace);   /* launches recorded */
 /* name: static kernel name; ms: device time of launch i (synchronises on its end event). */
 int gdn_trace_get(gdn_trace* trace, int32_t i, const char** name, float* ms);
+/* Start and end of launch i in ms after the start of launch 0 of the same trace (launches on
+ * different streams overlap on this common time line).  Synchronises on both end events. */
+int gdn_trace_span(gdn_trace* trace, int32_t i, float* start_ms, float* end_ms);
 
 /*
  * gdn_debug_wait_probe -- test aid for the bounded device waits: launches one CTA that waits

@@ -127,6 +127,8 @@ def test_trace_object_lifecycle(L):
     assert L.gdn_trace_attach(h) == gdn.GDN_OK
     assert L.gdn_trace_attach(None) == gdn.GDN_OK
     assert L.gdn_trace_get(h, 0, None, None) == gdn.GDN_ERR_INVALID_ARG
+    f = ctypes.c_float()
+    assert L.gdn_trace_span(h, 0, ctypes.byref(f), ctypes.byref(f)) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_trace_reset(h) == gdn.GDN_OK
     assert L.gdn_trace_destroy(h) == gdn.GDN_OK
     assert L.gdn_trace_create(None) == gdn.GDN_ERR_INVALID_ARG

@@ -98,3 +98,38 @@ def test_split_prefill_matches_whole():
     assert_close(torch.cat([a[0], b[0]]), ref_o, w.dtype, "split out")
     assert_close(b[1], ref_S, w.dtype, "split state")
     assert torch.equal(b[2], full[2])
+
+
+@pytest.fixture
+def pipeline_env(monkeypatch):
+    """Sets the library's pipeline knobs (segment length in chunks, chain d_v split)."""
+    def set_(seg, split):
+        monkeypatch.setenv("GDN_SEGMENT_CHUNKS", str(seg))
+        monkeypatch.setenv("GDN_CHAIN_SPLIT", str(split))
+    return set_
+
+
+@pytest.mark.parametrize("seg", [1, 2, 3, 5])
+@pytest.mark.parametrize("split", [1, 2, 4])
+def test_bf16_pipelined_segments(pipeline_env, seg, split):
+    # Segments of `seg` chunks: sequences cross segment boundaries (the state is carried in
+    # fp32 between launches), short and empty sequences fall inside one segment, and the
+    # chain's d_v split is forced so that every split meets every boundary case.
+    pipeline_env(seg, split)
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(700, 0, 5, 129, 0, 1100, 64, 260),
+                      s0_std=0.1)
+    _check(w, inputs.prefill_inputs(w, 1200 + 10 * seg + split, with_conv0=True),
+           f"seg={seg} split={split}")
+
+
+def test_bf16_pipelined_matches_single_launch_bitwise(pipeline_env):
+    # The pipeline reorders launches only: with the same split, the segmented and the single
+    # launch runs perform the same arithmetic and must agree to the bit.
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(900, 33, 1500), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 1300, with_conv0=True)
+    pipeline_env(1 << 19, 2)
+    one = gpu_prefill(w, inp)
+    pipeline_env(2, 2)
+    seg = gpu_prefill(w, inp)
+    for a, b, name in zip(one, seg, ("out", "final state", "conv state")):
+        assert torch.equal(a, b), name
