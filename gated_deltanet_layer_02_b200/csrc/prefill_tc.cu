@@ -227,12 +227,25 @@ __global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
 // cores) -> Y = N T_h, Z' = T_h Y diag(beta) (tcgen05) -> T diag(beta) -> W and U~ (tcgen05).
 // smem map (bytes from the 1024-aligned base)
 constexpr uint32_t kPrepKs = 0;        // K (TMA) -> K^ = diag(e^G) K, in place
-constexpr uint32_t kPrepR1 = 32768;    // A^T blocks (fp32) -> T_h^T (bf16) -> T diag(beta)
-constexpr uint32_t kPrepR2 = 65536;    // N (16 KB) + Y' (8 KB) -> V (TMA)
+constexpr uint32_t kPrepR1 = 32768;    // D -> T_h -> T diag(beta), row-major bf16
+constexpr uint32_t kPrepR2 = 65536;    // N (16 KB) + compact Y1 (16 KB) / Y' (8 KB) -> V (TMA)
 constexpr uint32_t kPrepEnd = 98304;
 constexpr uint32_t kPrepSmem = kPrepEnd + 1024 + 2048;
 // TMEM columns (256 allocated)
 constexpr uint32_t kColGram = 0, kColY = 128, kColZ = 192, kColW = 0, kColU = 128;
+constexpr uint32_t kColL = 128, kColY1 = 0, kColZ1 = 0;  // 32 -> 64 join (L1: packed bf16)
+
+// tcgen05.mma with the A operand in TMEM (row i in lane i, two bf16 per 32-bit column; one
+// K step of 16 = 8 columns) and B in shared memory.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
 __device__ __forceinline__ void zero_row_chunk(uint8_t* tile, uint32_t row, uint32_t chunk) {
   *reinterpret_cast<uint4*>(tile + sw128_off(row, chunk)) = make_uint4(0, 0, 0, 0);
@@ -326,189 +339,253 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
-  // ---------------- A from the gram: thread row i, column half wg
   {
-    const int i = quarter * 32 + lane, half = wg;
+  // ---------------- A from the gram: thread row i, column half wg (two 32-column chunks).
+  // The diagonal 32x32 blocks stay in the registers of the warps that invert them (row block q
+  // in column half q / 2: warps 0, 1, 6, 7).  The blocks (1,0) and (3,2) go to TMEM as the
+  // bf16 A operand L1 of the 32 -> 64 join; rows 64..127 x columns 0..63 go to the bf16 tile N
+  // of the 64 -> 128 join.  Everything above the diagonal is zero.
+  const int i = quarter * 32 + lane;
+  const bool solver = (quarter >> 1) == wg;  // warp-uniform
+  float adiag[32];
+  {
     const float Gi = G_s[i], bi = B_s[i];
-    float* ATh = reinterpret_cast<float*>(sm + kPrepR1) + half * 4096;
     uint8_t* Nt = sm + kPrepR2;
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
-      const int j0 = half * 64 + cc * 32;
-      // warp-uniform: does any row of this warp have j < i inside this column chunk?
-      const bool any_lower = j0 < quarter * 32 + 31;
-      const bool all_lower = j0 + 31 < quarter * 32;    // warp-uniform: every j < every i
-      const bool needed = ((i >> 6) == half) || (half == 0);
-      float av[32];
-      if (all_lower) {
-        // exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31: both exponents <= 0
-        float v[32];
-        tmem_ld32(lane_addr + kColGram + j0, v);
+      const int j0 = wg * 64 + cc * 32;
+      const int bj = j0 >> 5;  // column block (warp-uniform)
+      if (bj > quarter) continue;
+      float v[32];
+      tmem_ld32(lane_addr + kColGram + j0, v);
+      if (bj < quarter) {
+        // every j < every i: exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31,
+        // both exponents <= 0
         const float rf = bi * __expf(Gi - G_s[j0 + 31]);
         tmem_ld_wait();
+        float av[32];
 #pragma unroll
         for (int e = 0; e < 32; ++e) av[e] = rf * F_s[j0 + e] * v[e];
-      } else if (any_lower) {
-        float v[32];
-        tmem_ld32(lane_addr + kColGram + j0, v);
+        if (wg == 0 && quarter >= 2) {
+          // N: rows 64..127, columns 0..63 (bf16, K-major)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) st_row8_bf16(Nt, kTile, i, (j0 >> 3) + q, av + 8 * q);
+        } else {
+          // (1,0) or (3,2): L1 row, packed bf16 pairs at K = j0 .. j0 + 31 of 128
+          float pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = 0.f;
+          const int g = (j0 >> 1) >> 5;  // 32-column group of the packed K range
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[((j0 >> 1) & 31) + e] = __uint_as_float(pack_bf16x2(av[2 * e], av[2 * e + 1]));
+          float zz[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) zz[e] = 0.f;
+          tmem_st32(lane_addr + kColL + g * 32, pk);
+          tmem_st32(lane_addr + kColL + (g ^ 1) * 32, zz);
+        }
+      } else {
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int j = j0 + e;
-          av[e] = (j < i) ? bi * __expf(Gi - G_s[j]) * v[e] : 0.f;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) av[e] = 0.f;
-      }
-      if (needed) {
-        if ((i >> 6) == half) {
-          // diagonal block: transposed, ATh[jj][ii]
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ATh[((j0 + e) & 63) * 64 + (i & 63)] = av[e];
-        } else {
-          // lower-left block (i >= 64, j < 64) -> N (bf16, K-major)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) st_row8_bf16(Nt, kTile, i, (j0 >> 3) + q, av + 8 * q);
+          adiag[e] = (j < i) ? bi * __expf(Gi - G_s[j]) * v[e] : 0.f;
         }
       }
     }
-    if (i < 64 && half == 0) {
+    if (wg == 0 && quarter < 2) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) zero_row_chunk(Nt, i, q);
+      for (int q = 0; q < 8; ++q) zero_row_chunk(Nt, i, q);  // N rows 0..63 are zero
+    }
+    if (warp == 2 || warp == 4) {
+      // L1 rows 64..95 (warp 2) and 0..31 (warp 4) are zero
+      float zz[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) zz[e] = 0.f;
+      tmem_st32(lane_addr + kColL, zz);
+      tmem_st32(lane_addr + kColL + 32, zz);
     }
   }
-  tc_fence_before();
-  __syncthreads();
-  {
-    // ---- two 64x64 unit-lower inverses by forward substitution (threads 0..127: one column
-    // each).  Columns 32..63 are zero above their diagonal, so those warps skip ii < 32.
-    const int sb = (tid >> 6) & 1, sn = tid & 63;
-    float acc[64];
-    if (tid < 128) {
+  // ---------------- the four 32x32 diagonal inverses, one warp each, row i in lane i % 32:
+  // T_qq = (I + A_qq)^-1 row by row, T[l] = e_l - sum_{j<l} A[l][j] T[j]; row j is broadcast by
+  // shuffle once it is final (A[l][j] = 0 for j >= l, so every lane may take every step).
+  float trow[32];
+  uint8_t* Dt = sm + kPrepR1;  // D = blockdiag(T_00, T_11, T_22, T_33), row-major bf16
+  if (solver) {
 #pragma unroll
-      for (int rr = 0; rr < 64; ++rr) acc[rr] = (rr == sn) ? 1.f : 0.f;
-      const float* ATb = reinterpret_cast<const float*>(sm + kPrepR1) + sb * 4096;
-      const bool upper_cols = sn >= 32;  // warp-uniform
+    for (int e = 0; e < 32; ++e) trow[e] = (e == lane) ? 1.f : 0.f;
 #pragma unroll
-      for (int ii = 0; ii < 63; ++ii) {
-        if (ii < 32 && upper_cols) continue;
-        const float ti = acc[ii];
-        const float2 t2 = make_float2(-ti, -ti);
+    for (int j = 0; j < 31; ++j) {
+      const float2 cj = make_float2(-adiag[j], -adiag[j]);
 #pragma unroll
-        for (int r4 = (ii + 1) & ~3; r4 < 64; r4 += 4) {
-          const float4 av = *reinterpret_cast<const float4*>(ATb + ii * 64 + r4);
-          if (r4 > ii) {
-            const float2 lo =
-                __ffma2_rn(make_float2(av.x, av.y), t2, make_float2(acc[r4], acc[r4 + 1]));
-            acc[r4] = lo.x;
-            acc[r4 + 1] = lo.y;
-          } else if (r4 + 1 > ii) {
-            acc[r4 + 1] -= av.y * ti;
-          }
-          if (r4 + 2 > ii) {
-            const float2 hi =
-                __ffma2_rn(make_float2(av.z, av.w), t2, make_float2(acc[r4 + 2], acc[r4 + 3]));
-            acc[r4 + 2] = hi.x;
-            acc[r4 + 3] = hi.y;
-          } else if (r4 + 3 > ii) {
-            acc[r4 + 3] -= av.w * ti;
-          }
+      for (int e = 0; e <= j; e += 2) {
+        if (e + 1 <= j) {
+          const float x0 = __shfl_sync(0xffffffffu, trow[e], j);
+          const float x1 = __shfl_sync(0xffffffffu, trow[e + 1], j);
+          const float2 o = __ffma2_rn(cj, make_float2(x0, x1), make_float2(trow[e], trow[e + 1]));
+          trow[e] = o.x;
+          trow[e + 1] = o.y;
+        } else {
+          const float x0 = __shfl_sync(0xffffffffu, trow[e], j);
+          trow[e] = fmaf(cj.x, x0, trow[e]);
         }
       }
     }
-    __syncthreads();
-    // ---- T_h^T (bf16) into R1: row n' = column n' of T_h
-    uint8_t* TT = sm + kPrepR1;
-    if (tid < 128) {
-      const int row = sb * 64 + sn;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) st_row8_bf16(TT, kTile, row, sb * 8 + q, acc + 8 * q);
-      if (sb == 1) {
+    for (int q = 0; q < 4; ++q) st_row8_bf16(Dt, kTile, i, quarter * 4 + q, trow + 8 * q);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) zero_row_chunk(TT, row, q);
-      }
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    // ---- Y = N T_h (M=128, N=64, K=64)
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sN = smem_u32(sm + kPrepR2), sT = smem_u32(TT);
+    for (int q = 0; q < 4; ++q) zero_row_chunk(Dt + wg * kTile, i, ((quarter & 1) ? 0 : 4) + q);
+  } else {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kColY, desc_kmajor(sN, kk, kTile), desc_kmajor(sT, kk, kTile),
-                 idesc_bf16(128, 64, false, false), kk > 0);
-      mma_commit(bar);
-    }
-    ok = mbar_wait(bar, phase);
-    phase ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
+    for (int q = 0; q < 8; ++q) zero_row_chunk(Dt + wg * kTile, i, q);
+  }
+  tmem_st_wait();
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---------------- 32 -> 64:  T_64 = D - D L1 D   (Y1 = L1 D, Z1 = D Y1; (L1 D)^2 = 0 inside
+  // each 64 block).  L1 is non-zero in the K ranges 0..31 and 64..95 only.
+  const uint32_t sD = smem_u32(Dt);
+  uint8_t* Yc = sm + kPrepR2 + kTile;  // Y1 rows 32..63 and 96..127, compacted: [64][128] bf16
+  if (tid == 0) {
     tc_fence_after();
-    // ---- Y' = Y diag(beta) restricted to rows 64..127, cols 0..63 -> bf16 [64][64]
-    if (quarter >= 2) {
-      const int j = quarter * 32 + lane, half = wg;
+    constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+    const int ks[4] = {0, 1, 4, 5};
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      mma_bf16_ts(tmem + kColY1, tmem + kColL + ks[t] * 8, desc_mnmajor(sD, ks[t], kTile), id,
+                  t > 0);
+    mma_commit(bar);
+  }
+  ok = mbar_wait(bar, phase);
+  phase ^= 1;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  if (quarter & 1) {
+    // rows 32..63 -> compact rows 0..31, rows 96..127 -> 32..63 (swizzle phase kept: row & 7)
+    const int cr = quarter == 1 ? i - 32 : i - 64;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
       float v[32];
-      tmem_ld32(lane_addr + kColY + half * 32, v);
+      tmem_ld32(lane_addr + kColY1 + wg * 64 + cc * 32, v);
       tmem_ld_wait();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] *= B_s[half * 32 + e];
-      uint8_t* Yt = sm + kPrepR2 + kTile;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) st_row8_bf16(Yt, kTile, j - 64, half * 4 + q, v + 8 * q);
+      for (int q = 0; q < 4; ++q) st_row8_bf16(Yc, 8192, cr, wg * 8 + cc * 4 + q, v + 8 * q);
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- Z' = T_h Y' (M=128, N=64, K=64 over rows 64..127 of T_h)
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t sT = smem_u32(TT), sY = smem_u32(sm + kPrepR2 + kTile);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + kColZ, desc_mnmajor(sT + 8192, kk, kTile), desc_mnmajor(sY, kk, kTile),
-                 idesc_bf16(128, 64, true, true), kk > 0);
-      mma_commit(bar);
-    }
-    ok = mbar_wait(bar, phase);
-    phase ^= 1;
-    if (__syncthreads_or(!ok)) goto done;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0) {
     tc_fence_after();
-    // ---- V into R2 (N and Y' are consumed) while T diag(beta) and K^ are built
-    if (tid == 0) {
-      const int rowV = (c * Hv + h) * kC;
-      mbar_arrive_expect_tx(bar_v, 2 * kTile);
-      tma_load_2d(sm + kPrepR2, &mapV, bar_v, 0, rowV);
-      tma_load_2d(sm + kPrepR2 + kTile, &mapV, bar_v, 64, rowV);
-    }
-    uint8_t* TB = sm + kPrepR1;
-    if (tid < 128) {
-      // diagonal blocks from the column owners: element (sb*64+rr, sb*64+sn)
-      const int col = sb * 64 + sn;
-      const float bcol = B_s[col];
+    constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+    const uint32_t sYc = smem_u32(Yc);
+    const int ks[4] = {2, 3, 6, 7};
 #pragma unroll
-      for (int rr = 0; rr < 64; ++rr) {
-        const int row = sb * 64 + rr;
-        __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(
-            TB + sb * kTile + sw128_off(row, (sn >> 3)) + (sn & 7) * 2);
-        *p = __float2bfloat16_rn(acc[rr] * bcol);
-      }
-    } else if (tid < 192) {
-      const int row = tid - 128;  // upper-right block is zero
+    for (int t = 0; t < 4; ++t)
+      mma_bf16(tmem + kColZ1, desc_kmajor(sD, ks[t], kTile), desc_mnmajor(sYc, t, 8192), id,
+               t > 0);
+    mma_commit(bar);
+  }
+  ok = mbar_wait(bar, phase);
+  phase ^= 1;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  if ((quarter == 1 && wg == 0) || (quarter == 3 && wg == 1)) {
+    // -Z1 into the (1,0) and (3,2) blocks: D becomes T_h = blockdiag(T_64, T_64')
+    const int c0 = quarter == 1 ? 0 : 64;
+    float v[32];
+    tmem_ld32(lane_addr + kColZ1 + c0, v);
+    tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < 8; ++q) zero_row_chunk(TB + kTile, row, q);
-    }
+    for (int e = 0; e < 32; ++e) v[e] = -v[e];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) st_row8_bf16(Dt, kTile, i, (c0 >> 3) + q, v + 8 * q);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---------------- 64 -> 128:  T = T_h - T_h N T_h diag... (N = rows 64..127, cols 0..63)
+  // ---- Y = N T_h (M=128, N=64, K=64): B = T_h rows 0..63, columns 0..63 (MN-major)
+  if (tid == 0) {
+    tc_fence_after();
+    const uint32_t sN = smem_u32(sm + kPrepR2);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tmem + kColY, desc_kmajor(sN, kk, kTile), desc_mnmajor(sD, kk, kTile),
+               idesc_bf16(128, 64, false, true), kk > 0);
+    mma_commit(bar);
+  }
+  ok = mbar_wait(bar, phase);
+  phase ^= 1;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  // ---- Y' = Y diag(beta) restricted to rows 64..127, cols 0..63 -> bf16 [64][64]
+  if (quarter >= 2) {
+    const int half = wg;
+    float v[32];
+    tmem_ld32(lane_addr + kColY + half * 32, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] *= B_s[half * 32 + e];
+    uint8_t* Yt = sm + kPrepR2 + kTile;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) st_row8_bf16(Yt, kTile, i - 64, half * 4 + q, v + 8 * q);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  // ---- Z' = T_h[:, 64..127] Y' (M=128, N=64, K=64): A = T_h's second column tile (K-major)
+  if (tid == 0) {
+    tc_fence_after();
+    const uint32_t sY = smem_u32(sm + kPrepR2 + kTile);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tmem + kColZ, desc_kmajor(sD + kTile, kk, kTile), desc_mnmajor(sY, kk, kTile),
+               idesc_bf16(128, 64, false, true), kk > 0);
+    mma_commit(bar);
+  }
+  ok = mbar_wait(bar, phase);
+  phase ^= 1;
+  if (__syncthreads_or(!ok)) goto done;
+  tc_fence_after();
+  // ---- V into R2 (N and Y' are consumed) while T diag(beta) is written over T_h:
+  //   diagonal 32-blocks from the fp32 rows of the solver warps, the (1,0), (3,2) blocks from
+  //   -Z1 (TMEM), the lower-left 64x64 block from -Z' (which already carries diag(beta))
+  if (tid == 0) {
+    const int rowV = (c * Hv + h) * kC;
+    mbar_arrive_expect_tx(bar_v, 2 * kTile);
+    tma_load_2d(sm + kPrepR2, &mapV, bar_v, 0, rowV);
+    tma_load_2d(sm + kPrepR2 + kTile, &mapV, bar_v, 64, rowV);
+  }
+  if (solver) {
+#pragma unroll
+    for (int e = 0; e < 32; ++e) trow[e] *= B_s[quarter * 32 + e];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) st_row8_bf16(Dt, kTile, i, quarter * 4 + q, trow + 8 * q);
+  }
+  if ((quarter == 1 && wg == 1) || (quarter == 3 && wg == 0)) {
+    const int c0 = quarter == 1 ? 0 : 64;
+    float v[32];
+    tmem_ld32(lane_addr + kColZ1 + c0, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = -v[e] * B_s[c0 + e];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) st_row8_bf16(Dt, kTile, i, (c0 >> 3) + q, v + 8 * q);
   }
   if (quarter >= 2) {
     // lower-left block: -Z'
-    const int i = quarter * 32 + lane, half = wg;
+    const int half = wg;
     float v[32];
     tmem_ld32(lane_addr + kColZ + half * 32, v);
     tmem_ld_wait();
 #pragma unroll
     for (int e = 0; e < 32; ++e) v[e] = -v[e];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) st_row8_bf16(sm + kPrepR1, kTile, i, half * 4 + q, v + 8 * q);
+    for (int q = 0; q < 4; ++q) st_row8_bf16(Dt, kTile, i, half * 4 + q, v + 8 * q);
+  }
   }
   {
     // K^ = diag(e^G) K in place: thread pair per row, 8 chunks each
@@ -915,15 +992,6 @@ constexpr uint32_t kOutSmem = kOutEnd + 1024 + 4096;
 constexpr uint32_t kColQK = 0, kColP = 0, kColQh = 64, kColO = 128;  // 256 TMEM columns
 constexpr int kOutThreads = 256;
 
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
     PrefillArgs a, const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
