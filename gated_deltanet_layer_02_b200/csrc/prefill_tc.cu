@@ -265,7 +265,8 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   uint64_t* bar_k = reinterpret_cast<uint64_t*>(F_s + kC);
   uint64_t* bar_v = bar_k + 1;
   uint64_t* bar = bar_k + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_k + 3);
+  uint64_t* bar_w = bar_k + 3;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_k + 4);
 
   const int c = a.c0 + blockIdx.x;
   const int h = blockIdx.y;
@@ -281,6 +282,7 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
     mbar_init(bar_k, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar, 1);
+    mbar_init(bar_w, 1);
     fence_barrier_init();
     const int rowK = (c * a.Hk + hk) * kC;
     mbar_arrive_expect_tx(bar_k, 2 * kTile);
@@ -439,6 +441,21 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   } else {
 #pragma unroll
     for (int q = 0; q < 8; ++q) zero_row_chunk(Dt + wg * kTile, i, q);
+    // meanwhile K^ = diag(e^G) K in place (the gram has consumed K): one row per thread
+    const int row = ((warp - 2) & 3) * 32 + lane;  // warps 2..5 -> rows 0..127
+    const float gam = __expf(G_s[row]);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const uint32_t off = (q >> 3) * kTile + sw128_off(row, q & 7);
+      uint4 u = *reinterpret_cast<const uint4*>(sm + kPrepKs + off);
+      __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(hv[e]);
+        hv[e] = __floats2bfloat162_rn(f.x * gam, f.y * gam);
+      }
+      *reinterpret_cast<uint4*>(sm + kPrepKs + off) = u;
+    }
   }
   tmem_st_wait();
   fence_proxy_async_smem();
@@ -587,54 +604,41 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
     for (int q = 0; q < 4; ++q) st_row8_bf16(Dt, kTile, i, half * 4 + q, v + 8 * q);
   }
   }
-  {
-    // K^ = diag(e^G) K in place: thread pair per row, 8 chunks each
-    const int row = tid >> 1, part = tid & 1;
-    const float gam = __expf(G_s[row]);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int chunk16 = part * 8 + q;
-      const uint32_t off = (chunk16 >> 3) * kTile + sw128_off(row, chunk16 & 7);
-      uint4 u = *reinterpret_cast<const uint4*>(sm + kPrepKs + off);
-      __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hv[e]);
-        hv[e] = __floats2bfloat162_rn(f.x * gam, f.y * gam);
-      }
-      *reinterpret_cast<uint4*>(sm + kPrepKs + off) = u;
-    }
-  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
-  // ---- W = T diag(beta) K^,  U~ = T diag(beta) V
+  // ---- W = T diag(beta) K^ (issued at once), U~ = T diag(beta) V (once V has landed);
+  // separate commits, so that W is read out while U~ is computed
   if (tid == 0) {
+    tc_fence_after();
+    const uint32_t sTB = smem_u32(sm + kPrepR1), sK = smem_u32(sm + kPrepKs),
+                   sV = smem_u32(sm + kPrepR2);
+    constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16(tmem + kColW, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sK, kk, kTile), id, kk > 0);
+    mma_commit(bar_w);
     ok = mbar_wait(bar_v, 0);
     tc_fence_after();
     if (ok) {
-      const uint32_t sTB = smem_u32(sm + kPrepR1), sK = smem_u32(sm + kPrepKs),
-                     sV = smem_u32(sm + kPrepR2);
-      constexpr uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        mma_bf16(tmem + kColW, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sK, kk, kTile), id, kk > 0);
+      for (int kk = 0; kk < 8; ++kk)
         mma_bf16(tmem + kColU, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sV, kk, kTile), id, kk > 0);
-      }
       mma_commit(bar);
+    } else {
+      mbar_wait(bar_w, 0);  // let the W products finish before the CTA gives up its TMEM
     }
   }
   if (__syncthreads_or(!ok)) goto done;
-  ok = mbar_wait(bar, phase);
-  phase ^= 1;
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
-  // ---- W, U~ -> bf16 swizzled tiles in smem (R1, R2 are free) -> TMA stores (U~ replaces V)
+  // ---- W, then U~ -> bf16 swizzled tiles (W over K^, U~ over V) -> TMA stores
   {
     const int i = quarter * 32 + lane, half = wg;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      uint8_t* tile = sm + (m == 0 ? kPrepR1 : kPrepR2);
+      ok = mbar_wait(m == 0 ? bar_w : bar, m == 0 ? 0 : phase);
+      if (__syncthreads_or(!ok)) goto done;
+      tc_fence_after();
+      uint8_t* tile = sm + (m == 0 ? kPrepKs : kPrepR2);
       const uint32_t col = (m == 0 ? kColW : kColU) + half * 64;
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
@@ -644,21 +648,23 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
 #pragma unroll
         for (int q = 0; q < 4; ++q) st_row8_bf16(tile, kTile, i, half * 8 + cc * 4 + q, v + 8 * q);
       }
+      fence_proxy_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        const int row = (c * Hv + h) * kC;
+        const CUtensorMap* map = m == 0 ? &mapW : &mapV;
+        tma_store_2d(map, tile, 0, row);
+        tma_store_2d(map, tile + kTile, 64, row);
+        bulk_commit();
+      }
     }
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (tid == 0) {
-    const int row = (c * Hv + h) * kC;
-    tma_store_2d(&mapW, sm + kPrepR1, 0, row);
-    tma_store_2d(&mapW, sm + kPrepR1 + kTile, 64, row);
-    tma_store_2d(&mapV, sm + kPrepR2, 0, row);
-    tma_store_2d(&mapV, sm + kPrepR2 + kTile, 64, row);
-    bulk_commit();
-    bulk_wait_reads();  // the writes complete before the kernel is seen to end
+    if (tid == 0) bulk_wait_reads();  // the writes complete before the kernel is seen to end
   }
 done:
-  if (tid == 0 && !ok) report_status(a.status, GDN_ERR_TIMEOUT);
+  if (tid == 0 && !ok) {
+    report_status(a.status, GDN_ERR_TIMEOUT);
+    bulk_wait_reads();  // a store already issued still reads shared memory
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(*tslot, 256);
