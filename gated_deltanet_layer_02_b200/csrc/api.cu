@@ -242,8 +242,12 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
   a.q_scale = dims->q_scale;
   a.l2_eps = dims->l2_eps;
   a.norm_eps = dims->norm_eps;
+  // the final conv history comes out of the q/k/v kernel unless it overwrites conv0 in place
+  // (another chunk of the sequence may still read conv0 then)
+  const bool separate_conv_state = convN && (convN == conv0 || num_tokens == 0);
+  a.convN = separate_conv_state ? nullptr : static_cast<__nv_bfloat16*>(convN);
   cudaError_t e = gdn_host::launch_prefill_tc(a, workspace, s);
-  if (e == cudaSuccess && convN)
+  if (e == cudaSuccess && separate_conv_state)
     e = gdn_host::launch_conv_state_out(true, x, cu_seqlens, num_seqs, Cc, conv0, convN, s);
   return map_cuda(e);
 }

@@ -49,6 +49,8 @@ struct Workspace {
   __nv_bfloat16* Uw;     // [NCmax][Hv][128][128]  U~ from prep, overwritten with U by chain
   __nv_bfloat16* Sw;     // [NCmax][Hv][128 (d_k)][128 (d_v)]  S^T entering each chunk
   float* Gw;             // [NCmax][Hv][128]  cumulative log decay inside the chunk
+  int* ready;            // [NCmax][Hv]  prep published (chunk, value head); zeroed per call
+  int* counter;          // next prep unit of the persistent workers; zeroed per call
 };
 
 struct PrefillArgs {
@@ -62,6 +64,8 @@ struct PrefillArgs {
   const float* S0;
   float* SN;
   const __nv_bfloat16* conv0;
+  __nv_bfloat16* convN;  // written by the q/k/v kernel (and the chunk table for empty sequences)
+                         // when set; NULL when the caller wants none or it aliases conv0
   __nv_bfloat16* out;
   int32_t* status;
   int N, T, Hk, Hv, nsplit;

@@ -29,6 +29,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <utility>
 #include <cstdlib>
 
 namespace gdn {
@@ -40,7 +41,12 @@ constexpr uint32_t kTile = 16384;  // one [128][64] bf16 row tile
 
 
 // ------------------------------------------------------------------------------ schedule
-__global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Workspace ws) {
+__global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Workspace ws,
+                                      int nready, const __nv_bfloat16* conv0,
+                                      __nv_bfloat16* convN, int Cc) {
+  // publication flags and work counter of the persistent prep + chain kernel
+  for (int k = threadIdx.x; k < nready; k += blockDim.x) ws.ready[k] = 0;
+  if (threadIdx.x == 0 && nready > 0) *ws.counter = 0;
   // single CTA, sequential prefix over sequences in blocks of blockDim
   __shared__ int carry;
   __shared__ int part[1024];
@@ -75,6 +81,14 @@ __global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Wor
     __syncthreads();
   }
   if (threadIdx.x == 0) ws.seq_first[N] = carry;
+  // final conv history of empty sequences (the q/k/v kernel writes the others): the initial one
+  if (convN) {
+    for (int n = 0; n < N; ++n) {
+      if (cu[n + 1] != cu[n]) continue;
+      for (int k = threadIdx.x; k < 3 * Cc; k += blockDim.x)
+        convN[(size_t)n * 3 * Cc + k] = conv0 ? conv0[(size_t)n * 3 * Cc + k] : __float2bfloat16(0.f);
+    }
+  }
 }
 
 
@@ -118,6 +132,7 @@ __global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 2 * kXBox);
   const int grp = blockIdx.x, c = a.c0 + blockIdx.y;
+  pdl_wait();  // the chunk table, and the end of every reader of the previous call's tiles
   if (c >= a.ws.seq_first[a.N]) return;
   const ChunkInfo ci = a.ws.chunks[c];
   const int tid = threadIdx.x, vec = tid & 15, run = tid >> 4;
@@ -147,8 +162,8 @@ __global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
       const float2 f0 = __bfloat1622float2(hw[0]), f1 = __bfloat1622float2(hw[1]);
       const float t[4] = {f0.x, f0.y, f1.x, f1.y};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (e & 1) wv[k][e >> 1].y = t[k]; else wv[k][e >> 1].x = t[k];
+      for (int k = 0; k < 4; ++k) {  // halved: the conv then yields h = x / 2 for the SiLU
+        if (e & 1) wv[k][e >> 1].y = 0.5f * t[k]; else wv[k][e >> 1].x = 0.5f * t[k];
       }
     }
   }
@@ -156,6 +171,7 @@ __global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
   const uint32_t chunk = vec & 7;
   auto row_ptr = [&](int r) { return reinterpret_cast<uint4*>(box + sw128_off(r, chunk)); };
   const bool ok = mbar_wait(bar, 0);
+  pdl_trigger();
   if (!ok) {
     if (tid == 0) report_status(a.status, GDN_ERR_TIMEOUT);
     return;
@@ -170,6 +186,13 @@ __global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
     }
   }
   __syncthreads();
+  // last chunk of its sequence: the final conv history is the box's rows L .. L+2 (the three
+  // inputs before the sequence end, conv state rows included when L < 3)
+  if (a.convN && run == 0 && ci.t0 + ci.L == __ldg(a.cu + ci.n + 1)) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      *reinterpret_cast<uint4*>(a.convN + ((size_t)ci.n * 3 + j) * Cc + ch) = *row_ptr(ci.L + j);
+  }
   const int i0 = run * 16;
   float2 hst[3][4];
 #pragma unroll
@@ -185,33 +208,40 @@ __global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
     const int i = i0 + u;
     float xv[8], y[8];
     unpack8(*row_ptr(i + 3), xv);
+    float2 y2[4];
     if (a.conv_w) {
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         const float2 xp = make_float2(xv[2 * p], xv[2 * p + 1]);
-        float2 acc = __fmul2_rn(wv[3][p], xp);
-        acc = __ffma2_rn(wv[2][p], hst[2][p], acc);
-        acc = __ffma2_rn(wv[1][p], hst[1][p], acc);
-        acc = __ffma2_rn(wv[0][p], hst[0][p], acc);
-        y[2 * p] = silu_fast(acc.x);
-        y[2 * p + 1] = silu_fast(acc.y);
+        float2 hh = __fmul2_rn(wv[3][p], xp);  // h = conv / 2
+        hh = __ffma2_rn(wv[2][p], hst[2][p], hh);
+        hh = __ffma2_rn(wv[1][p], hst[1][p], hh);
+        hh = __ffma2_rn(wv[0][p], hst[0][p], hh);
+        // silu(x) = x sigmoid(x) = h + h tanh(h), h = x / 2
+        y2[p] = __ffma2_rn(hh, make_float2(tanh_approx(hh.x), tanh_approx(hh.y)), hh);
         hst[0][p] = hst[1][p];
         hst[1][p] = hst[2][p];
         hst[2][p] = xp;
       }
     } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = xv[e];
+      for (int p = 0; p < 4; ++p) y2[p] = make_float2(xv[2 * p], xv[2 * p + 1]);
     }
     if (kind < 2) {
-      float ss = 0.f;
+      float2 s2 = __fmul2_rn(y2[0], y2[0]);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss += y[e] * y[e];
+      for (int p = 1; p < 4; ++p) s2 = __ffma2_rn(y2[p], y2[p], s2);
+      float ss = s2.x + s2.y;
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
       const float sc = sc_mul * rsqrtf(ss + a.l2_eps);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] *= sc;
+      for (int p = 0; p < 4; ++p) y2[p] = __fmul2_rn(y2[p], make_float2(sc, sc));
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      y[2 * p] = y2[p].x;
+      y[2 * p + 1] = y2[p].y;
     }
     if (i >= ci.L) {
 #pragma unroll
@@ -251,45 +281,73 @@ __device__ __forceinline__ void zero_row_chunk(uint8_t* tile, uint32_t row, uint
   *reinterpret_cast<uint4*>(tile + sw128_off(row, chunk)) = make_uint4(0, 0, 0, 0);
 }
 
-__global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
-                                                          const __grid_constant__ CUtensorMap mapK,
-                                                          const __grid_constant__ CUtensorMap mapV,
-                                                          const __grid_constant__ CUtensorMap mapW) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
-  float* G_s = reinterpret_cast<float*>(sm + kPrepEnd);        // [128]
-  float* B_s = G_s + kC;                                        // [128]
-  float* wt_s = B_s + kC;                                       // [4] warp totals
-  float* F_s = wt_s + 8;                                        // [128] column factors
-  uint64_t* bar_k = reinterpret_cast<uint64_t*>(F_s + kC);
-  uint64_t* bar_v = bar_k + 1;
-  uint64_t* bar = bar_k + 2;
-  uint64_t* bar_w = bar_k + 3;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_k + 4);
+// Barriers and small arrays of a prep CTA, above the tiles.
+struct PrepCtl {
+  float* G_s;       // [128]
+  float* B_s;       // [128]
+  float* wt_s;      // [8] warp totals
+  float* F_s;       // [128] column factors
+  uint64_t* bar_k;  // K landed
+  uint64_t* bar_v;  // V landed
+  uint64_t* bar;    // MMA completions (six per unit)
+  uint64_t* bar_w;  // W products done
+  uint32_t* tslot;  // TMEM address
+  int* unit;        // next work unit (persistent workers)
+  __device__ explicit PrepCtl(uint8_t* sm) {
+    G_s = reinterpret_cast<float*>(sm + kPrepEnd);
+    B_s = G_s + kC;
+    wt_s = B_s + kC;
+    F_s = wt_s + 8;
+    bar_k = reinterpret_cast<uint64_t*>(F_s + kC);
+    bar_v = bar_k + 1;
+    bar = bar_k + 2;
+    bar_w = bar_k + 3;
+    tslot = reinterpret_cast<uint32_t*>(bar_k + 4);
+    unit = reinterpret_cast<int*>(tslot + 1);
+  }
+  __device__ void init() const {  // one thread; a __syncthreads must follow before any wait
+    mbar_init(bar_k, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar, 1);
+    mbar_init(bar_w, 1);
+    fence_barrier_init();
+  }
+};
 
-  const int c = a.c0 + blockIdx.x;
-  const int h = blockIdx.y;
-  const int total_chunks = a.ws.seq_first[a.N];
-  if (c >= total_chunks) return;
+// One (chunk c, value head h) unit of prep on a CTA whose barriers are initialised and whose 256
+// TMEM columns are allocated.  `par` is the parity of this unit on bar_k, bar_v and bar_w (one
+// completion each per unit; bar completes six times, so its parity starts at 0 every unit).
+// With `ready` set, W, U~ and G are published for the chain: once the TMA stores have completed,
+// thread 0 sets ready[c * Hv + h] with release semantics.  Returns false after a wait ran out
+// (the status word is set; the CTA must not start another unit).
+__device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMap& mapK,
+                                          const CUtensorMap& mapV, const CUtensorMap& mapW,
+                                          int c, int h, uint8_t* sm, uint32_t tmem, uint32_t par,
+                                          int* ready) {
+  const PrepCtl ctl(sm);
+  float* G_s = ctl.G_s;
+  float* B_s = ctl.B_s;
+  float* wt_s = ctl.wt_s;
+  float* F_s = ctl.F_s;
+  uint64_t* bar_k = ctl.bar_k;
+  uint64_t* bar_v = ctl.bar_v;
+  uint64_t* bar = ctl.bar;
+  uint64_t* bar_w = ctl.bar_w;
   const ChunkInfo ci = a.ws.chunks[c];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int quarter = warp & 3, wg = warp >> 2;
   const int Hv = a.Hv;
   const int hk = h / (Hv / a.Hk);
 
-  if (tid == 0) {
-    mbar_init(bar_k, 1);
-    mbar_init(bar_v, 1);
-    mbar_init(bar, 1);
-    mbar_init(bar_w, 1);
-    fence_barrier_init();
+  // thread 128 (a warp that does not scan the gates) waits for the q/k/v tiles of the previous
+  // kernel and starts the K load; the gates below overlap that kernel's tail
+  if (tid == 128) {
+    pdl_wait();
     const int rowK = (c * a.Hk + hk) * kC;
     mbar_arrive_expect_tx(bar_k, 2 * kTile);
     tma_load_2d(sm + kPrepKs, &mapK, bar_k, 0, rowK);
     tma_load_2d(sm + kPrepKs + kTile, &mapK, bar_k, 64, rowK);
   }
-  if (warp == 0) tmem_alloc(tslot, 256);
   // ---------------- gates: G = inclusive cumsum of g inside the chunk, beta
   if (warp < 4) {
     const int i = warp * 32 + lane;
@@ -319,14 +377,13 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   if (tid < kC) F_s[tid] = __expf(G_s[tid | 31] - G_s[tid]);
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tslot;
   const uint32_t sKs = smem_u32(sm + kPrepKs);
   const uint32_t lane_addr = tmem_at(tmem, quarter * 32, 0);
   uint32_t phase = 0;
   bool ok = true;
   // ---------------- gram K K^T
   if (tid == 0) {
-    ok = mbar_wait(bar_k, 0);
+    ok = mbar_wait(bar_k, par);
     tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -571,6 +628,7 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   //   diagonal 32-blocks from the fp32 rows of the solver warps, the (1,0), (3,2) blocks from
   //   -Z1 (TMEM), the lower-left 64x64 block from -Z' (which already carries diag(beta))
   if (tid == 0) {
+    pdl_wait();  // returns at once: thread 128 has seen the previous kernel complete
     const int rowV = (c * Hv + h) * kC;
     mbar_arrive_expect_tx(bar_v, 2 * kTile);
     tma_load_2d(sm + kPrepR2, &mapV, bar_v, 0, rowV);
@@ -618,7 +676,8 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
     for (int kk = 0; kk < 8; ++kk)
       mma_bf16(tmem + kColW, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sK, kk, kTile), id, kk > 0);
     mma_commit(bar_w);
-    ok = mbar_wait(bar_v, 0);
+    pdl_trigger();
+    ok = mbar_wait(bar_v, par);
     tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -626,7 +685,7 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
         mma_bf16(tmem + kColU, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sV, kk, kTile), id, kk > 0);
       mma_commit(bar);
     } else {
-      mbar_wait(bar_w, 0);  // let the W products finish before the CTA gives up its TMEM
+      mbar_wait(bar_w, par);  // let the W products finish before the CTA gives up its TMEM
     }
   }
   if (__syncthreads_or(!ok)) goto done;
@@ -635,7 +694,7 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
     const int i = quarter * 32 + lane, half = wg;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      ok = mbar_wait(m == 0 ? bar_w : bar, m == 0 ? 0 : phase);
+      ok = mbar_wait(m == 0 ? bar_w : bar, m == 0 ? par : phase);
       if (__syncthreads_or(!ok)) goto done;
       tc_fence_after();
       uint8_t* tile = sm + (m == 0 ? kPrepKs : kPrepR2);
@@ -658,16 +717,50 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
         bulk_commit();
       }
     }
-    if (tid == 0) bulk_wait_reads();  // the writes complete before the kernel is seen to end
+    if (tid == 0) {
+      if (ready) {
+        bulk_wait_all();             // W and U~ are in global memory
+        fence_proxy_async_global();  // ... for the TMA loads of the chain as well
+        __threadfence();
+        st_release_gpu(ready + c * Hv + h, 1);
+      } else {
+        bulk_wait_reads();  // the writes complete before the kernel is seen to end
+      }
+    }
   }
 done:
-  if (tid == 0 && !ok) {
+  // every exit reaches this point on all threads (each early exit follows a block-wide vote)
+  const bool all_ok = !__syncthreads_or(!ok);
+  if (tid == 0 && !all_ok) {
     report_status(a.status, GDN_ERR_TIMEOUT);
     bulk_wait_reads();  // a store already issued still reads shared memory
   }
+  return all_ok;
+}
+
+__global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
+                                                          const __grid_constant__ CUtensorMap mapK,
+                                                          const __grid_constant__ CUtensorMap mapV,
+                                                          const __grid_constant__ CUtensorMap mapW) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const PrepCtl ctl(sm);
+  const int c = a.c0 + blockIdx.x;
+  const int h = blockIdx.y;
+  if (c >= a.ws.seq_first[a.N]) {
+    pdl_wait();
+    return;
+  }
+  if (threadIdx.x == 128) ctl.init();
+  if (threadIdx.x < 32) tmem_alloc(ctl.tslot, 256);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *ctl.tslot;
+  prep_unit(a, mapK, mapV, mapW, c, h, sm, tmem, 0, nullptr);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(*tslot, 256);
+  if (threadIdx.x < 32) tmem_dealloc(tmem, 256);
 }
 
 // --------------------------------------------------------------------------------- chain
@@ -677,13 +770,14 @@ done:
 // when the sequence ends there, else to carry_out.  Shared memory: W tile(s), one K tile and one
 // bf16 operand tile that holds S_b^T for X and then U^ for the state update (X has consumed S_b
 // by the time U^ is written).  It stays near 100 KB so that a prep or out CTA fits beside it.
-template <int DV>
+template <int DV, int WS = (DV > 64 ? 1 : 2)>
 struct ChainCfg {
   static_assert(DV == 32 || DV == 64 || DV == 128, "d_v block");
+  static_assert(WS == 1 || WS == 2, "W stages");
   static constexpr int kThreads = DV >= 64 ? 256 : 128;
   static constexpr int kCPT = DV * 128 / kThreads;              // value columns per thread
   static constexpr uint32_t kOpTiles = DV > 64 ? 2 : 1;         // 64-col tiles of S_b / U^
-  static constexpr uint32_t kWStages = DV > 64 ? 1 : 2;         // W tiles in flight
+  static constexpr uint32_t kWStages = WS;                      // W tiles in flight
   static constexpr uint32_t kK = kWStages * 2 * kTile;          // K tile pair
   static constexpr uint32_t kOp = kK + 2 * kTile;               // S_b^T, then U^
   static constexpr uint32_t kEnd = kOp + kOpTiles * kTile;
@@ -691,25 +785,28 @@ struct ChainCfg {
   static constexpr uint32_t kTmemCols = 2 * DV;                 // S^T | X
 };
 
-template <int DV>
-__global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(PrefillArgs a,
-                                                           const __grid_constant__ CUtensorMap mapW,
-                                                           const __grid_constant__ CUtensorMap mapK) {
-  using Cfg = ChainCfg<DV>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+// The chain of CTA `bid` = (sequence, value head, d_v block).  With `ready` set (persistent
+// prep + chain kernel), thread 0 waits for prep to publish each chunk before loading it.
+template <int DV, int WS>
+__device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorMap& mapW,
+                                           const CUtensorMap& mapK, int bid, uint8_t* sm,
+                                           const int* ready) {
+  using Cfg = ChainCfg<DV, WS>;
+  // the chain's own threads (the first Cfg::kThreads of the block) synchronise on barrier 1
+#define CSYNC() bar_sync_n(1, Cfg::kThreads)
+#define CSYNC_OR(x) bar_or_n(1, Cfg::kThreads, (x))
   uint64_t* bar_w = reinterpret_cast<uint64_t*>(sm + Cfg::kEnd);  // [kWStages]
   uint64_t* bar_k = bar_w + 2;
   uint64_t* bar_mma = bar_k + 1;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_mma + 1);
 
   const int nsplit = a.nsplit;
-  const int blk = blockIdx.x % nsplit;
-  const int h = (blockIdx.x / nsplit) % a.Hv;
-  const int n = blockIdx.x / (nsplit * a.Hv);
+  const int blk = bid % nsplit;
+  const int h = (bid / nsplit) % a.Hv;
+  const int n = bid / (nsplit * a.Hv);
   const int hk = h / (a.Hv / a.Hk);
   const int tid = threadIdx.x, warp = tid >> 5;
+  pdl_wait();  // W, U~, G of this call (unless `ready`), and the carry of the previous launch
   const int s_first = a.ws.seq_first[n], s_end = a.ws.seq_first[n + 1];
   const int first = max(s_first, a.c0);
   const int nch = min(s_end, a.c1) - first;
@@ -728,7 +825,7 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(tslot, Cfg::kTmemCols);
-  __syncthreads();
+  CSYNC();
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t colS = 0, colX = Cfg::kTmemCols / 2;
@@ -774,6 +871,18 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
   // thread 0's count of loads issued and waited for, to drain them after a failed wait
   int w_issued = 0, w_done = 0, k_issued = 0, k_done = 0;
   bool mma_pending = false;
+  bool flag_ok = true;
+  int flag_next = 0;  // thread 0: relaxed read of the next chunk's flag
+  if (ready && nch > 0) {
+    if (tid == 0) flag_ok = wait_flag(ready + first * a.Hv + h);
+    if (CSYNC_OR(!flag_ok)) {
+      if (tid == 0) report_status(a.status, GDN_ERR_TIMEOUT);
+      tc_fence_before();
+      CSYNC();
+      if (warp == 0) tmem_dealloc(tmem, Cfg::kTmemCols);
+      return;
+    }
+  }
   if (tid == 0 && nch > 0) {
     issue_w(0);
     issue_k(0);
@@ -802,7 +911,21 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
     const int c = first + ci;
     const int wst = Cfg::kWStages == 1 ? 0 : (ci & 1);
     const uint32_t wphase = Cfg::kWStages == 1 ? (ci & 1) : ((ci >> 1) & 1);
-    if (Cfg::kWStages == 2 && tid == 0 && ci + 1 < nch) {
+    // the next chunk's prep must be published before any of its loads (thread 0 issues the W
+    // load; every thread reads its U~ rows after the barrier below)
+    if (ready && tid == 0 && ci + 1 < nch) {
+      // the flag of chunk c + 1 was read (relaxed) one step ago; if it was set, an acquire
+      // fence completes the synchronisation, otherwise wait for it
+      if (flag_next != 0) {
+        fence_acq_rel_gpu();
+        fence_proxy_async_global();
+      } else {
+        flag_ok = wait_flag(ready + (c + 1) * a.Hv + h);
+      }
+      flag_next = ci + 2 < nch ? ld_relaxed_gpu(ready + (c + 2) * a.Hv + h) : 1;
+    }
+    __syncwarp();  // warp 0 reconverges before its TMEM loads
+    if (Cfg::kWStages == 2 && tid == 0 && ci + 1 < nch && flag_ok) {
       issue_w(ci + 1);
       ++w_issued;
     }
@@ -836,10 +959,10 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
     if constexpr (!kOverlap) tmem_st_wait();
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    CSYNC();
     // ---- X = W S_b^T  (M = 128 tokens, N = DV, K = d_k)
     if (tid == 0) {
-      ok = mbar_wait(bar_w + wst, wphase);
+      ok = flag_ok && mbar_wait(bar_w + wst, wphase);
       tc_fence_after();
       if (ok) {
         ++w_done;
@@ -870,9 +993,9 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
       tmem_st_wait();
     }
     if (ci + 1 < nch) load_chunk_rows(ci + 1, ut_nxt, Gi_nxt, Gl_nxt);
-    if ((failed = __syncthreads_or(!ok))) break;
+    if ((failed = CSYNC_OR(!ok))) break;
     ok = mbar_wait(bar_mma, mma_phase);
-    if ((failed = __syncthreads_or(!ok))) break;
+    if ((failed = CSYNC_OR(!ok))) break;
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
@@ -917,7 +1040,7 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    CSYNC();
     // ---- S^T += K^T U^  (M = d_k, N = DV, K = tokens)
     if (tid == 0) {
       ok = mbar_wait(bar_k, ci & 1);
@@ -943,9 +1066,9 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
         store8(Urow + q * 8, u8);
       }
     }
-    if ((failed = __syncthreads_or(!ok))) break;
+    if ((failed = CSYNC_OR(!ok))) break;
     ok = mbar_wait(bar_mma, mma_phase);
-    if ((failed = __syncthreads_or(!ok))) break;
+    if ((failed = CSYNC_OR(!ok))) break;
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
@@ -981,8 +1104,73 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
     if (mma_pending) mbar_wait(bar_mma, mma_phase);
   }
   tc_fence_before();
-  __syncthreads();
+  CSYNC();
   if (warp == 0) tmem_dealloc(tmem, Cfg::kTmemCols);
+#undef CSYNC
+#undef CSYNC_OR
+}
+
+template <int DV>
+__global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(PrefillArgs a,
+                                                           const __grid_constant__ CUtensorMap mapW,
+                                                           const __grid_constant__ CUtensorMap mapK) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  pdl_trigger();
+  chain_body<DV, ChainCfg<DV>::kWStages>(a, mapW, mapK, blockIdx.x, sm, nullptr);
+}
+
+// ------------------------------------------------------------------------ prep + chain
+// One persistent launch of prep and chain, for a chunk table with few chains: CTAs below
+// `nchain` run one chain each (d_v blocks of DV columns); every other CTA is a prep worker that
+// takes (chunk, value head) units in chunk-major order from a device counter and publishes each
+// unit with a flag the chain waits for.  Workers never wait on the chains, so the chains make
+// progress as long as a worker holds an SM slot, which a grid of (SM slots) CTAs with fewer
+// chains than slots guarantees; every wait is bounded in any case.  The flags and the counter
+// are zeroed by the chunk-table kernel of the same call.
+// The chain role keeps a single W buffer here, so that two CTAs of either role fit on an SM.
+template <int DV>
+constexpr uint32_t fused_smem() {
+  return ChainCfg<DV, 1>::kSmem > kPrepSmem ? ChainCfg<DV, 1>::kSmem : kPrepSmem;
+}
+
+template <int DV>
+__global__ void __launch_bounds__(256, 2) gdn_prep_chain_kernel(
+    PrefillArgs a, const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+    const __grid_constant__ CUtensorMap mapW, int nchain) {
+  static_assert(ChainCfg<DV, 1>::kThreads <= 256, "block size");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  if ((int)blockIdx.x < nchain) {
+    // a chain uses the first ChainCfg::kThreads threads; the others leave at once
+    if ((int)threadIdx.x < ChainCfg<DV, 1>::kThreads)
+      chain_body<DV, 1>(a, mapW, mapK, blockIdx.x, sm, a.ws.ready);
+    return;
+  }
+  const PrepCtl ctl(sm);
+  const int tid = threadIdx.x;
+  pdl_wait();  // the chunk table
+  const int units = a.ws.seq_first[a.N] * a.Hv;
+  if (tid == 128) ctl.init();
+  if (tid < 32) tmem_alloc(ctl.tslot, 256);
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *ctl.tslot;
+  uint32_t par = 0;
+  while (true) {
+    if (tid == 0) *ctl.unit = atomicAdd(a.ws.counter, 1);
+    __syncthreads();
+    const int u = *ctl.unit;
+    if (u >= units) break;
+    if (!prep_unit(a, mapK, mapV, mapW, u / a.Hv, u % a.Hv, sm, tmem, par, a.ws.ready)) break;
+    par ^= 1;
+    __syncthreads();  // shared memory and the unit slot are reused
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid < 32) tmem_dealloc(tmem, 256);
 }
 
 // ----------------------------------------------------------------------------------- out
@@ -1017,7 +1205,10 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
 
   const int c = a.c0 + blockIdx.x, h = blockIdx.y;
   const int total_chunks = a.ws.seq_first[a.N];
-  if (c >= total_chunks) return;
+  if (c >= total_chunks) {
+    pdl_wait();
+    return;
+  }
   const ChunkInfo ci = a.ws.chunks[c];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int quarter = warp & 3, half = warp >> 2;
@@ -1025,7 +1216,9 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
   const bool valid = i < ci.L;
   const int Hv = a.Hv;
   const int hk = h / (Hv / a.Hk);
-  if (tid == 0) {
+  // Q, K (q/k/v kernel) and the gates (prep) are complete before the chain starts, so their
+  // loads go out at once; U comes from the chain, which thread 32 waits for
+  if (tid == 32) {
     mbar_init(bar_qk, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_u, 1);
@@ -1037,6 +1230,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
     tma_load_2d(sm + kOutQ + kTile, &mapQ, bar_qk, 64, rowQK);
     tma_load_2d(sm + kOutKS, &mapK, bar_qk, 0, rowQK);
     tma_load_2d(sm + kOutKS + kTile, &mapK, bar_qk, 64, rowQK);
+    pdl_wait();
     mbar_arrive_expect_tx(bar_u, 2 * kTile);
     tma_load_2d(sm + kOutU, &mapU, bar_u, 0, rowV);
     tma_load_2d(sm + kOutU + kTile, &mapU, bar_u, 64, rowV);
@@ -1079,6 +1273,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
   if (tid == 0) {  // K is consumed: S^T of this chunk and value head into the same buffer
+    pdl_wait();    // returns at once: thread 32 has seen the chain complete
     const int rowS = (c * Hv + h) * kC;
     mbar_arrive_expect_tx(bar_s, 2 * kTile);
     tma_load_2d(sm + kOutKS, &mapS, bar_s, 0, rowS);
@@ -1224,6 +1419,26 @@ static int env_int(const char* name, int dflt) {
   return (end && *end == 0 && x >= 0 && x < (1 << 20)) ? (int)x : dflt;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while the previous kernel
+// in the stream drains, and waits for it with griddepcontrol.wait before touching its outputs.
+// GDN_PDL=0 turns this off (plain stream order).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, Args&&... args) {
+  static const bool enabled = env_int("GDN_PDL", 1) != 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (pdl && enabled) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Software pipeline over the chunk table.  The chunk range [0, NCmax) (NCmax = T/128 + N, an
 // upper bound on the chunks the table can hold) is cut into `nseg` segments of `seg` chunks.
 // Segment k's q/k/v + prep run while the chain works on segment k-1 and out on segment k-2, so
@@ -1249,7 +1464,7 @@ static SegPlan seg_plan(int N, int T) {
 }
 
 struct WsLayout {
-  size_t chunks, seq_first, Qw, Kw, Ww, Uw, Sw, Gw, carry, total;
+  size_t chunks, seq_first, Qw, Kw, Ww, Uw, Sw, Gw, ready, carry, total;
 };
 
 static WsLayout ws_layout(int N, int T, int Hk, int Hv) {
@@ -1266,6 +1481,7 @@ static WsLayout ws_layout(int N, int T, int Hk, int Hv) {
   l.Uw = o; o = align_up(o + NC * Hv * tile, 1024);
   l.Sw = o; o = align_up(o + NC * Hv * tile, 1024);
   l.Gw = o; o = align_up(o + NC * Hv * kC * 4, 1024);
+  l.ready = o; o = align_up(o + NC * Hv * 4 + 4, 1024);  // flags, then the work counter
   // one fp32 [Hv][d][d] state per segment boundary (at most one sequence crosses each)
   l.carry = o; o = align_up(o + (size_t)(p.nseg - 1) * Hv * kD * kD * 4, 1024);
   l.total = o;
@@ -1315,7 +1531,7 @@ static bool make_map_x(CUtensorMap* m, const void* base, int T, int Cc) {
 
 template <int DV>
 static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW,
-                                const CUtensorMap& mK, cudaStream_t s) {
+                                const CUtensorMap& mK, cudaStream_t s, bool pdl) {
   using Cfg = gdn::ChainCfg<DV>;
   static bool attr = false;
   if (!attr) {
@@ -1325,9 +1541,10 @@ static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW
     attr = true;
   }
   trace_begin("gdn_chain", s);
-  gdn::gdn_chain_kernel<DV><<<a.N * a.Hv * a.nsplit, Cfg::kThreads, Cfg::kSmem, s>>>(a, mW, mK);
+  cudaError_t e = launch_k(pdl, gdn::gdn_chain_kernel<DV>, dim3(a.N * a.Hv * a.nsplit),
+                           dim3(Cfg::kThreads), Cfg::kSmem, s, a, mW, mK);
   trace_end(s);
-  return cudaGetLastError();
+  return e;
 }
 
 int choose_nsplit(int N, int Hv) {
@@ -1383,6 +1600,34 @@ static cudaError_t pipe_streams(PipeStreams** out) {
   return cudaSuccess;
 }
 
+// Grid of the persistent prep + chain kernel: two CTAs per SM.  Its shape (256 threads of at most
+// 128 registers, about 100 KB of shared memory) is built to fit twice on an SM; with fewer
+// resident, the chains (low block indices) still leave slots to the workers, only fewer.
+static cudaError_t fused_slots(int* grid) {
+  static_assert(gdn::fused_smem<32>() + 1024 <= 232448 / 2, "two CTAs per SM");
+  constexpr int kMaxDev = 64;
+  static int cached[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (!cached[dev]) {
+    if ((e = cudaFuncSetAttribute(gdn::gdn_prep_chain_kernel<32>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  gdn::fused_smem<32>())) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(gdn::gdn_prep_chain_kernel<32>,
+                                  cudaFuncAttributePreferredSharedMemoryCarveout,
+                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+      return e;
+    int nsm = 0;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    cached[dev] = 2 * nsm;
+  }
+  *grid = cached[dev];
+  return cudaSuccess;
+}
+
 cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t s) {
   const WsLayout l = ws_layout(a.N, a.T, a.Hk, a.Hv);
   const SegPlan plan = seg_plan(a.N, a.T);
@@ -1395,9 +1640,11 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   a.ws.Uw = reinterpret_cast<__nv_bfloat16*>(w + l.Uw);
   a.ws.Sw = reinterpret_cast<__nv_bfloat16*>(w + l.Sw);
   a.ws.Gw = reinterpret_cast<float*>(w + l.Gw);
+  const size_t NC = (size_t)a.T / kC + (size_t)a.N + 1;
+  a.ws.ready = reinterpret_cast<int*>(w + l.ready);
+  a.ws.counter = a.ws.ready + NC * a.Hv;
   float* carry = reinterpret_cast<float*>(w + l.carry);
   const size_t carry_stride = (size_t)a.Hv * kD * kD;
-  const size_t NC = (size_t)a.T / kC + (size_t)a.N + 1;
   CUtensorMap mQ, mK, mW, mU, mS, mX;
   const int Cc = (2 * a.Hk + a.Hv) * kD;
   if (a.T > 0 && !make_map_x(&mX, a.x, a.T, Cc)) return cudaErrorInvalidValue;
@@ -1420,48 +1667,83 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     attr = true;
   }
   cudaError_t e;
+  // Persistent prep + chain (one launch), opt-in with GDN_FUSED=1: one chain CTA per (sequence,
+  // value head, 32-column block), the other SM slots as prep workers.  It hides the chain
+  // behind prep, but a chain step sharing its SM with a worker (and acquiring the ready flag)
+  // takes about twice as long as alone, so at the Qwen3-Next shape with T = 4096 it measured
+  // slower than the separate launches (177 us against 64 + 64 us); off by default.
+  int fused_grid = 0, nchain = 0;
+  if (plan.nseg <= 1 && a.T > 0 && env_int("GDN_FUSED", 0) != 0) {
+    if ((e = fused_slots(&fused_grid)) != cudaSuccess) return e;
+    nchain = a.N * a.Hv * 4;
+    if (2 * nchain > fused_grid) fused_grid = 0;
+  }
+  const bool fused = fused_grid > 0;
   trace_begin("chunk_schedule", s);
-  gdn::chunk_schedule_kernel<<<1, 1024, 0, s>>>(a.cu, a.N, a.ws);
+  gdn::chunk_schedule_kernel<<<1, 1024, 0, s>>>(a.cu, a.N, a.ws, fused ? (int)(NC * a.Hv) : 0,
+                                                a.conv0, a.convN, Cc);
   trace_end(s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   // one segment's kernels on the given streams
-  auto launch_parallel_front = [&](const gdn::PrefillArgs& sa, cudaStream_t st) -> cudaError_t {
+  // one segment's kernels on the given streams; `pdl` where each follows the previous kernel
+  // of the same stream with no other dependency in between
+  auto launch_parallel_front = [&](const gdn::PrefillArgs& sa, cudaStream_t st,
+                                   bool pdl) -> cudaError_t {
     const unsigned nc = (unsigned)(sa.c1 - sa.c0);
     trace_begin("gdn_qkv", st);
-    gdn::gdn_qkv_kernel<<<dim3(2 * sa.Hk + sa.Hv, nc), 128, gdn::kQkvSmem, st>>>(sa, mX);
+    cudaError_t e2 = launch_k(pdl, gdn::gdn_qkv_kernel, dim3(2 * sa.Hk + sa.Hv, nc), dim3(128),
+                              gdn::kQkvSmem, st, sa, mX);
     trace_end(st);
-    cudaError_t e2 = cudaGetLastError();
     if (e2 != cudaSuccess) return e2;
     trace_begin("gdn_prep", st);
-    gdn::gdn_prep_kernel<<<dim3(nc, sa.Hv), 256, gdn::kPrepSmem, st>>>(sa, mK, mU, mW);
+    e2 = launch_k(pdl, gdn::gdn_prep_kernel, dim3(nc, sa.Hv), dim3(256), gdn::kPrepSmem, st, sa, mK,
+                  mU, mW);
     trace_end(st);
-    return cudaGetLastError();
+    return e2;
   };
-  auto launch_chain_any = [&](gdn::PrefillArgs sa, cudaStream_t st) -> cudaError_t {
+  auto launch_chain_any = [&](gdn::PrefillArgs sa, cudaStream_t st, bool pdl) -> cudaError_t {
     switch (sa.nsplit) {
-      case 4: return launch_chain<32>(sa, mW, mK, st);
-      case 2: return launch_chain<64>(sa, mW, mK, st);
-      default: sa.nsplit = 1; return launch_chain<128>(sa, mW, mK, st);
+      case 4: return launch_chain<32>(sa, mW, mK, st, pdl);
+      case 2: return launch_chain<64>(sa, mW, mK, st, pdl);
+      default: sa.nsplit = 1; return launch_chain<128>(sa, mW, mK, st, pdl);
     }
   };
-  auto launch_out = [&](const gdn::PrefillArgs& sa, cudaStream_t st) -> cudaError_t {
+  auto launch_out = [&](const gdn::PrefillArgs& sa, cudaStream_t st, bool pdl) -> cudaError_t {
     trace_begin("gdn_out", st);
-    gdn::gdn_out_kernel<<<dim3((unsigned)(sa.c1 - sa.c0), sa.Hv), gdn::kOutThreads, gdn::kOutSmem,
-                          st>>>(sa, mQ, mK, mS, mU);
+    cudaError_t e2 = launch_k(pdl, gdn::gdn_out_kernel, dim3((unsigned)(sa.c1 - sa.c0), sa.Hv),
+                              dim3(gdn::kOutThreads), gdn::kOutSmem, st, sa, mQ, mK, mS, mU);
     trace_end(st);
-    return cudaGetLastError();
+    return e2;
   };
 
   const int NCmax = a.T / kC + a.N;
+  if (fused) {
+    a.c0 = 0;
+    a.c1 = NCmax;
+    a.carry_in = nullptr;
+    a.carry_out = nullptr;
+    a.nsplit = 4;
+    trace_begin("gdn_qkv", s);
+    e = launch_k(true, gdn::gdn_qkv_kernel, dim3(2 * a.Hk + a.Hv, NCmax), dim3(128), gdn::kQkvSmem,
+                 s, a, mX);
+    trace_end(s);
+    if (e != cudaSuccess) return e;
+    trace_begin("gdn_prep_chain", s);
+    e = launch_k(true, gdn::gdn_prep_chain_kernel<32>, dim3(fused_grid), dim3(256),
+                 gdn::fused_smem<32>(), s, a, mK, mU, mW, nchain);
+    trace_end(s);
+    if (e != cudaSuccess) return e;
+    return launch_out(a, s, true);
+  }
   if (plan.nseg <= 1) {
     a.c0 = 0;
     a.c1 = NCmax;
     a.carry_in = nullptr;
     a.carry_out = nullptr;
-    if (a.T > 0 && (e = launch_parallel_front(a, s)) != cudaSuccess) return e;
-    if ((e = launch_chain_any(a, s)) != cudaSuccess) return e;
-    if (a.T > 0 && (e = launch_out(a, s)) != cudaSuccess) return e;
+    if (a.T > 0 && (e = launch_parallel_front(a, s, true)) != cudaSuccess) return e;
+    if ((e = launch_chain_any(a, s, a.T > 0)) != cudaSuccess) return e;
+    if (a.T > 0 && (e = launch_out(a, s, true)) != cudaSuccess) return e;
     return cudaSuccess;
   }
 
@@ -1484,13 +1766,13 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     sa.carry_in = k > 0 ? carry + (size_t)(k - 1) * carry_stride : nullptr;
     sa.carry_out = k + 1 < plan.nseg ? carry + (size_t)k * carry_stride : nullptr;
     cudaStream_t P = ps->P[k % W], O = ps->O[k % W];
-    if ((e = launch_parallel_front(sa, P)) != cudaSuccess) return e;
+    if ((e = launch_parallel_front(sa, P, false)) != cudaSuccess) return e;
     if ((e = cudaEventRecord(ps->evP, P)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(ps->C, ps->evP, 0)) != cudaSuccess) return e;
-    if ((e = launch_chain_any(sa, ps->C)) != cudaSuccess) return e;
+    if ((e = launch_chain_any(sa, ps->C, false)) != cudaSuccess) return e;
     if ((e = cudaEventRecord(ps->evC, ps->C)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(O, ps->evC, 0)) != cudaSuccess) return e;
-    if ((e = launch_out(sa, O)) != cudaSuccess) return e;
+    if ((e = launch_out(sa, O, false)) != cudaSuccess) return e;
   }
   // join: s continues after every helper stream
   for (int i = 0; i < 2 * W + 1; ++i)

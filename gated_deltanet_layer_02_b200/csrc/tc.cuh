@@ -74,6 +74,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Orders this thread's global accesses in the generic proxy with those of the async proxy (TMA).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Bounded wait until *flag is non-zero (acquire), then a proxy fence so that TMA loads issued
+// afterwards see what the flag publishes.  Returns false after kWaitLimitNs.
+__device__ __forceinline__ bool wait_flag(const int* flag) {
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_gpu(flag) == 0) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
 // 2-D tiled TMA load, completion signalled on `bar` (transaction bytes).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y) {
@@ -254,6 +278,38 @@ __device__ __forceinline__ void st_row8_bf16(uint8_t* base, uint32_t tile_bytes,
   uint8_t* dst = base + (chunk16 >> 3) * tile_bytes + sw128_off(row, chunk16 & 7u);
   *reinterpret_cast<uint4*>(dst) = p;
 }
+
+// Programmatic dependent launch.  pdl_wait: the calling thread waits until the grids this grid
+// depends on have completed and their memory is visible (returns at once without the launch
+// attribute).  pdl_trigger: lets the dependent grid be scheduled once every CTA of this grid
+// has triggered or exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Named barrier `id` over the first `n` threads (a multiple of 32), and its OR-reduction.
+__device__ __forceinline__ void bar_sync_n(int id, int n) {
+  asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ bool bar_or_n(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

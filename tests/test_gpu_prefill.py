@@ -7,7 +7,7 @@ import torch
 
 import gated_deltanet_layer_02_b200 as gdn
 from gated_deltanet_layer_02_b200 import inputs
-from gpu_util import assert_close, gpu_prefill, np64, oracle_prefill
+from gpu_util import assert_close, dev, dims_of, gpu_prefill, np64, oracle_prefill
 
 pytestmark = pytest.mark.gpu
 
@@ -133,3 +133,44 @@ def test_bf16_pipelined_matches_single_launch_bitwise(pipeline_env):
     seg = gpu_prefill(w, inp)
     for a, b, name in zip(one, seg, ("out", "final state", "conv state")):
         assert torch.equal(a, b), name
+
+
+@pytest.mark.parametrize("lengths", [(300,), (1, 0, 700, 129), (2000,)])
+def test_bf16_fused_prep_and_chain(monkeypatch, lengths):
+    # The opt-in persistent prep + chain kernel (chains waiting on flags the prep workers set).
+    monkeypatch.setenv("GDN_FUSED", "1")
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=lengths, s0_std=0.1)
+    _check(w, inputs.prefill_inputs(w, 1400 + len(lengths), with_conv0=True), f"fused {lengths}")
+
+
+def test_bf16_fused_matches_separate_launches_bitwise(monkeypatch):
+    # The persistent prep + chain kernel runs the same arithmetic as the separate launches with
+    # 32-column chain blocks; only the schedule differs.
+    w = inputs.custom(16, 32, 128, torch.bfloat16, lengths=(1500,), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 1450, with_conv0=True)
+    monkeypatch.setenv("GDN_FUSED", "0")
+    monkeypatch.setenv("GDN_CHAIN_SPLIT", "4")
+    sep = gpu_prefill(w, inp)
+    monkeypatch.setenv("GDN_FUSED", "1")
+    fused = gpu_prefill(w, inp)
+    for x, y, name in zip(sep, fused, ("out", "final state", "conv state")):
+        assert torch.equal(x, y), name
+
+
+def test_bf16_states_updated_in_place():
+    # SN = S0 and convN = conv0: the call reads the initial states and overwrites them, as a
+    # serving loop does; the conv history then comes from its own kernel after the layer.
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300, 0, 2, 129), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 1500, with_conv0=True)
+    ref_o, ref_S, ref_c = oracle_prefill(w, inp)
+    S = dev(inp["S0"]).clone()
+    conv = dev(inp["conv0"]).clone()
+    out, SN, convN = gdn.chunk_prefill(
+        dev(inp["x"]), dev(inp["beta"]), dev(inp["g"]), dev(inp["cu_seqlens"]),
+        conv_w=dev(inp["conv_w"]), z=dev(inp["z"]), norm_w=dev(inp["norm_w"]), S0=S, SN=S,
+        conv0=conv, convN=conv, dims=dims_of(w))
+    torch.cuda.synchronize()
+    assert SN.data_ptr() == S.data_ptr() and convN.data_ptr() == conv.data_ptr()
+    assert_close(out, ref_o, w.dtype, "in place: out")
+    assert_close(S, ref_S, w.dtype, "in place: final state")
+    np.testing.assert_array_equal(np64(conv), ref_c)
