@@ -40,22 +40,28 @@ L2_FLUSH_BYTES = 256 << 20
 # --------------------------------------------------------------------------- work per token
 def flops_per_token_by_kernel(w, C=CHUNK):
     """Useful (triangle-masked) chunk-form FLOPs per token, split by the kernel that does them.
-    Their sum is F(C) = 2 [Hv (3 d^2 + 1.5 C d + C^2/6) + Hk C d]."""
+    Their sum is F(C) = 2 [Hv (3 d^2 + 1.5 C d + C^2/6) + Hk C d].  The q/k/v kernel (conv,
+    SiLU, norms) does no contraction."""
     Hv, Hk, d = w.num_v_heads, w.num_k_heads, w.head_dim
-    return {
+    f = {
+        "gdn_qkv": 0.0,
         "gdn_prep": 2.0 * (Hv * (C * d + C * C / 6.0) + Hk * C * d / 2.0),   # K K^T, solve, W, U~
         "gdn_chain": 2.0 * (Hv * 2.0 * d * d),                               # W S^T, K^T U
         "gdn_out": 2.0 * (Hv * (d * d + C * d / 2.0) + Hk * C * d / 2.0),    # Q K^T, Q S^T, P U
     }
+    f["gdn_prep_chain"] = f["gdn_prep"] + f["gdn_chain"]  # the opt-in persistent kernel
+    return f
 
 
 def bytes_per_token_by_kernel(w):
     """Algorithmic HBM bytes per token (the layer's own inputs and outputs), by the kernel that
-    moves them: x, beta, g in prep; z in, output out in gdn_out."""
+    moves them: x in gdn_qkv; beta, g in gdn_prep; z in and the output in gdn_out."""
     esz = 2 if w.dtype == torch.bfloat16 else 4
     Hv, d = w.num_v_heads, w.head_dim
-    return {"gdn_prep": w.channels * esz + 2 * Hv * 4, "gdn_chain": 0,
-            "gdn_out": 2 * Hv * d * esz}
+    b = {"gdn_qkv": w.channels * esz, "gdn_prep": 2 * Hv * 4, "gdn_chain": 0,
+         "gdn_out": 2 * Hv * d * esz}
+    b["gdn_prep_chain"] = b["gdn_prep"]
+    return b
 
 
 def load_peaks():
@@ -403,8 +409,8 @@ def main():
                 "unit": "TFLOP/s", "frac": dk["tc_frac"]}
     roof.update({"kernel": dom, "traffic": ncu_traffic(dom),
                  "peak_source": f"{peak_src} ({'burst bf16' if roof['bound'] == 'tensor' else 'copy'})"})
-    F = sum(fl.values())
-    B = sum(by.values())
+    F = sum(v for k, v in fl.items() if k != "gdn_prep_chain")
+    B = sum(v for k, v in by.items() if k != "gdn_prep_chain")
     step_roof = {"tc_frac": F * value / n / (peaks["bf16_tflops"] * 1e12),
                  "hbm_frac": B * value / n / (peaks["hbm_gbs"] * 1e9),
                  "flops_per_token": F, "bytes_per_token": B, "chunk": CHUNK,

@@ -14,7 +14,11 @@ substitute it into u_i = beta_i (v_i - alpha_i S_(i-1) k_i).
 The kernels also rely on two facts checked here:
   * padding a partial chunk with k = q = v = 0, beta = 0, g = 0 leaves every result unchanged;
   * the 128-token inverse can be assembled from the two 64-token diagonal inverses:
-    T = T_h - T_h N T_h, T_h = blockdiag((I + A_00)^-1, (I + A_11)^-1), N = lower-left block of A.
+    T = T_h - T_h N T_h, T_h = blockdiag((I + A_00)^-1, (I + A_11)^-1), N = lower-left block of A;
+  * each 64-token inverse from its two 32-token diagonal inverses, both at once:
+    T_h = D - D L1 D, D = blockdiag of the four 32-token inverses, L1 = the blocks (1,0) and
+    (3,2) of A (exact: (L1 D)^2 = 0 inside each 64-token block);
+  * the 32-token inverses by row substitution T[l] = e_l - sum_{j<l} A[l][j] T[j].
 """
 import numpy as np
 import pytest
@@ -107,4 +111,34 @@ def test_block_inverse_assembly(g_low):
     N = np.zeros((C, C))
     N[h:, :h] = A[h:, :h]
     T = Th - Th @ N @ Th
+    np.testing.assert_allclose(T, np.linalg.inv(np.eye(C) + A), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("g_low", [-0.05, -1.0])
+def test_two_level_block_inverse_assembly(g_low):
+    # the order the prep kernel uses: 32-token blocks by row substitution, joined in pairs by
+    # D - D L1 D, then the two 64-token halves by T_h - T_h N T_h
+    r = np.random.default_rng(62)
+    C, d = 128, 128
+    K = r.standard_normal((C, d)) + 0.5
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    b = r.uniform(0, 1, C)
+    G = np.cumsum(r.uniform(g_low, 0, C))
+    A = b[:, None] * _masked_decay(G, True) * (K @ K.T)
+    D = np.zeros((C, C))
+    for q in range(4):
+        blk = A[32 * q:32 * q + 32, 32 * q:32 * q + 32]
+        T = np.zeros((32, 32))
+        for l in range(32):  # row substitution, as the warps do it
+            T[l] = np.eye(32)[l] - blk[l, :l] @ T[:l]
+        D[32 * q:32 * q + 32, 32 * q:32 * q + 32] = T
+    L1 = np.zeros((C, C))
+    L1[32:64, 0:32] = A[32:64, 0:32]
+    L1[96:128, 64:96] = A[96:128, 64:96]
+    Th = D - D @ L1 @ D
+    N = np.zeros((C, C))
+    N[64:, :64] = A[64:, :64]
+    T = Th - Th @ N @ Th
+    np.testing.assert_allclose(Th[:64, :64], np.linalg.inv(np.eye(64) + A[:64, :64]),
+                               rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(T, np.linalg.inv(np.eye(C) + A), rtol=1e-10, atol=1e-12)
