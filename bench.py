@@ -414,7 +414,8 @@ def main():
     step_roof = {"tc_frac": F * value / n / (peaks["bf16_tflops"] * 1e12),
                  "hbm_frac": B * value / n / (peaks["hbm_gbs"] * 1e9),
                  "flops_per_token": F, "bytes_per_token": B, "chunk": CHUNK,
-                 "flops_per_token_chunk64": sum(flops_per_token_by_kernel(w, 64).values())}
+                 "flops_per_token_chunk64": sum(v for k, v in flops_per_token_by_kernel(w, 64).items()
+                                                if k != "gdn_prep_chain")}
 
     dec_ms, dec_bytes, dec_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev, gdn,
                                               args.decode_steps)
