@@ -42,6 +42,17 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
   const T* w = static_cast<const T*>(a.conv_w);
   T* cs = static_cast<T*>(a.conv_state) + (size_t)slot * 3 * Cc;
 
+  // the first batch of state rows does not depend on q and k: its loads go out before the conv
+  const int rows_per_warp = R * d / (kDecodeThreads / 32);
+  const int nbatch = rows_per_warp / kRowBatch;
+  auto row_ptr = [&](int gr) {
+    const int hr = gr / d, v = gr % d;
+    return reinterpret_cast<float4*>(a.S + (((size_t)slot * a.Hv + hk * R + hr) * d + v) * d) + lane;
+  };
+  float4 sv[kRowBatch], sn[kRowBatch];
+#pragma unroll
+  for (int i = 0; i < kRowBatch; ++i) sv[i] = __ldcs(row_ptr(warp * rows_per_warp + i));
+
   // ---- conv + SiLU with in-place history shift: 2 channels per item
   const int items = (2 + R) * d / 2;
   for (int it = tid; it < items; it += kDecodeThreads) {
@@ -85,19 +96,14 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
     qreg[j] = y_s[4 * lane + j] * rq;
   }
 
-  // ---- state pass: R*d rows split over the warps
-  const int rows_total = R * d;
-  const int rows_per_warp = rows_total / (kDecodeThreads / 32);
-  for (int r0 = warp * rows_per_warp; r0 < (warp + 1) * rows_per_warp; r0 += kRowBatch) {
-    float4 sv[kRowBatch];
-    float dk[kRowBatch], dq[kRowBatch];
+  // ---- state pass: R*d rows split over the warps, two batches of rows in flight
+  for (int bt = 0; bt < nbatch; ++bt) {
+    const int r0 = warp * rows_per_warp + bt * kRowBatch;
+    if (bt + 1 < nbatch) {
 #pragma unroll
-    for (int i = 0; i < kRowBatch; ++i) {
-      const int gr = r0 + i, hr = gr / d, v = gr % d;
-      const int h = hk * R + hr;
-      const float4* p = reinterpret_cast<const float4*>(a.S + (((size_t)slot * a.Hv + h) * d + v) * d) + lane;
-      sv[i] = __ldcs(p);
+      for (int i = 0; i < kRowBatch; ++i) sn[i] = __ldcs(row_ptr(r0 + kRowBatch + i));
     }
+    float dk[kRowBatch], dq[kRowBatch];
 #pragma unroll
     for (int i = 0; i < kRowBatch; ++i) {
       dk[i] = sv[i].x * kreg[0] + sv[i].y * kreg[1] + sv[i].z * kreg[2] + sv[i].w * kreg[3];
@@ -125,9 +131,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
       nv.y = alpha * sv[i].y + u * kreg[1];
       nv.z = alpha * sv[i].z + u * kreg[2];
       nv.w = alpha * sv[i].w + u * kreg[3];
-      float4* p = reinterpret_cast<float4*>(a.S + (((size_t)slot * a.Hv + h) * d + v) * d) + lane;
-      __stcs(p, nv);
+      __stcs(row_ptr(gr), nv);
     }
+#pragma unroll
+    for (int i = 0; i < kRowBatch; ++i) sv[i] = sn[i];
   }
   __syncthreads();
   // ---- gated RMSNorm (or plain output), one warp per value head
