@@ -74,28 +74,35 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_hash():
+# source files of each kernel family (a change to any of them invalidates its ncu traffic figure)
+KERNEL_SOURCES = {
+    "prefill": ("prefill_tc.cu", "args.cuh", "common.cuh", "tc.cuh"),
+    "decode_step": ("decode.cu", "args.cuh", "common.cuh"),
+}
+
+
+def source_hash(family="prefill"):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_deltanet_layer_02_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(f.read())
+    for name in KERNEL_SOURCES[family]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel sources are unchanged."""
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's sources are unchanged."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             t = json.load(f)
     except Exception:
         return None
-    if t.get("source_hash") != source_hash():
-        return None
     k = t.get("kernels", {}).get(kernel)
-    return None if k is None else float(k["dram_bytes_per_launch_full_size"])
+    family = "decode_step" if kernel == "decode_step" else "prefill"
+    if k is None or k.get("source_hash") != source_hash(family):
+        return None
+    return float(k["dram_bytes_per_launch_full_size"])
 
 
 # ------------------------------------------------------------------------------- clocks
