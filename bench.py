@@ -308,9 +308,9 @@ def bench_prefill(args, w, seed, dev, gdn):
     return step_ms, recs, clk.summary(), (statistics.mean(e2e_ms), h2d, d2h), statistics.mean(eager_ms)
 
 
-def bench_decode(w, seed, dev, gdn, steps):
+def bench_decode(w, seed, dev, gdn, steps, state_dtype=torch.float32):
     st = inputs.decode_state(w, seed)
-    S, cs = st["S"].to(dev), st["conv_state"].to(dev)
+    S, cs = st["S"].to(dev).to(state_dtype), st["conv_state"].to(dev)
     cw, nw = st["conv_w"].to(dev), st["norm_w"].to(dev)
     dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
     steps_in = [{k: v.to(dev) for k, v in inputs.decode_step_inputs(w, seed, s).items()}
@@ -330,7 +330,7 @@ def bench_decode(w, seed, dev, gdn, steps):
             ev[i][1].record()
         torch.cuda.synchronize()
     ms = [a.elapsed_time(b) for a, b in ev]
-    state_bytes = 2 * S.numel() * 4
+    state_bytes = 2 * S.numel() * S.element_size()
     return statistics.median(ms), state_bytes, clk.summary()
 
 
@@ -428,13 +428,25 @@ def main():
                                               args.decode_steps)
     dec_ms = max_over_ranks([dec_ms], dev)[0]
     dec_gbs = n * dec_bytes / (dec_ms * 1e-3) / 1e9
+    # the serving option of a bf16 recurrent state (same workload, half the state bytes)
+    d16_ms, d16_bytes, d16_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev, gdn,
+                                              args.decode_steps, torch.bfloat16)
+    d16_ms = max_over_ranks([d16_ms], dev)[0]
+    d16_gbs = n * d16_bytes / (d16_ms * 1e-3) / 1e9
     decode = {"workload": inputs.CONFIGS[3].name, "value": dec_gbs, "unit": "GB/s",
               "ms_per_step": dec_ms, "steps": args.decode_steps,
               "roofline": {"bound": "hbm", "achieved": dec_gbs / n, "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": dec_gbs / n / peaks["hbm_gbs"],
                            "traffic": ncu_traffic("decode_step"),
                            "peak_source": f"{peak_src} (copy)"},
-              "clocks": dec_clk}
+              "clocks": dec_clk,
+              "bf16_state": {"value": d16_gbs, "unit": "GB/s", "ms_per_step": d16_ms,
+                             "sequence_steps_per_s": n * inputs.CONFIGS[3].batch / (d16_ms * 1e-3),
+                             "roofline": {"bound": "hbm", "achieved": d16_gbs / n,
+                                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                          "frac": d16_gbs / n / peaks["hbm_gbs"],
+                                          "traffic": None, "peak_source": f"{peak_src} (copy)"},
+                             "clocks": d16_clk}}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -29,7 +29,7 @@ EXPORTS = (
     "gdn_gated_rmsnorm", "gdn_chunk_prefill_workspace_size", "gdn_chunk_prefill",
     "gdn_decode_step", "gdn_trace_create", "gdn_trace_destroy", "gdn_trace_attach",
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
-    "gdn_chunk_prefill_static_ws", "gdn_trace_span",
+    "gdn_chunk_prefill_static_ws", "gdn_trace_span", "gdn_decode_step_bf16_state",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
@@ -85,6 +85,7 @@ def lib():
                                             vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
             L.gdn_decode_step.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                           vp, vp]
+            L.gdn_decode_step_bf16_state.argtypes = L.gdn_decode_step.argtypes
             L.gdn_trace_create.argtypes = [ctypes.POINTER(vp)]
             L.gdn_trace_destroy.argtypes = [vp]
             L.gdn_trace_attach.argtypes = [vp]
@@ -246,18 +247,21 @@ def chunk_prefill_static_ws(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=
 
 def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx=None,
                 out=None, dims: Dims | None = None):
-    """One token per sequence; conv_state and S are updated in place.  Returns out [B, Hv, d]."""
+    """One token per sequence; conv_state and S are updated in place.  Returns out [B, Hv, d].
+    S may be fp32 (gdn_decode_step) or bf16 (gdn_decode_step_bf16_state)."""
     dims = dims or Dims()
     dt = _act_dtype(x)
     B = x.shape[0]
     if out is None:
         out = torch.empty((B, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
-    _check("gdn_decode_step", lib().gdn_decode_step(
+    bf16_state = S is not None and S.dtype == torch.bfloat16
+    name = "gdn_decode_step_bf16_state" if bf16_state else "gdn_decode_step"
+    _check(name, getattr(lib(), name)(
         ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype, False),
         _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
         _ptr(norm_w, "norm_w", x.dtype), _ptr(conv_state, "conv_state", x.dtype),
-        _ptr(S, "S", torch.float32), _ptr(slot_idx, "slot_idx", torch.int32), B,
-        _ptr(out, "out", x.dtype), _stream()))
+        _ptr(S, "S", torch.bfloat16 if bf16_state else torch.float32),
+        _ptr(slot_idx, "slot_idx", torch.int32), B, _ptr(out, "out", x.dtype), _stream()))
     return out
 
 

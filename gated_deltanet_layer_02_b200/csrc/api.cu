@@ -18,7 +18,7 @@ cudaError_t launch_conv_state_out(bool bf16, const void* x, const int32_t* cu, i
                                   const void* st_in, void* st_out, cudaStream_t s);
 cudaError_t launch_gated_rmsnorm(bool bf16, const void* o, const void* z, const void* w, float eps,
                                  int rows, int dim, void* y, cudaStream_t s);
-cudaError_t launch_decode(bool bf16, const gdn::DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode(bool bf16, bool state_bf16, const gdn::DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_recurrent_f32(const gdn::RecArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t s);
 size_t prefill_tc_workspace(int N, int T, int Hk, int Hv);
@@ -252,10 +252,13 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
   return map_cuda(e);
 }
 
-int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
-                    const float* beta, const float* g, const void* z, const void* norm_w,
-                    void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
-                    void* out, void* stream) {
+}  // extern "C"
+
+namespace {
+int decode_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
+                const float* beta, const float* g, const void* z, const void* norm_w,
+                void* conv_state, void* S, bool state_bf16, const int32_t* slot_idx,
+                int32_t batch, void* out, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return GDN_ERR_UNSUPPORTED;
@@ -283,7 +286,27 @@ int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const 
   a.q_scale = dims->q_scale;
   a.l2_eps = dims->l2_eps;
   a.norm_eps = dims->norm_eps;
-  return map_cuda(gdn_host::launch_decode(dtype == GDN_BF16, a, static_cast<cudaStream_t>(stream)));
+  return map_cuda(gdn_host::launch_decode(dtype == GDN_BF16, state_bf16, a,
+                                          static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+extern "C" {
+
+int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
+                    const float* beta, const float* g, const void* z, const void* norm_w,
+                    void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
+                    void* out, void* stream) {
+  return decode_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, conv_state, S, false, slot_idx,
+                     batch, out, stream);
+}
+
+int gdn_decode_step_bf16_state(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                               const void* conv_w, const float* beta, const float* g,
+                               const void* z, const void* norm_w, void* conv_state, void* S,
+                               const int32_t* slot_idx, int32_t batch, void* out, void* stream) {
+  return decode_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, conv_state, S, true, slot_idx,
+                     batch, out, stream);
 }
 
 int gdn_trace_create(gdn_trace** out) {

@@ -13,7 +13,7 @@ struct DecodeArgs {
   const void* z;
   const void* norm_w;
   void* conv_state;
-  float* S;
+  void* S;  // fp32 or bf16 (see the decode kernel's state type)
   const int32_t* slot_idx;
   void* out;
   int B, Hk, Hv;

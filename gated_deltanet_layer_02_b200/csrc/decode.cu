@@ -20,11 +20,49 @@
 namespace gdn {
 
 constexpr int kDecodeThreads = 256;
-constexpr int kRowBatch = 8;
 constexpr int kMaxR = 8;
 
+// Four consecutive state elements of a lane: fp32 (16 bytes) or bf16 (8 bytes, the serving
+// option of a bf16 recurrent state: arithmetic stays fp32, the new state is rounded to nearest
+// even once per step).  Loads stay raw until used, so that the bf16 state keeps as many bytes
+// in flight (twice the rows) in the same registers.  Streaming loads and stores: the state is
+// touched once per step.
+template <typename TS>
+struct StateIO;
+template <>
+struct StateIO<float> {
+  using Raw = float4;
+  static constexpr int kRows = 8;  // rows per batch and warp
+  static __device__ __forceinline__ Raw load(const float* p) {
+    return __ldcs(reinterpret_cast<const float4*>(p));
+  }
+  static __device__ __forceinline__ float4 f4(Raw r) { return r; }
+  static __device__ __forceinline__ void store(float* p, float4 v) {
+    __stcs(reinterpret_cast<float4*>(p), v);
+  }
+};
+template <>
+struct StateIO<__nv_bfloat16> {
+  using Raw = uint2;
+  static constexpr int kRows = 16;
+  static __device__ __forceinline__ Raw load(const __nv_bfloat16* p) {
+    return __ldcs(reinterpret_cast<const uint2*>(p));
+  }
+  static __device__ __forceinline__ float4 f4(Raw u) {
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, float4 v) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    __stcs(reinterpret_cast<uint2*>(p), u);
+  }
+};
 
-template <typename T>
+template <typename T, typename TS>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
   constexpr int d = kHeadDim;
   const int b = blockIdx.x / a.Hk;
@@ -43,15 +81,18 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
   T* cs = static_cast<T*>(a.conv_state) + (size_t)slot * 3 * Cc;
 
   // the first batch of state rows does not depend on q and k: its loads go out before the conv
+  using IO = StateIO<TS>;
+  constexpr int kRowBatch = IO::kRows;
   const int rows_per_warp = R * d / (kDecodeThreads / 32);
   const int nbatch = rows_per_warp / kRowBatch;
+  TS* S = static_cast<TS*>(a.S);
   auto row_ptr = [&](int gr) {
     const int hr = gr / d, v = gr % d;
-    return reinterpret_cast<float4*>(a.S + (((size_t)slot * a.Hv + hk * R + hr) * d + v) * d) + lane;
+    return S + (((size_t)slot * a.Hv + hk * R + hr) * d + v) * d + 4 * lane;
   };
-  float4 sv[kRowBatch], sn[kRowBatch];
+  typename IO::Raw sv[kRowBatch], sn[kRowBatch];
 #pragma unroll
-  for (int i = 0; i < kRowBatch; ++i) sv[i] = __ldcs(row_ptr(warp * rows_per_warp + i));
+  for (int i = 0; i < kRowBatch; ++i) sv[i] = IO::load(row_ptr(warp * rows_per_warp + i));
 
   // ---- conv + SiLU with in-place history shift: 2 channels per item
   const int items = (2 + R) * d / 2;
@@ -101,13 +142,14 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
     const int r0 = warp * rows_per_warp + bt * kRowBatch;
     if (bt + 1 < nbatch) {
 #pragma unroll
-      for (int i = 0; i < kRowBatch; ++i) sn[i] = __ldcs(row_ptr(r0 + kRowBatch + i));
+      for (int i = 0; i < kRowBatch; ++i) sn[i] = IO::load(row_ptr(r0 + kRowBatch + i));
     }
     float dk[kRowBatch], dq[kRowBatch];
 #pragma unroll
     for (int i = 0; i < kRowBatch; ++i) {
-      dk[i] = sv[i].x * kreg[0] + sv[i].y * kreg[1] + sv[i].z * kreg[2] + sv[i].w * kreg[3];
-      dq[i] = sv[i].x * qreg[0] + sv[i].y * qreg[1] + sv[i].z * qreg[2] + sv[i].w * qreg[3];
+      const float4 f = IO::f4(sv[i]);
+      dk[i] = f.x * kreg[0] + f.y * kreg[1] + f.z * kreg[2] + f.w * kreg[3];
+      dq[i] = f.x * qreg[0] + f.y * qreg[1] + f.z * qreg[2] + f.w * qreg[3];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -126,12 +168,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
       const float vv = y_s[(2 + hr) * d + v];
       const float u = beta * (vv - alpha * dk[i]);
       if (lane == 0) o_s[hr * d + v] = alpha * dq[i] + u * kq;
+      const float4 f = IO::f4(sv[i]);
       float4 nv;
-      nv.x = alpha * sv[i].x + u * kreg[0];
-      nv.y = alpha * sv[i].y + u * kreg[1];
-      nv.z = alpha * sv[i].z + u * kreg[2];
-      nv.w = alpha * sv[i].w + u * kreg[3];
-      __stcs(row_ptr(gr), nv);
+      nv.x = alpha * f.x + u * kreg[0];
+      nv.y = alpha * f.y + u * kreg[1];
+      nv.z = alpha * f.z + u * kreg[2];
+      nv.w = alpha * f.w + u * kreg[3];
+      IO::store(row_ptr(gr), nv);
     }
 #pragma unroll
     for (int i = 0; i < kRowBatch; ++i) sv[i] = sn[i];
@@ -167,13 +210,19 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
 
 namespace gdn_host {
 
-cudaError_t launch_decode(bool bf16, const gdn::DecodeArgs& a, cudaStream_t s) {
+cudaError_t launch_decode(bool bf16, bool state_bf16, const gdn::DecodeArgs& a,
+                          cudaStream_t s) {
   if (a.B == 0) return cudaSuccess;
-  trace_begin("decode_step", s);
-  if (bf16)
-    gdn::decode_kernel<__nv_bfloat16><<<a.B * a.Hk, gdn::kDecodeThreads, 0, s>>>(a);
+  const dim3 grid(a.B * a.Hk), block(gdn::kDecodeThreads);
+  trace_begin(state_bf16 ? "decode_step_bf16_state" : "decode_step", s);
+  if (bf16 && state_bf16)
+    gdn::decode_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, block, 0, s>>>(a);
+  else if (bf16)
+    gdn::decode_kernel<__nv_bfloat16, float><<<grid, block, 0, s>>>(a);
+  else if (state_bf16)
+    gdn::decode_kernel<float, __nv_bfloat16><<<grid, block, 0, s>>>(a);
   else
-    gdn::decode_kernel<float><<<a.B * a.Hk, gdn::kDecodeThreads, 0, s>>>(a);
+    gdn::decode_kernel<float, float><<<grid, block, 0, s>>>(a);
   trace_end(s);
   return cudaGetLastError();
 }

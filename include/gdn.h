@@ -146,6 +146,20 @@ int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const 
                     void* out, void* stream);
 
 /*
+ * gdn_decode_step_bf16_state -- gdn_decode_step with the recurrent state stored in bf16.
+ * Source: the "Qwen3-Next" SGLang cookbook, section 3.2: --mamba-ssm-dtype selects bf16 or fp32
+ * (the default) for the recurrent state of the GDN layers.  Each step reads the bf16 state,
+ * does all arithmetic in fp32 exactly as gdn_decode_step, and rounds the new state to bf16
+ * (round to nearest even) once when it is written back: half the state bytes of the fp32 call.
+ *   S [slots, Hv, d, d] bf16 in/out (16-byte aligned); every other argument, the layout, the
+ *   ownership and the status codes are those of gdn_decode_step.
+ */
+int gdn_decode_step_bf16_state(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                               const void* conv_w, const float* beta, const float* g,
+                               const void* z, const void* norm_w, void* conv_state, void* S,
+                               const int32_t* slot_idx, int32_t batch, void* out, void* stream);
+
+/*
  * gdn_chunk_prefill_static_ws -- gdn_chunk_prefill for callers that cannot allocate device
  * memory.  No counterpart on the source pages: this is a deployment aid of this library.
  * Some callers have no way to obtain a device workspace: extensions loaded into a host

@@ -69,3 +69,32 @@ def test_decode_config():
     e_s = assert_close(S_d, S_ref, w.dtype, "decode state after 64 steps")
     np.testing.assert_array_equal(np64(cs_d), cs_ref)
     print(f"decode: worst out err {worst:.3g}, state err {e_s:.3g}")
+
+
+def test_decode_config_bf16_state():
+    # the decode workload with the recurrent state stored in bf16: the oracle state is rounded to
+    # bf16 after every step, as the kernel stores it (fp32 arithmetic in between)
+    ensure_built()
+    w = inputs.CONFIGS[3]
+    seed = inputs.config_seed(3)
+    st = inputs.decode_state(w, seed)
+    S_d = dev(st["S"]).to(torch.bfloat16)
+    cs_d = dev(st["conv_state"])
+    S_ref = S_d.double().cpu().numpy().copy()
+    cs_ref = st["conv_state"].double().numpy().copy()
+    cw, nw = dev(st["conv_w"]), dev(st["norm_w"])
+    dims, od = dims_of(w), oracle_dims_of(w)
+    worst = 0.0
+    for step in range(16):
+        s = inputs.decode_step_inputs(w, seed, step)
+        out = gdn.decode_step(dev(s["x"]), dev(s["beta"]), dev(s["g"]), cs_d, S_d, cw,
+                              z=dev(s["z"]), norm_w=nw, dims=dims)
+        torch.cuda.synchronize()
+        ref = oracle.decode_step(od, s["x"], s["beta"], s["g"], cs_ref, S_ref,
+                                 conv_w=st["conv_w"], z=s["z"], norm_w=st["norm_w"])
+        S_ref[...] = torch.from_numpy(S_ref).to(torch.bfloat16).double().numpy()
+        worst = max(worst, assert_close(out, ref, w.dtype, f"bf16-state decode out step {step}"))
+    assert S_d.dtype == torch.bfloat16
+    e_s = assert_close(S_d.float(), S_ref, torch.bfloat16, "bf16 decode state after 16 steps")
+    np.testing.assert_array_equal(np64(cs_d), cs_ref)
+    print(f"bf16-state decode: worst out err {worst:.3g}, state err {e_s:.3g}")
