@@ -106,6 +106,11 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, MIS, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_decode_step(ctypes.byref(gdn.Dims(1, 16)), 1, A, A, A, A, None, None, A, A, None,
                              4, A, None) == gdn.GDN_ERR_UNSUPPORTED
+    bs = L.gdn_decode_step_bf16_state
+    assert bs(d, 1, A, A, A, A, None, None, A, A, None, -1, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert bs(d, 1, A, A, A, A, None, None, A, None, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert bs(d, 1, A, A, A, A, None, None, A, MIS, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
+    assert bs(d, 3, A, A, A, A, None, None, A, A, None, 4, A, None) == gdn.GDN_ERR_UNSUPPORTED
     assert L.gdn_debug_wait_probe(None, 10, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_debug_wait_probe(A, 10_000_000, None) == gdn.GDN_ERR_INVALID_ARG
 
@@ -117,6 +122,8 @@ def test_zero_size_calls_launch_nothing(L):
                                None, None, None, A, 1 << 30, None, None) == gdn.GDN_OK
     assert L.gdn_decode_step(d, 1, None, None, None, None, None, None, None, None, None, 0, None,
                              None) == gdn.GDN_OK
+    assert L.gdn_decode_step_bf16_state(d, 1, None, None, None, None, None, None, None, None,
+                                        None, 0, None, None) == gdn.GDN_OK
     assert L.gdn_gated_rmsnorm(1, None, None, None, 1e-6, 0, 128, None, None) == gdn.GDN_OK
 
 
