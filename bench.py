@@ -308,6 +308,48 @@ def bench_prefill(args, w, seed, dev, gdn):
     return step_ms, recs, clk.summary(), (statistics.mean(e2e_ms), h2d, d2h), statistics.mean(eager_ms)
 
 
+def bench_chunk_states(args, w, seed, dev, gdn):
+    """The prefill step with and without the chunk-boundary states (gdn_chunk_prefill_states),
+    each timed as CUDA-graph replays with L2 flushed in between; extra bytes = the state writes."""
+    inp = inputs.prefill_inputs(w, seed)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    T, N = w.tokens, len(w.lengths)
+    C = sum((int(L) + 127) // 128 for L in w.lengths)
+    cs = torch.empty((C, w.num_v_heads, w.head_dim, w.head_dim), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(N, T, w.dtype, dims), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((T, w.num_v_heads, w.head_dim), dtype=w.dtype, device=dev)
+    SN = torch.empty((N, w.num_v_heads, w.head_dim, w.head_dim), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    res = {}
+    for name, states in (("without", None), ("with", cs)):
+        def step():
+            gdn.chunk_prefill(d["x"], d["beta"], d["g"], d["cu_seqlens"], conv_w=d["conv_w"],
+                              z=d["z"], norm_w=d["norm_w"], S0=d["S0"], SN=SN, out=out,
+                              workspace=ws, dims=dims, chunk_states=states)
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        ms = []
+        for _ in range(max(10, args.steps // 4)):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+        del graph
+        res[name] = statistics.median(ms)
+    return {"workload": w.name, "ms_per_step_without": res["without"],
+            "ms_per_step_with": res["with"], "chunks": C,
+            "extra_bytes_per_step": cs.numel() * 4}
+
+
 def bench_decode(w, seed, dev, gdn, steps, state_dtype=torch.float32):
     st = inputs.decode_state(w, seed)
     S, cs = st["S"].to(dev).to(state_dtype), st["conv_state"].to(dev)
@@ -448,6 +490,8 @@ def main():
                                           "traffic": None, "peak_source": f"{peak_src} (copy)"},
                              "clocks": d16_clk}}
 
+    chunk_states = bench_chunk_states(args, w, seed, dev, gdn)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_rate(w, seed)
@@ -466,7 +510,7 @@ def main():
         "e2e": {"value": job_tokens_per_s(n, T, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": len(recs), "eager_ms_per_step": eager_ms,
-        "clocks": clocks, "decode": decode, "cpu_baseline": cpu,
+        "clocks": clocks, "decode": decode, "chunk_states": chunk_states, "cpu_baseline": cpu,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)

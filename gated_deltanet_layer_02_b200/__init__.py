@@ -30,6 +30,7 @@ EXPORTS = (
     "gdn_decode_step", "gdn_trace_create", "gdn_trace_destroy", "gdn_trace_attach",
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
     "gdn_chunk_prefill_static_ws", "gdn_trace_span", "gdn_decode_step_bf16_state",
+    "gdn_chunk_prefill_states",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
@@ -83,6 +84,9 @@ def lib():
             L.gdn_chunk_prefill_workspace_size.restype = ctypes.c_size_t
             L.gdn_chunk_prefill.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, i32, i32,
                                             vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
+            L.gdn_chunk_prefill_states.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                                   i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                                   ctypes.c_size_t, vp, vp]
             L.gdn_decode_step.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                           vp, vp]
             L.gdn_decode_step_bf16_state.argtypes = L.gdn_decode_step.argtypes
@@ -182,11 +186,13 @@ def prefill_workspace_size(num_seqs: int, num_tokens: int, dtype=torch.bfloat16,
 
 def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None, SN=None,
                   conv0=None, convN=None, out=None, workspace=None, dev_status=None,
-                  want_state=True, dims: Dims | None = None):
+                  want_state=True, dims: Dims | None = None, chunk_states=None):
     """The whole layer over packed sequences.  Returns (out, SN, convN).
 
     x [T, Cc], beta/g [T, Hv] fp32, z [T, Hv, d] or None, cu_seqlens [N+1] int32 (device),
-    S0 [N, Hv, d, d] fp32 or None, conv0 [N, K-1, Cc] or None.
+    S0 [N, Hv, d, d] fp32 or None, conv0 [N, K-1, Cc] or None.  chunk_states [C, Hv, d, d] fp32
+    (C = sum of ceil(L_n / 128)) receives the state after every 128-token chunk
+    (gdn_chunk_prefill_states).
     """
     dims = dims or Dims()
     dt = _act_dtype(x)
@@ -203,14 +209,19 @@ def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=N
     need = prefill_workspace_size(N, T, x.dtype, dims)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
-    _check("gdn_chunk_prefill", lib().gdn_chunk_prefill(
-        ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
-        _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
-        _ptr(norm_w, "norm_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N, T,
-        _ptr(S0, "S0", torch.float32), _ptr(SN, "SN", torch.float32),
-        _ptr(conv0, "conv0", x.dtype), _ptr(convN, "convN", x.dtype), _ptr(out, "out", x.dtype),
-        _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
-        _ptr(dev_status, "dev_status", torch.int32), _stream()))
+    head = (ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
+            _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
+            _ptr(norm_w, "norm_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N, T,
+            _ptr(S0, "S0", torch.float32), _ptr(SN, "SN", torch.float32),
+            _ptr(conv0, "conv0", x.dtype), _ptr(convN, "convN", x.dtype),
+            _ptr(out, "out", x.dtype))
+    tail = (_ptr(workspace, "workspace", torch.uint8), workspace.numel(),
+            _ptr(dev_status, "dev_status", torch.int32), _stream())
+    if chunk_states is None:
+        _check("gdn_chunk_prefill", lib().gdn_chunk_prefill(*head, *tail))
+    else:
+        _check("gdn_chunk_prefill_states", lib().gdn_chunk_prefill_states(
+            *head, _ptr(chunk_states, "chunk_states", torch.float32), *tail))
     return out, SN, convN
 
 

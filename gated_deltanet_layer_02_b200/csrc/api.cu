@@ -173,12 +173,12 @@ size_t gdn_chunk_prefill_workspace_size(const gdn_dims* dims, gdn_dtype dtype, i
                                         dims->num_v_heads);
 }
 
-int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
-                      const float* beta, const float* g, const void* z, const void* norm_w,
-                      const int32_t* cu_seqlens, int32_t num_seqs, int32_t num_tokens,
-                      const float* S0, float* SN, const void* conv0, void* convN, void* out,
-                      void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                      void* stream) {
+static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                        const void* conv_w, const float* beta, const float* g, const void* z,
+                        const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
+                        int32_t num_tokens, const float* S0, float* SN, const void* conv0,
+                        void* convN, void* out, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, float* chunk_states, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return GDN_ERR_UNSUPPORTED;
@@ -186,11 +186,12 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
   if (num_seqs == 0 && num_tokens > 0) return GDN_ERR_INVALID_ARG;
   if (num_seqs > 0 && !cu_seqlens) return GDN_ERR_INVALID_ARG;
   if (num_tokens > 0 && (!x || !beta || !g || !out)) return GDN_ERR_INVALID_ARG;
-  const void* ptrs[] = {x, conv_w, beta, g, z, norm_w, S0, SN, conv0, convN, out};
+  const void* ptrs[] = {x, conv_w, beta, g, z, norm_w, S0, SN, conv0, convN, out, chunk_states};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GDN_ERR_INVALID_ARG;
   const bool bf16 = dtype == GDN_BF16;
+  if (chunk_states && !bf16) return GDN_ERR_UNSUPPORTED;  // the fp32 path has no chunks
   if (bf16 && dims->num_v_heads != 2 * dims->num_k_heads) return GDN_ERR_UNSUPPORTED;
   const size_t need = gdn_chunk_prefill_workspace_size(dims, dtype, num_seqs, num_tokens);
   if (bf16 && (!workspace || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
@@ -233,6 +234,7 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
   a.SN = SN;
   a.conv0 = static_cast<const __nv_bfloat16*>(conv0);
   a.out = static_cast<__nv_bfloat16*>(out);
+  a.chunk_states = chunk_states;
   a.status = dev_status;
   a.N = num_seqs;
   a.T = num_tokens;
@@ -250,6 +252,30 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
   if (e == cudaSuccess && separate_conv_state)
     e = gdn_host::launch_conv_state_out(true, x, cu_seqlens, num_seqs, Cc, conv0, convN, s);
   return map_cuda(e);
+}
+
+int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
+                      const float* beta, const float* g, const void* z, const void* norm_w,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int32_t num_tokens,
+                      const float* S0, float* SN, const void* conv0, void* convN, void* out,
+                      void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                      void* stream) {
+  return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
+                      num_tokens, S0, SN, conv0, convN, out, workspace, workspace_bytes,
+                      dev_status, nullptr, stream);
+}
+
+int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                             const void* conv_w, const float* beta, const float* g,
+                             const void* z, const void* norm_w, const int32_t* cu_seqlens,
+                             int32_t num_seqs, int32_t num_tokens, const float* S0, float* SN,
+                             const void* conv0, void* convN, void* out, float* chunk_states,
+                             void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                             void* stream) {
+  if (num_tokens > 0 && !chunk_states) return GDN_ERR_INVALID_ARG;
+  return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
+                      num_tokens, S0, SN, conv0, convN, out, workspace, workspace_bytes,
+                      dev_status, chunk_states, stream);
 }
 
 }  // extern "C"

@@ -67,6 +67,7 @@ struct PrefillArgs {
   __nv_bfloat16* convN;  // written by the q/k/v kernel (and the chunk table for empty sequences)
                          // when set; NULL when the caller wants none or it aliases conv0
   __nv_bfloat16* out;
+  float* chunk_states;  // [chunks][Hv][d_v][d_k] fp32: state after each chunk, or NULL
   int32_t* status;
   int N, T, Hk, Hv, nsplit;
   float q_scale, l2_eps, norm_eps;

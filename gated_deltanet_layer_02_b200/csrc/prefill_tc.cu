@@ -940,6 +940,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     for (int gi = 0; gi < kGroups; ++gi) {
       tmem_ld32(lane_addr + colS + cs + gi * 32, sreg[gi]);
       tmem_ld_wait();
+
 #pragma unroll
       for (int q = 0; q < 4; ++q)
         st_row8_bf16(OP, kTile, k_row, (cs + gi * 32 + 8 * q) >> 3, sreg[gi] + 8 * q);
@@ -1072,6 +1073,18 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
+    if (a.chunk_states) {
+      // the state after chunk c (fp32, layout [v][k]), for prefix and branch caching
+      float* cst = a.chunk_states + (((size_t)c * a.Hv + h) * kD + v0 + cs) * kD + k_row;
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) {
+        float v[32];
+        tmem_ld32(lane_addr + colS + cs + gi * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) cst[(gi * 32 + e) * kD] = v[e];
+      }
+    }
     // the update has consumed K and the operand tile
     if (tid == 0 && ci + 1 < nch) {
       issue_k(ci + 1);

@@ -131,6 +131,28 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * gdn_chunk_prefill_states -- gdn_chunk_prefill that also returns the recurrent state after
+ * every chunk (128 tokens, the last chunk of a sequence possibly shorter).
+ * Source: the "Qwen3-Next" SGLang cookbook, section 3.2: the radix cache of the hybrid GDN
+ * layers keeps states at branching points, with a page size that divides or is divided by the
+ * kernel's chunk; a prefill that emits the chunk-boundary states supplies them.
+ *   chunk_states [C, Hv, d, d] fp32 (layout as SN), C = sum over sequences of ceil(L_n / 128);
+ *     entry c is the state after chunk c, chunks numbered sequence by sequence (sequence n's
+ *     chunk j, covering its tokens [128 j, min(128 (j + 1), L_n)), is c = j + sum_{m<n}
+ *     ceil(L_m / 128)); required when num_tokens > 0, 16-byte aligned.  The entry of a
+ *     sequence's last chunk equals its final state.
+ * bf16 only (GDN_ERR_UNSUPPORTED for GDN_F32).  Every other argument, the workspace size and
+ * the status codes are those of gdn_chunk_prefill.  The extra cost is the write of C Hv d^2 fp32.
+ */
+int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                             const void* conv_w, const float* beta, const float* g,
+                             const void* z, const void* norm_w, const int32_t* cu_seqlens,
+                             int32_t num_seqs, int32_t num_tokens, const float* S0, float* SN,
+                             const void* conv0, void* convN, void* out, float* chunk_states,
+                             void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                             void* stream);
+
+/*
  * gdn_decode_step -- one token for each of B sequences; conv and recurrent state in place.
  * Source: as gdn_chunk_prefill with T = 1 per sequence; states resident in a slot pool, fp32
  * recurrent state as the "Qwen3-Next" SGLang cookbook's default --mamba-ssm-dtype.

@@ -174,3 +174,39 @@ def test_bf16_states_updated_in_place():
     assert_close(out, ref_o, w.dtype, "in place: out")
     assert_close(S, ref_S, w.dtype, "in place: final state")
     np.testing.assert_array_equal(np64(conv), ref_c)
+
+
+@pytest.mark.parametrize("seg,split", [(0, 0), (1, 4), (2, 1)])
+def test_bf16_chunk_boundary_states(pipeline_env, seg, split):
+    # gdn_chunk_prefill_states: entry c is the state after chunk c of the sequence-by-sequence
+    # chunk numbering; the oracle gives it as the final state of the prefix ending there
+    if seg:
+        pipeline_env(seg, split)
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300, 0, 129, 256, 5), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 1600 + seg, with_conv0=True)
+    lengths = [int(v) for v in w.lengths]
+    C = sum((L + 127) // 128 for L in lengths)
+    cs = torch.full((C, w.num_v_heads, 128, 128), float("nan"), dtype=torch.float32,
+                    device="cuda")
+    out, SN, convN = gpu_prefill(w, inp, chunk_states=cs)
+    starts = np.cumsum([0] + lengths)
+    c = 0
+    for n, L in enumerate(lengths):
+        for j in range((L + 127) // 128):
+            P = min(128 * (j + 1), L)
+            t0 = int(starts[n])
+            sub = dict(inp)
+            for k in ("x", "beta", "g", "z"):
+                if inp[k] is not None:
+                    sub[k] = inp[k][t0:t0 + P].contiguous()
+            sub["cu_seqlens"] = torch.tensor([0, P], dtype=torch.int32)
+            sub["S0"] = inp["S0"][n:n + 1].contiguous()
+            sub["conv0"] = inp["conv0"][n:n + 1].contiguous()
+            _, ref_S, _ = oracle_prefill(w, sub)
+            assert_close(cs[c], ref_S[0], w.dtype, f"state after chunk {c} (sequence {n})")
+            c += 1
+    assert c == C
+    last = np.cumsum([(L + 127) // 128 for L in lengths]) - 1
+    for n, L in enumerate(lengths):
+        if L:
+            assert torch.equal(cs[int(last[n])], SN[n]), f"last chunk of sequence {n}"
