@@ -350,6 +350,33 @@ def bench_chunk_states(args, w, seed, dev, gdn):
             "extra_bytes_per_step": cs.numel() * 4}
 
 
+def bench_decode_multi(w, seed, dev, gdn, k=4, reps=20):
+    """k tokens per sequence per call (speculative verification), fp32 state, no snapshots."""
+    st = inputs.decode_state(w, seed)
+    S, cs = st["S"].to(dev), st["conv_state"].to(dev)
+    cw, nw = st["conv_w"].to(dev), st["norm_w"].to(dev)
+    dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    toks = [inputs.decode_step_inputs(w, seed, t) for t in range(k)]
+    stk = {key: torch.stack([t[key] for t in toks], dim=1).contiguous().to(dev)
+           for key in ("x", "beta", "g", "z")}
+    out = torch.empty((w.batch, k, w.num_v_heads, w.head_dim), dtype=w.dtype, device=dev)
+    call = lambda: gdn.decode_multi(stk["x"], stk["beta"], stk["g"], cs, S, cw, z=stk["z"],  # noqa: E731
+                                    norm_w=nw, out=out, dims=dims)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    m = statistics.median(ms)
+    return m, 2 * S.numel() * 4, w.batch * k / (m * 1e-3)
+
+
 def bench_decode(w, seed, dev, gdn, steps, state_dtype=torch.float32):
     st = inputs.decode_state(w, seed)
     S, cs = st["S"].to(dev).to(state_dtype), st["conv_state"].to(dev)
@@ -475,6 +502,9 @@ def main():
                                               args.decode_steps, torch.bfloat16)
     d16_ms = max_over_ranks([d16_ms], dev)[0]
     d16_gbs = n * d16_bytes / (d16_ms * 1e-3) / 1e9
+    dm_ms, dm_bytes, dm_tps = bench_decode_multi(inputs.CONFIGS[3], inputs.config_seed(3), dev,
+                                                 gdn)
+    dm_ms = max_over_ranks([dm_ms], dev)[0]
     decode = {"workload": inputs.CONFIGS[3].name, "value": dec_gbs, "unit": "GB/s",
               "ms_per_step": dec_ms, "steps": args.decode_steps,
               "roofline": {"bound": "hbm", "achieved": dec_gbs / n, "peak": peaks["hbm_gbs"],
@@ -488,7 +518,11 @@ def main():
                                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                           "frac": d16_gbs / n / peaks["hbm_gbs"],
                                           "traffic": None, "peak_source": f"{peak_src} (copy)"},
-                             "clocks": d16_clk}}
+                             "clocks": d16_clk},
+              "multi_token": {"tokens_per_call": 4, "ms_per_call": dm_ms,
+                              "sequence_tokens_per_s": n * inputs.CONFIGS[3].batch * 4 / (dm_ms * 1e-3),
+                              "one_token_steps_ms": 4 * dec_ms,
+                              "state_gbs": n * dm_bytes / (dm_ms * 1e-3) / 1e9}}
 
     chunk_states = bench_chunk_states(args, w, seed, dev, gdn)
 

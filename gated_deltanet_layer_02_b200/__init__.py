@@ -30,7 +30,7 @@ EXPORTS = (
     "gdn_decode_step", "gdn_trace_create", "gdn_trace_destroy", "gdn_trace_attach",
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
     "gdn_chunk_prefill_static_ws", "gdn_trace_span", "gdn_decode_step_bf16_state",
-    "gdn_chunk_prefill_states",
+    "gdn_chunk_prefill_states", "gdn_decode_multi",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
@@ -90,6 +90,8 @@ def lib():
             L.gdn_decode_step.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
                                           vp, vp]
             L.gdn_decode_step_bf16_state.argtypes = L.gdn_decode_step.argtypes
+            L.gdn_decode_multi.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                           i32, i32, vp, vp, vp]
             L.gdn_trace_create.argtypes = [ctypes.POINTER(vp)]
             L.gdn_trace_destroy.argtypes = [vp]
             L.gdn_trace_attach.argtypes = [vp]
@@ -276,6 +278,25 @@ def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx
     return out
 
 
+def decode_multi(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx=None,
+                 out=None, snapshots=None, dims: Dims | None = None):
+    """k tokens per sequence (x [B, k, Cc]); conv_state and S (fp32) are updated in place.
+    Returns out [B, k, Hv, d]; snapshots [B, k, Hv, d, d] fp32 receives the state after each
+    token when given."""
+    dims = dims or Dims()
+    dt = _act_dtype(x)
+    B, k = x.shape[0], x.shape[1]
+    if out is None:
+        out = torch.empty((B, k, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
+    _check("gdn_decode_multi", lib().gdn_decode_multi(
+        ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype, False),
+        _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
+        _ptr(norm_w, "norm_w", x.dtype), _ptr(conv_state, "conv_state", x.dtype),
+        _ptr(S, "S", torch.float32), _ptr(slot_idx, "slot_idx", torch.int32), B, k,
+        _ptr(out, "out", x.dtype), _ptr(snapshots, "snapshots", torch.float32), _stream()))
+    return out
+
+
 def debug_wait_probe(dev_status, limit_us: int):
     """Launch a kernel whose wait nothing satisfies; it gives up after limit_us."""
     _check("gdn_debug_wait_probe", lib().gdn_debug_wait_probe(
@@ -334,6 +355,7 @@ class Trace:
 
 
 __all__ = ["Dims", "GdnError", "lib", "conv1d_update", "gated_rmsnorm", "chunk_prefill",
+           "decode_multi",
            "chunk_prefill_static_ws", "STATIC_WORKSPACE_BYTES",
            "decode_step", "prefill_workspace_size", "conv_channels", "status_string", "Trace",
            "debug_wait_probe", "EXPORTS", "LIB_PATH"]

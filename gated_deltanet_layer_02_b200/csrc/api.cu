@@ -19,6 +19,8 @@ cudaError_t launch_conv_state_out(bool bf16, const void* x, const int32_t* cu, i
 cudaError_t launch_gated_rmsnorm(bool bf16, const void* o, const void* z, const void* w, float eps,
                                  int rows, int dim, void* y, cudaStream_t s);
 cudaError_t launch_decode(bool bf16, bool state_bf16, const gdn::DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_multi(bool bf16, const gdn::DecodeArgs& a, int k, float* snaps,
+                                cudaStream_t s);
 cudaError_t launch_recurrent_f32(const gdn::RecArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t s);
 size_t prefill_tc_workspace(int N, int T, int Hk, int Hv);
@@ -325,6 +327,42 @@ int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const 
                     void* out, void* stream) {
   return decode_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, conv_state, S, false, slot_idx,
                      batch, out, stream);
+}
+
+int gdn_decode_multi(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
+                     const float* beta, const float* g, const void* z, const void* norm_w,
+                     void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
+                     int32_t tokens, void* out, float* snapshots, void* stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!dtype_ok(dtype)) return GDN_ERR_UNSUPPORTED;
+  if (batch < 0 || tokens < 0) return GDN_ERR_INVALID_ARG;
+  if (tokens > 8) return GDN_ERR_UNSUPPORTED;
+  if (batch > 0 && tokens > 0 && (!x || !conv_w || !beta || !g || !conv_state || !S || !out))
+    return GDN_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, conv_w, beta, g, z, norm_w, conv_state, S, out, snapshots};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+  if (dims->num_v_heads / dims->num_k_heads > 8) return GDN_ERR_UNSUPPORTED;
+  gdn::DecodeArgs a{};
+  a.x = x;
+  a.conv_w = conv_w;
+  a.beta = beta;
+  a.g = g;
+  a.z = z;
+  a.norm_w = norm_w;
+  a.conv_state = conv_state;
+  a.S = S;
+  a.slot_idx = slot_idx;
+  a.out = out;
+  a.B = batch;
+  a.Hk = dims->num_k_heads;
+  a.Hv = dims->num_v_heads;
+  a.q_scale = dims->q_scale;
+  a.l2_eps = dims->l2_eps;
+  a.norm_eps = dims->norm_eps;
+  return map_cuda(gdn_host::launch_decode_multi(dtype == GDN_BF16, a, tokens, snapshots,
+                                                static_cast<cudaStream_t>(stream)));
 }
 
 int gdn_decode_step_bf16_state(const gdn_dims* dims, gdn_dtype dtype, const void* x,

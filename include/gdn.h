@@ -168,6 +168,26 @@ int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const 
                     void* out, void* stream);
 
 /*
+ * gdn_decode_multi -- k tokens for each of B sequences in one call: the verification step of
+ * speculative decoding with multi-token prediction.
+ * Source: the "Qwen3-Next" SGLang cookbook, section 4.2.4 (MTP / NEXTN speculative decoding,
+ * 4 draft tokens per step).  The result is that of k calls of gdn_decode_step on tokens
+ * 0..k-1 in order (the same fp32 arithmetic per token): outputs of every token, conv and
+ * recurrent state after token k-1.  The state rows are read and written once for all k tokens.
+ *   x [B, k, Cc], beta/g [B, k, Hv] fp32, z [B, k, Hv, d] nullable, out [B, k, Hv, d];
+ *   conv_w, norm_w, conv_state, S (fp32), slot_idx as gdn_decode_step; 0 <= k <= 8
+ *   (GDN_ERR_UNSUPPORTED above 8; k = 0 or B = 0 launch nothing).
+ *   snapshots [B, k, Hv, d, d] fp32, nullable: the recurrent state after each token, indexed by
+ *     position in the call (not by slot), for a caller that accepts only the first m tokens
+ *     (it restores snapshot m - 1; the conv history after m tokens is the last 3 rows of the
+ *     old history followed by x[b, 0..m-1]).
+ */
+int gdn_decode_multi(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
+                     const float* beta, const float* g, const void* z, const void* norm_w,
+                     void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
+                     int32_t tokens, void* out, float* snapshots, void* stream);
+
+/*
  * gdn_decode_step_bf16_state -- gdn_decode_step with the recurrent state stored in bf16.
  * Source: the "Qwen3-Next" SGLang cookbook, section 3.2: --mamba-ssm-dtype selects bf16 or fp32
  * (the default) for the recurrent state of the GDN layers.  Each step reads the bf16 state,

@@ -111,6 +111,11 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert bs(d, 1, A, A, A, A, None, None, A, None, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
     assert bs(d, 1, A, A, A, A, None, None, A, MIS, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
     assert bs(d, 3, A, A, A, A, None, None, A, A, None, 4, A, None) == gdn.GDN_ERR_UNSUPPORTED
+    mt = L.gdn_decode_multi
+    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, -1, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, 9, A, None, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert mt(d, 1, A, None, A, A, None, None, A, A, None, 4, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, 4, A, MIS, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_debug_wait_probe(None, 10, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_debug_wait_probe(A, 10_000_000, None) == gdn.GDN_ERR_INVALID_ARG
 
@@ -124,6 +129,10 @@ def test_zero_size_calls_launch_nothing(L):
                              None) == gdn.GDN_OK
     assert L.gdn_decode_step_bf16_state(d, 1, None, None, None, None, None, None, None, None,
                                         None, 0, None, None) == gdn.GDN_OK
+    assert L.gdn_decode_multi(d, 1, None, None, None, None, None, None, None, None, None, 0, 4,
+                              None, None, None) == gdn.GDN_OK
+    assert L.gdn_decode_multi(d, 1, None, None, None, None, None, None, None, None, None, 4, 0,
+                              None, None, None) == gdn.GDN_OK
     assert L.gdn_gated_rmsnorm(1, None, None, None, 1e-6, 0, 128, None, None) == gdn.GDN_OK
 
 
