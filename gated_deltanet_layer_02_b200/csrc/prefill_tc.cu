@@ -11,15 +11,14 @@
 //   S <- e^(G_L) S + U^T diag(e^(G_L - G)) K
 // Padded rows of a partial chunk carry k = q = v = 0, beta = 0, g = 0, which changes nothing.
 //
-// Kernels (one stream, in order):
+// Kernels (in order, programmatic dependent launch between them; optionally pipelined):
 //   schedule   one CTA: chunk table (sequence, first token, length) from cu_seqlens.
-//   prep       per (chunk, key head): conv + SiLU + L2 norms, gates, K K^T on tcgen05, the
-//              128x128 inverse (two 64x64 forward substitutions on CUDA cores, joined by two
-//              tcgen05 products: T = T_h - T_h N T_h), then W and U~ on tcgen05.
-//   chain      per (sequence, value head, d_v block): the sequential part.  S^T lives in TMEM
+//   qkv        per (chunk, 128-channel slice): conv + SiLU + L2 norms -> bf16 Q, K, V tiles.
+//   prep       per (chunk, value head): gates, K K^T on tcgen05, the 128x128 inverse (four
+//              32x32 in-warp row substitutions joined on tcgen05 in two levels), then W and U~.
+//   chain      per (sequence, value head, d_v block): the sequential part; S^T lives in TMEM
 //              (fp32); per chunk: X = W S_b^T (tcgen05), U = U~ - X, S^T += K^T diag(.) U.
-//              W and K tiles arrive by TMA, double-buffered one chunk ahead.
-//   out        per (chunk, key head): P from Q K^T (tcgen05), O = e^G Q S^T + P U (tcgen05),
+//   out        per (chunk, value head): P from Q K^T, O = e^G Q S^T + P U (TMEM A operands),
 //              z-gated RMSNorm epilogue, bf16 output.
 // Workspace tiles are plain row-major [128][128] bf16; TMA loads them with 128-byte swizzle.
 #include "args.cuh"
