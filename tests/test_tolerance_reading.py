@@ -26,3 +26,19 @@ def test_bf16_rounding_of_exact_output_breaks_max_abs_reading_only():
     assert max_abs_reading > 2e-2          # the exact answer in bf16 "fails"
     assert rel_rms_reading < 2e-3          # and sits 10x inside the relative RMS bar
     assert np.max(np.abs(ref)) > 10 * rms  # because the normalised output is heavy-tailed
+
+
+def test_bench_work_model_matches_the_closed_forms():
+    # the per-kernel split of the algorithmic work adds up to F(C) and 33,024 B/token
+    import bench
+    w = inputs.CONFIGS[1]
+    Hv, Hk, d = w.num_v_heads, w.num_k_heads, w.head_dim
+    for C in (64, 128):
+        f = bench.flops_per_token_by_kernel(w, C)
+        total = sum(v for k, v in f.items() if k != "gdn_prep_chain")
+        F = 2 * (Hv * (3 * d * d + 1.5 * C * d + C * C / 6) + Hk * C * d)
+        assert abs(total - F) < 1e-6 * F
+    assert abs(sum(v for k, v in bench.flops_per_token_by_kernel(w, 128).items()
+                   if k != "gdn_prep_chain") - 5.4176e6) < 1e3
+    b = bench.bytes_per_token_by_kernel(w)
+    assert sum(v for k, v in b.items() if k != "gdn_prep_chain") == 33024
