@@ -117,14 +117,14 @@ __device__ __forceinline__ float silu_fast(float x) {
 // preceding rows, arrive by TMA as two [131][64] boxes (128-byte swizzle); for the first chunk
 // of a sequence the 3 preceding rows are replaced by the caller's conv state (or zeros).
 // 128 threads: 16 column vectors x 8 runs of 16 tokens; the 16 threads of a row share a
-// half-warp, so the norm is a 4-step shuffle.  Outputs are bf16 [128][128] tiles per (chunk,
+// half-warp, so the norm is a 4-step shuffle.  At most 96 registers: five CTAs per SM.  Outputs are bf16 [128][128] tiles per (chunk,
 // head): Q -> Qw, K -> Kw, V -> Uw (read by gdn_prep, which overwrites it with U~).  Rows past
 // the chunk's length are written as zeros.
 constexpr int kXRows = kC + 3;
 constexpr uint32_t kXBox = 17408;  // one [131][64] bf16 box, rounded up to 1024 bytes
 constexpr uint32_t kQkvSmem = 2 * kXBox + 1024 + 64;
 
-__global__ void __launch_bounds__(128, 4) gdn_qkv_kernel(PrefillArgs a,
+__global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a,
                                                          const __grid_constant__ CUtensorMap mapX) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1692,8 +1692,10 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   }
   const bool fused = fused_grid > 0;
   trace_begin("chunk_schedule", s);
-  gdn::chunk_schedule_kernel<<<1, 1024, 0, s>>>(a.cu, a.N, a.ws, fused ? (int)(NC * a.Hv) : 0,
-                                                a.conv0, a.convN, Cc);
+  // one CTA; its width only needs to cover the sequences of one pass of the scan
+  const int sched_threads = a.N <= 32 ? 32 : (a.N <= 256 ? 256 : 1024);
+  gdn::chunk_schedule_kernel<<<1, sched_threads, 0, s>>>(
+      a.cu, a.N, a.ws, fused ? (int)(NC * a.Hv) : 0, a.conv0, a.convN, Cc);
   trace_end(s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
