@@ -30,7 +30,8 @@ EXPORTS = (
     "gdn_decode_step", "gdn_trace_create", "gdn_trace_destroy", "gdn_trace_attach",
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
     "gdn_chunk_prefill_static_ws", "gdn_trace_span", "gdn_decode_step_bf16_state",
-    "gdn_chunk_prefill_states", "gdn_decode_multi",
+    "gdn_chunk_prefill_states", "gdn_decode_multi", "gdn_block_prefill_workspace_size",
+    "gdn_block_prefill",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
@@ -92,6 +93,10 @@ def lib():
             L.gdn_decode_step_bf16_state.argtypes = L.gdn_decode_step.argtypes
             L.gdn_decode_multi.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                            i32, i32, vp, vp, vp]
+            L.gdn_block_prefill_workspace_size.argtypes = [dp, i32, i32, i32]
+            L.gdn_block_prefill_workspace_size.restype = ctypes.c_size_t
+            L.gdn_block_prefill.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                            i32, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
             L.gdn_trace_create.argtypes = [ctypes.POINTER(vp)]
             L.gdn_trace_destroy.argtypes = [vp]
             L.gdn_trace_attach.argtypes = [vp]
@@ -297,6 +302,38 @@ def decode_multi(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_id
     return out
 
 
+def block_prefill(h, w_qkv, w_z, w_ba, a_log, dt_bias, w_out, cu_seqlens, conv_w=None,
+                  norm_w=None, S0=None, SN=None, conv0=None, convN=None, y=None, workspace=None,
+                  dev_status=None, dims: Dims | None = None):
+    """Projections + gates + layer + output projection (bf16).  h [T, H] -> y [T, H].
+    Returns (y, SN, convN)."""
+    dims = dims or Dims()
+    T, H = h.shape
+    N = cu_seqlens.numel() - 1
+    Hv, d, K = dims.num_v_heads, dims.head_dim, dims.conv_kernel
+    dev = h.device
+    if y is None:
+        y = torch.empty((T, H), dtype=h.dtype, device=dev)
+    if SN is None:
+        SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
+    if convN is None:
+        convN = torch.empty((N, K - 1, dims.channels), dtype=h.dtype, device=dev)
+    need = lib().gdn_block_prefill_workspace_size(ctypes.byref(dims), H, N, T)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    bf = torch.bfloat16
+    _check("gdn_block_prefill", lib().gdn_block_prefill(
+        ctypes.byref(dims), H, _ptr(h, "h", bf), _ptr(w_qkv, "w_qkv", bf), _ptr(w_z, "w_z", bf),
+        _ptr(w_ba, "w_ba", bf), _ptr(a_log, "a_log", torch.float32),
+        _ptr(dt_bias, "dt_bias", torch.float32), _ptr(conv_w, "conv_w", bf),
+        _ptr(norm_w, "norm_w", bf), _ptr(w_out, "w_out", bf),
+        _ptr(cu_seqlens, "cu_seqlens", torch.int32), N, T, _ptr(S0, "S0", torch.float32),
+        _ptr(SN, "SN", torch.float32), _ptr(conv0, "conv0", bf), _ptr(convN, "convN", bf),
+        _ptr(y, "y", bf), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
+        _ptr(dev_status, "dev_status", torch.int32), _stream()))
+    return y, SN, convN
+
+
 def debug_wait_probe(dev_status, limit_us: int):
     """Launch a kernel whose wait nothing satisfies; it gives up after limit_us."""
     _check("gdn_debug_wait_probe", lib().gdn_debug_wait_probe(
@@ -355,7 +392,7 @@ class Trace:
 
 
 __all__ = ["Dims", "GdnError", "lib", "conv1d_update", "gated_rmsnorm", "chunk_prefill",
-           "decode_multi",
+           "decode_multi", "block_prefill",
            "chunk_prefill_static_ws", "STATIC_WORKSPACE_BYTES",
            "decode_step", "prefill_workspace_size", "conv_channels", "status_string", "Trace",
            "debug_wait_probe", "EXPORTS", "LIB_PATH"]

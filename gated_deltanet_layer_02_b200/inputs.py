@@ -167,6 +167,33 @@ def decode_step_inputs(w: Workload, seed: int, step: int) -> dict:
     return dict(x=x, z=z, beta=beta, g=g)
 
 
+def block_inputs(w: Workload, seed: int, hidden: int, with_conv0: bool = False) -> dict:
+    """Inputs of one token-mixer (projections + layer) call on CPU, bf16 unless stated:
+    h [T, H] ~ N(0, 1); projection weights [in, out] ~ N(0, 1/in), so that x, z, b and a come
+    out near unit variance; A_log ~ N(0, 0.5), dt_bias ~ N(0, 1) (fp32 [Hv]); conv_w ~
+    N(0, 0.5); norm_w = 1; S0 ~ N(0, s0_std) when s0_std > 0."""
+    lengths = tuple(int(v) for v in w.lengths)
+    T, N = int(sum(lengths)), len(lengths)
+    Hv, d, K, H, Cc = w.num_v_heads, w.head_dim, w.conv_kernel, hidden, w.channels
+    ss = np.random.SeedSequence(seed).spawn(10)
+    h = _normal_rows(ss[0], T, H, 1.0, w.dtype)
+    w_qkv = _normal_rows(ss[1], H, Cc, H ** -0.5, w.dtype)
+    w_z = _normal_rows(ss[2], H, Hv * d, H ** -0.5, w.dtype)
+    w_ba = _normal_rows(ss[3], H, 2 * Hv, H ** -0.5, w.dtype)
+    w_out = _normal_rows(ss[4], Hv * d, H, (Hv * d) ** -0.5, w.dtype)
+    small = np.random.default_rng(ss[5])
+    a_log = torch.from_numpy(small.normal(0.0, 0.5, Hv).astype(np.float32))
+    dt_bias = torch.from_numpy(small.normal(0.0, 1.0, Hv).astype(np.float32))
+    conv_w = _normal_rows(ss[6], Cc, K, 0.5, w.dtype)
+    S0 = (_normal_rows(ss[7], N * Hv * d, d, w.s0_std, torch.float32).view(N, Hv, d, d)
+          if w.s0_std > 0 else None)
+    conv0 = (_normal_rows(ss[8], N * (K - 1), Cc, 1.0, w.dtype).view(N, K - 1, Cc)
+             if with_conv0 else None)
+    return dict(h=h, w_qkv=w_qkv, w_z=w_z, w_ba=w_ba, a_log=a_log, dt_bias=dt_bias, w_out=w_out,
+                conv_w=conv_w, norm_w=torch.ones(d, dtype=w.dtype),
+                cu_seqlens=cu_seqlens_of(lengths), S0=S0, conv0=conv0)
+
+
 def config_seed(idx: int) -> int:
     return 1000 + idx
 
@@ -180,4 +207,4 @@ def custom(num_k_heads=2, num_v_heads=4, head_dim=128, dtype=torch.bfloat16, len
 
 
 __all__ = ["CONFIGS", "Workload", "prefill_inputs", "decode_state", "decode_step_inputs",
-           "config_seed", "custom", "cu_seqlens_of"]
+           "config_seed", "custom", "cu_seqlens_of", "block_inputs"]

@@ -168,6 +168,30 @@ int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const 
                     void* out, void* stream);
 
 /*
+ * gdn_block_prefill -- the token mixer of a Gated DeltaNet decoder layer: input projections,
+ * gates, gdn_chunk_prefill and the output projection, bf16 activations and weights.
+ * Source: the hyper.ai Qwen3-Next paragraph (QKV and a separate Z projection around the gated
+ * delta rule) and the Qwen3-Coder-Next config table (hidden_size 2048).  The gate formulas are
+ * not on the pages; this library reads them as beta = sigmoid(b), g = log(alpha) =
+ * -exp(A_log) * softplus(a + dt_bias) per value head.
+ *   h [T, H]; w_qkv [H, Cc], w_z [H, Hv d], w_ba [H, 2 Hv] (columns: b for the Hv heads, then
+ *   a), all row-major (input x output); a_log, dt_bias [Hv] fp32; w_out [Hv d, H]; y [T, H].
+ *   conv_w, norm_w, cu_seqlens, S0, SN, conv0, convN, dev_status: as gdn_chunk_prefill.
+ *   workspace: at least gdn_block_prefill_workspace_size() bytes, 256-byte aligned.
+ * The four projections are plain GEMMs (fp32 accumulation) and run in cuBLAS, loaded on the
+ * first call (GDN_ERR_UNSUPPORTED when it cannot be loaded); cuBLAS creates one handle per
+ * device and host thread on that first call (not inside a stream capture).
+ */
+size_t gdn_block_prefill_workspace_size(const gdn_dims* dims, int32_t hidden, int32_t num_seqs,
+                                        int32_t num_tokens);
+int gdn_block_prefill(const gdn_dims* dims, int32_t hidden, const void* h, const void* w_qkv,
+                      const void* w_z, const void* w_ba, const float* a_log, const float* dt_bias,
+                      const void* conv_w, const void* norm_w, const void* w_out,
+                      const int32_t* cu_seqlens, int32_t num_seqs, int32_t num_tokens,
+                      const float* S0, float* SN, const void* conv0, void* convN, void* y,
+                      void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
  * gdn_decode_multi -- k tokens for each of B sequences in one call: the verification step of
  * speculative decoding with multi-token prediction.
  * Source: the "Qwen3-Next" SGLang cookbook, section 4.2.4 (MTP / NEXTN speculative decoding,

@@ -9,6 +9,8 @@ This module is argument marshalling around ``gdn_oracle.c`` (plain C, fp64, sequ
 (sequence, value head) unit).  The header of that file lists what is computed, the sources and
 every reading taken where the pages are silent.
 
+``block_prefill`` composes the layer with plain matrix products and ``block_gates``.
+
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py`` (closed forms,
 invariants, brute force, library routines); none is "parity unpinned".
 """
@@ -213,6 +215,42 @@ def prefill(dims: Dims, x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None
     if rc != 0:
         raise ValueError(f"orc_prefill failed: {rc}")
     return out, SN, convN
+
+
+def block_gates(ba, a_log, dt_bias):
+    """Per-token, per-value-head gates of the token mixer from the [T, 2 Hv] projection rows
+    [b | a]: beta = sigmoid(b) and g = log(alpha) = -exp(A_log) * softplus(a + dt_bias).
+    The pages (hyper.ai's Qwen3-Next paragraph) say only that beta sets the update strength
+    and alpha the decay; this parameterisation is the reading taken for it.  fp64 numpy."""
+    ba = np.asarray(ba, np.float64)
+    Hv = ba.shape[1] // 2
+    b, a = ba[:, :Hv], ba[:, Hv:] + np.asarray(dt_bias, np.float64)[None, :]
+    beta = 1.0 / (1.0 + np.exp(-b))
+    softplus = np.logaddexp(0.0, a)
+    g = -np.exp(np.asarray(a_log, np.float64))[None, :] * softplus
+    return beta, g
+
+
+def block_prefill(dims: Dims, h, w_qkv, w_z, w_ba, a_log, dt_bias, w_out, cu_seqlens,
+                  conv_w=None, norm_w=None, S0=None, conv0=None, nthreads: int | None = None):
+    """The token mixer of a decoder layer in fp64: x = h W_qkv, z = h W_z, [b | a] = h W_ba,
+    the gates of block_gates, the layer (prefill) and y = o W_out.  Weights are [in, out].
+    Returns (y [T, H], SN, convN) as fp64 numpy; the gates enter the layer rounded to fp32
+    (its beta and g are fp32 inputs)."""
+    f64 = lambda t: np.asarray(t.detach().cpu().double().numpy() if isinstance(t, torch.Tensor)
+                               else t, np.float64)
+    hh = f64(h)
+    T = hh.shape[0]
+    x = hh @ f64(w_qkv)
+    z = hh @ f64(w_z)
+    beta, g = block_gates(hh @ f64(w_ba), f64(a_log), f64(dt_bias))
+    to64 = lambda t: None if t is None else torch.from_numpy(f64(t))
+    o, SN, convN = prefill(dims, torch.from_numpy(x), beta.astype(np.float32),
+                           g.astype(np.float32), cu_seqlens, conv_w=to64(conv_w),
+                           z=torch.from_numpy(z), norm_w=to64(norm_w), S0=S0, conv0=to64(conv0),
+                           nthreads=nthreads)
+    y = o.reshape(T, -1) @ f64(w_out)
+    return y, SN, convN
 
 
 def decode_step(dims: Dims, x, beta, g, conv_state, S, conv_w=None, z=None, norm_w=None,

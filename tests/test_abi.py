@@ -120,6 +120,38 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert L.gdn_debug_wait_probe(A, 10_000_000, None) == gdn.GDN_ERR_INVALID_ARG
 
 
+def _block(L, dims, hidden=256, N=1, T=16, h=A, ws=A, ws_bytes=1 << 40, y=A, a_log=A):
+    return L.gdn_block_prefill(dims, hidden, h, A, A, A, a_log, A, None, None, A, A, N, T, None,
+                               None, None, None, y, ws, ws_bytes, None, None)
+
+
+def test_block_prefill_argument_errors(L):
+    d = ctypes.byref(gdn.Dims())
+    size = L.gdn_block_prefill_workspace_size
+    assert size(None, 256, 1, 16) == 0
+    assert size(d, 0, 1, 16) == 0
+    assert size(d, 256, -1, 16) == 0
+    layer = L.gdn_chunk_prefill_workspace_size(d, 1, 1, 4096)
+    # layer scratch + bf16 x, z, o and fp32 b|a, beta, g per token
+    assert size(d, 2048, 1, 4096) >= layer + 4096 * (8192 * 2 + 2 * 4096 * 2 + 4 * 32 * 4)
+    assert _block(L, None) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, hidden=0) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, hidden=260) == gdn.GDN_ERR_INVALID_ARG      # rows of 16-byte multiples
+    assert _block(L, d, N=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, h=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, y=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, a_log=None) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, h=MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, ws=P((1 << 20) + 16)) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, ws=None) == gdn.GDN_ERR_WORKSPACE
+    assert _block(L, d, ws_bytes=1024) == gdn.GDN_ERR_WORKSPACE
+    assert _block(L, ctypes.byref(gdn.Dims(head_dim=64))) == gdn.GDN_ERR_INVALID_ARG
+    # no sequences and no tokens: valid, nothing to launch
+    assert L.gdn_block_prefill(d, 256, None, None, None, None, None, None, None, None, None, None,
+                               0, 0, None, None, None, None, None, A, 1 << 30, None,
+                               None) == gdn.GDN_OK
+
+
 def test_zero_size_calls_launch_nothing(L):
     d = ctypes.byref(gdn.Dims())
     # no sequences, no tokens: valid and a no-op

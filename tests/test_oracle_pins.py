@@ -14,6 +14,8 @@ operand anywhere in the oracle fails at least one of them:
   P9  conv + SiLU = torch.nn.functional.conv1d (library routine) then SiLU.
   P10 gated RMSNorm = torch.nn.functional.rms_norm (library routine) * w * silu(z); z = 0 -> 0.
   P11 contraction bound |S_t|_F <= alpha_t |S_{t-1}|_F + beta_t |v_t|.
+  P12 token-mixer gates: sigmoid / softplus special values and torch's softplus; with
+      identity projections the token mixer reduces to the layer.
 The chunked (WY/UT) form the CUDA path uses is checked against the oracle in
 test_chunk_algebra.py (P6).
 """
@@ -376,3 +378,55 @@ def test_layer_constants_match_model_card():
     assert oracle.Dims().norm_eps == c["rms_norm_eps"]
     assert inputs.CONFIGS[4].tokens == c["max_position_embeddings"]
     assert inputs.CONFIGS[2].tokens == 40677
+
+
+# ---------------------------------------------------------------------------------------- P12
+def test_p12_block_gates_special_values():
+    Hv = 3
+    ba = np.zeros((2, 2 * Hv))
+    ba[1, :Hv] = [40.0, -40.0, np.log(3.0)]            # b
+    ba[1, Hv:] = [60.0, -3.0, 1.5]                     # a
+    beta, g = oracle.block_gates(ba, np.zeros(Hv), np.zeros(Hv))
+    np.testing.assert_allclose(beta[0], 0.5, rtol=0, atol=0)        # sigmoid(0)
+    np.testing.assert_allclose(g[0], -np.log(2.0), rtol=1e-15)      # -softplus(0)
+    np.testing.assert_allclose(beta[1], [1.0, 0.0, 0.75], atol=1e-15)
+    np.testing.assert_allclose(g[1, 0], -60.0, rtol=1e-15)          # softplus(u) -> u
+    # A_log scales, dt_bias shifts: against torch's softplus (library routine)
+    rng = _rng(12)
+    ba = rng.normal(0, 2, (50, 2 * Hv))
+    a_log, dt = rng.normal(0, 1, Hv), rng.normal(0, 1, Hv)
+    beta, g = oracle.block_gates(ba, a_log, dt)
+    sp = F.softplus(torch.from_numpy(ba[:, Hv:] + dt)).numpy()
+    np.testing.assert_allclose(g, -np.exp(a_log) * sp, rtol=1e-12)
+    np.testing.assert_allclose(beta + oracle.block_gates(-ba, a_log, dt)[0], 1.0, rtol=1e-14)
+    assert np.all(g < 0) and np.all((beta > 0) & (beta < 1))
+
+
+def test_p12_block_with_identity_projections_is_the_layer():
+    d, hk, hv = 8, 1, 2
+    dims = _dims(hk, hv, d)
+    Cc, T = (2 * hk + hv) * d, 11
+    rng = _rng(1212)
+    x = rng.normal(0, 1, (T, Cc))
+    z = rng.normal(0, 1, (T, hv * d))
+    ba = rng.normal(0, 1, (T, 2 * hv))
+    H = Cc + hv * d + 2 * hv
+    h = np.concatenate([x, z, ba], axis=1)              # the hidden row holds x | z | b a
+    eye = np.eye(H)
+    w_qkv, w_z, w_ba = eye[:, :Cc], eye[:, Cc:Cc + hv * d], eye[:, Cc + hv * d:]
+    a_log, dt = rng.normal(0, 0.5, hv), rng.normal(0, 1, hv)
+    w_out = rng.normal(0, 1, (hv * d, 5))
+    conv_w = rng.normal(0, 0.5, (Cc, 4))
+    norm_w = rng.normal(1, 0.1, d)
+    cu = inputs.cu_seqlens_of([4, 7])
+    y, SN, convN = oracle.block_prefill(dims, h, w_qkv, w_z, w_ba, a_log, dt, w_out, cu,
+                                        conv_w=conv_w, norm_w=norm_w, nthreads=2)
+    beta = 1.0 / (1.0 + np.exp(-ba[:, :hv]))
+    g = -np.exp(a_log) * F.softplus(torch.from_numpy(ba[:, hv:] + dt)).numpy()
+    o, SN2, convN2 = oracle.prefill(dims, torch.from_numpy(x), torch.from_numpy(_f32(beta)),
+                                    torch.from_numpy(_f32(g)), cu,
+                                    conv_w=torch.from_numpy(conv_w), z=torch.from_numpy(z),
+                                    norm_w=torch.from_numpy(norm_w), nthreads=2)
+    np.testing.assert_allclose(y, o.reshape(T, -1) @ w_out, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(SN, SN2)
+    np.testing.assert_array_equal(convN, convN2)
