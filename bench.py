@@ -15,6 +15,7 @@ replicas (the layer needs no collective): weak scaling, max time over ranks.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -350,6 +351,43 @@ def bench_chunk_states(args, w, seed, dev, gdn):
             "extra_bytes_per_step": cs.numel() * 4}
 
 
+def bench_block(w, seed, dev, gdn, hidden=2048, reps=20):
+    """The token mixer (gdn_block_prefill: cuBLAS projections, gates, the layer, output
+    projection) on the same sequences, hidden size 2048, eager calls with L2 flushed in between.
+    flops_per_step counts the four projection GEMMs only."""
+    bw = inputs.custom(w.num_k_heads, w.num_v_heads, w.head_dim, w.dtype, lengths=w.lengths)
+    inp = inputs.block_inputs(bw, seed, hidden)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    T, N, Hv, dh = w.tokens, len(w.lengths), w.num_v_heads, w.head_dim
+    y = torch.empty((T, hidden), dtype=w.dtype, device=dev)
+    SN = torch.empty((N, Hv, dh, dh), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.lib().gdn_block_prefill_workspace_size(ctypes.byref(dims), hidden, N, T),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        gdn.block_prefill(d["h"], d["w_qkv"], d["w_z"], d["w_ba"], d["a_log"], d["dt_bias"],
+                          d["w_out"], d["cu_seqlens"], conv_w=d["conv_w"], norm_w=d["norm_w"],
+                          SN=SN, y=y, workspace=ws, dims=dims)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    t = statistics.median(ms)
+    flops = 2 * T * hidden * (w.channels + 2 * Hv * dh + 2 * Hv)
+    return {"workload": f"{w.name}, hidden {hidden}", "ms_per_step": t,
+            "tokens_per_s": T / (t * 1e-3), "projection_flops_per_step": flops}
+
+
 def bench_decode_multi(w, seed, dev, gdn, k=4, reps=20):
     """k tokens per sequence per call (speculative verification), fp32 state, no snapshots."""
     st = inputs.decode_state(w, seed)
@@ -525,6 +563,7 @@ def main():
                               "state_gbs": n * dm_bytes / (dm_ms * 1e-3) / 1e9}}
 
     chunk_states = bench_chunk_states(args, w, seed, dev, gdn)
+    block = bench_block(w, seed, dev, gdn)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -544,7 +583,8 @@ def main():
         "e2e": {"value": job_tokens_per_s(n, T, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": len(recs), "eager_ms_per_step": eager_ms,
-        "clocks": clocks, "decode": decode, "chunk_states": chunk_states, "cpu_baseline": cpu,
+        "clocks": clocks, "decode": decode, "chunk_states": chunk_states, "block": block,
+        "cpu_baseline": cpu,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)

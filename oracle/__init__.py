@@ -249,7 +249,7 @@ def block_prefill(dims: Dims, h, w_qkv, w_z, w_ba, a_log, dt_bias, w_out, cu_seq
                            g.astype(np.float32), cu_seqlens, conv_w=to64(conv_w),
                            z=torch.from_numpy(z), norm_w=to64(norm_w), S0=S0, conv0=to64(conv0),
                            nthreads=nthreads)
-    y = o.reshape(T, -1) @ f64(w_out)
+    y = o.reshape(T, dims.num_v_heads * dims.head_dim) @ f64(w_out)
     return y, SN, convN
 
 
