@@ -31,7 +31,7 @@ EXPORTS = (
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
     "gdn_chunk_prefill_static_ws", "gdn_trace_span", "gdn_decode_step_bf16_state",
     "gdn_chunk_prefill_states", "gdn_decode_multi", "gdn_block_prefill_workspace_size",
-    "gdn_block_prefill",
+    "gdn_block_prefill", "gdn_chunk_prefill_slots",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
@@ -93,6 +93,9 @@ def lib():
             L.gdn_decode_step_bf16_state.argtypes = L.gdn_decode_step.argtypes
             L.gdn_decode_multi.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                            i32, i32, vp, vp, vp]
+            L.gdn_chunk_prefill_slots.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                                  i32, i32, vp, vp, vp, vp, vp, ctypes.c_size_t,
+                                                  vp, vp]
             L.gdn_block_prefill_workspace_size.argtypes = [dp, i32, i32, i32]
             L.gdn_block_prefill_workspace_size.restype = ctypes.c_size_t
             L.gdn_block_prefill.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
@@ -230,6 +233,31 @@ def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=N
         _check("gdn_chunk_prefill_states", lib().gdn_chunk_prefill_states(
             *head, _ptr(chunk_states, "chunk_states", torch.float32), *tail))
     return out, SN, convN
+
+
+def chunk_prefill_slots(x, beta, g, cu_seqlens, S_pool, slot_idx=None, conv_pool=None,
+                        conv_w=None, z=None, norm_w=None, out=None, workspace=None,
+                        dev_status=None, dims: Dims | None = None):
+    """chunk_prefill with the states in pools shared with decode_step: sequence n starts from
+    and overwrites S_pool[slot_idx[n]] ([slots, Hv, d, d] fp32) and conv_pool[slot_idx[n]]
+    ([slots, K-1, Cc]).  Slots must be distinct.  Returns out [T, Hv, d]."""
+    dims = dims or Dims()
+    T = x.shape[0]
+    N = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((T, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(prefill_workspace_size(N, T, x.dtype, dims), 256),
+                                dtype=torch.uint8, device=x.device)
+    _check("gdn_chunk_prefill_slots", lib().gdn_chunk_prefill_slots(
+        ctypes.byref(dims), _act_dtype(x), _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
+        _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
+        _ptr(norm_w, "norm_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N, T,
+        _ptr(slot_idx, "slot_idx", torch.int32), _ptr(S_pool, "S_pool", torch.float32),
+        _ptr(conv_pool, "conv_pool", x.dtype), _ptr(out, "out", x.dtype),
+        _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
+        _ptr(dev_status, "dev_status", torch.int32), _stream()))
+    return out
 
 
 def chunk_prefill_static_ws(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None,
@@ -392,7 +420,7 @@ class Trace:
 
 
 __all__ = ["Dims", "GdnError", "lib", "conv1d_update", "gated_rmsnorm", "chunk_prefill",
-           "decode_multi", "block_prefill",
+           "decode_multi", "block_prefill", "chunk_prefill_slots",
            "chunk_prefill_static_ws", "STATIC_WORKSPACE_BYTES",
            "decode_step", "prefill_workspace_size", "conv_channels", "status_string", "Trace",
            "debug_wait_probe", "EXPORTS", "LIB_PATH"]

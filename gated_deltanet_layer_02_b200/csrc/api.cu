@@ -15,7 +15,8 @@ cudaError_t launch_conv1d(bool bf16, const void* x, void* y, const void* w, cons
                           int N, int T_total, int Cc, const void* st_in, void* st_out,
                           cudaStream_t s);
 cudaError_t launch_conv_state_out(bool bf16, const void* x, const int32_t* cu, int N, int Cc,
-                                  const void* st_in, void* st_out, cudaStream_t s);
+                                  const void* st_in, void* st_out, const int32_t* slot,
+                                  cudaStream_t s);
 cudaError_t launch_gated_rmsnorm(bool bf16, const void* o, const void* z, const void* w, float eps,
                                  int rows, int dim, void* y, cudaStream_t s);
 cudaError_t launch_decode(bool bf16, bool state_bf16, const gdn::DecodeArgs& a, cudaStream_t s);
@@ -180,7 +181,8 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
                         const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
                         int32_t num_tokens, const float* S0, float* SN, const void* conv0,
                         void* convN, void* out, void* workspace, size_t workspace_bytes,
-                        int32_t* dev_status, float* chunk_states, void* stream) {
+                        int32_t* dev_status, float* chunk_states, const int32_t* slot,
+                        void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return GDN_ERR_UNSUPPORTED;
@@ -213,6 +215,7 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
     a.SN = SN;
     a.conv0 = static_cast<const float*>(conv0);
     a.out = static_cast<float*>(out);
+    a.slot = slot;
     a.N = num_seqs;
     a.Hk = dims->num_k_heads;
     a.Hv = dims->num_v_heads;
@@ -221,7 +224,8 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
     a.norm_eps = dims->norm_eps;
     cudaError_t e = gdn_host::launch_recurrent_f32(a, s);
     if (e == cudaSuccess && convN)
-      e = gdn_host::launch_conv_state_out(false, x, cu_seqlens, num_seqs, Cc, conv0, convN, s);
+      e = gdn_host::launch_conv_state_out(false, x, cu_seqlens, num_seqs, Cc, conv0, convN, slot,
+                                          s);
     return map_cuda(e);
   }
   gdn::PrefillArgs a{};
@@ -237,6 +241,7 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
   a.conv0 = static_cast<const __nv_bfloat16*>(conv0);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.chunk_states = chunk_states;
+  a.slot = slot;
   a.status = dev_status;
   a.N = num_seqs;
   a.T = num_tokens;
@@ -252,7 +257,7 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
   a.convN = separate_conv_state ? nullptr : static_cast<__nv_bfloat16*>(convN);
   cudaError_t e = gdn_host::launch_prefill_tc(a, workspace, s);
   if (e == cudaSuccess && separate_conv_state)
-    e = gdn_host::launch_conv_state_out(true, x, cu_seqlens, num_seqs, Cc, conv0, convN, s);
+    e = gdn_host::launch_conv_state_out(true, x, cu_seqlens, num_seqs, Cc, conv0, convN, slot, s);
   return map_cuda(e);
 }
 
@@ -264,7 +269,7 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
                       void* stream) {
   return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
                       num_tokens, S0, SN, conv0, convN, out, workspace, workspace_bytes,
-                      dev_status, nullptr, stream);
+                      dev_status, nullptr, nullptr, stream);
 }
 
 int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* x,
@@ -277,7 +282,19 @@ int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* 
   if (num_tokens > 0 && !chunk_states) return GDN_ERR_INVALID_ARG;
   return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
                       num_tokens, S0, SN, conv0, convN, out, workspace, workspace_bytes,
-                      dev_status, chunk_states, stream);
+                      dev_status, chunk_states, nullptr, stream);
+}
+
+int gdn_chunk_prefill_slots(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                            const void* conv_w, const float* beta, const float* g, const void* z,
+                            const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
+                            int32_t num_tokens, const int32_t* slot_idx, float* S_pool,
+                            void* conv_pool, void* out, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream) {
+  if (num_seqs > 0 && !S_pool) return GDN_ERR_INVALID_ARG;
+  return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
+                      num_tokens, S_pool, S_pool, conv_pool, conv_pool, out, workspace,
+                      workspace_bytes, dev_status, nullptr, slot_idx, stream);
 }
 
 }  // extern "C"

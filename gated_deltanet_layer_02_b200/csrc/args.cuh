@@ -5,6 +5,11 @@
 
 namespace gdn {
 
+// Row of a state pool that holds the states of sequence n: slot[n], or n without a slot map.
+__device__ __forceinline__ int state_row(const int32_t* slot, int n) {
+  return slot ? __ldg(slot + n) : n;
+}
+
 struct DecodeArgs {
   const void* x;
   const void* conv_w;
@@ -32,6 +37,7 @@ struct RecArgs {
   float* SN;
   const float* conv0;
   float* out;
+  const int32_t* slot;  // [N] state-pool row of each sequence (S0, SN, conv0), or NULL (= n)
   int N, Hk, Hv;
   float q_scale, l2_eps, norm_eps;
 };
@@ -68,6 +74,7 @@ struct PrefillArgs {
                          // when set; NULL when the caller wants none or it aliases conv0
   __nv_bfloat16* out;
   float* chunk_states;  // [chunks][Hv][d_v][d_k] fp32: state after each chunk, or NULL
+  const int32_t* slot;  // [N] state-pool row of each sequence (S0, SN, conv0, convN), or NULL
   int32_t* status;
   int N, T, Hk, Hv, nsplit;
   float q_scale, l2_eps, norm_eps;

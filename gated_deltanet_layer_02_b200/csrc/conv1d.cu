@@ -7,6 +7,7 @@
 // the 3-token history in registers; sequence boundaries inside a run restart the history from
 // the caller's conv state.  Reads and writes are 16-byte vectors, consecutive threads on
 // consecutive channels, so every warp access is one contiguous 256/512-byte segment.
+#include "args.cuh"
 #include "common.cuh"
 
 namespace gdn {
@@ -82,11 +83,13 @@ template <typename T>
 __global__ void __launch_bounds__(128) conv_state_out_kernel(const T* __restrict__ x,
                                                              const int32_t* __restrict__ cu, int N,
                                                              int Cc, const T* state_in,
-                                                             T* state_out) {
+                                                             T* state_out,
+                                                             const int32_t* __restrict__ slot) {
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   const int n = blockIdx.y;
   if (c >= Cc || n >= N) return;
   const int s = __ldg(cu + n), L = __ldg(cu + n + 1) - s;
+  const size_t row = (size_t)state_row(slot, n) * 3;
   float r[3][8];
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
@@ -94,14 +97,14 @@ __global__ void __launch_bounds__(128) conv_state_out_kernel(const T* __restrict
     if (e >= 3) {
       load8(x + (size_t)(s + e - 3) * Cc + c, r[j]);
     } else if (state_in) {
-      load8(state_in + ((size_t)n * 3 + e) * Cc + c, r[j]);
+      load8(state_in + (row + e) * Cc + c, r[j]);
     } else {
 #pragma unroll
       for (int k = 0; k < 8; ++k) r[j][k] = 0.f;
     }
   }
 #pragma unroll
-  for (int j = 0; j < 3; ++j) store8(state_out + ((size_t)n * 3 + j) * Cc + c, r[j]);
+  for (int j = 0; j < 3; ++j) store8(state_out + (row + j) * Cc + c, r[j]);
 }
 
 }  // namespace gdn
@@ -127,7 +130,7 @@ static cudaError_t conv1d_impl(const void* x, void* y, const void* w, const int3
     trace_begin("conv_state_out", s);
     gdn::conv_state_out_kernel<T><<<grid, 128, 0, s>>>(static_cast<const T*>(x), cu, N, Cc,
                                                        static_cast<const T*>(st_in),
-                                                       static_cast<T*>(st_out));
+                                                       static_cast<T*>(st_out), nullptr);
     trace_end(s);
     return cudaGetLastError();
   }
@@ -142,18 +145,19 @@ cudaError_t launch_conv1d(bool bf16, const void* x, void* y, const void* w, cons
 }
 
 cudaError_t launch_conv_state_out(bool bf16, const void* x, const int32_t* cu, int N, int Cc,
-                                  const void* st_in, void* st_out, cudaStream_t s) {
+                                  const void* st_in, void* st_out, const int32_t* slot,
+                                  cudaStream_t s) {
   if (!st_out || N == 0) return cudaSuccess;
   dim3 grid((Cc / 8 + 127) / 128, N);
   trace_begin("conv_state_out", s);
   if (bf16)
     gdn::conv_state_out_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), cu, N, Cc,
-        static_cast<const __nv_bfloat16*>(st_in), static_cast<__nv_bfloat16*>(st_out));
+        static_cast<const __nv_bfloat16*>(st_in), static_cast<__nv_bfloat16*>(st_out), slot);
   else
     gdn::conv_state_out_kernel<float><<<grid, 128, 0, s>>>(static_cast<const float*>(x), cu, N,
                                                            Cc, static_cast<const float*>(st_in),
-                                                           static_cast<float*>(st_out));
+                                                           static_cast<float*>(st_out), slot);
   trace_end(s);
   return cudaGetLastError();
 }

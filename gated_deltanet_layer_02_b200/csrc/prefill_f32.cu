@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(256) recurrent_f32_kernel(RecArgs a) {
     if (a.conv0) {
 #pragma unroll
       for (int j = 0; j < 3; ++j) {
-        const float* row = a.conv0 + ((size_t)n * 3 + j) * Cc;
+        const float* row = a.conv0 + ((size_t)state_row(a.slot, n) * 3 + j) * Cc;
         hq[j] = row[cq + tid];
         hkk[j] = row[ck + tid];
         hv[j] = row[cv + tid];
@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(256) recurrent_f32_kernel(RecArgs a) {
   }
   // state rows of this warp
   float st[kRows][4];
-  const size_t sbase = ((size_t)n * a.Hv + h) * d * d;
+  const size_t sbase = ((size_t)state_row(a.slot, n) * a.Hv + h) * d * d;
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
     const int v = warp * kRows + r;

@@ -42,7 +42,7 @@ constexpr uint32_t kTile = 16384;  // one [128][64] bf16 row tile
 // ------------------------------------------------------------------------------ schedule
 __global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Workspace ws,
                                       int nready, const __nv_bfloat16* conv0,
-                                      __nv_bfloat16* convN, int Cc) {
+                                      __nv_bfloat16* convN, const int32_t* slot, int Cc) {
   // publication flags and work counter of the persistent prep + chain kernel
   for (int k = threadIdx.x; k < nready; k += blockDim.x) ws.ready[k] = 0;
   if (threadIdx.x == 0 && nready > 0) *ws.counter = 0;
@@ -84,8 +84,9 @@ __global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Wor
   if (convN) {
     for (int n = 0; n < N; ++n) {
       if (cu[n + 1] != cu[n]) continue;
+      const size_t row = (size_t)state_row(slot, n) * 3 * Cc;
       for (int k = threadIdx.x; k < 3 * Cc; k += blockDim.x)
-        convN[(size_t)n * 3 * Cc + k] = conv0 ? conv0[(size_t)n * 3 * Cc + k] : __float2bfloat16(0.f);
+        convN[row + k] = conv0 ? conv0[row + k] : __float2bfloat16(0.f);
     }
   }
 }
@@ -180,7 +181,9 @@ __global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a,
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (a.conv0) v = *reinterpret_cast<const uint4*>(a.conv0 + ((size_t)ci.n * 3 + j) * Cc + ch);
+      if (a.conv0)
+        v = *reinterpret_cast<const uint4*>(
+            a.conv0 + ((size_t)state_row(a.slot, ci.n) * 3 + j) * Cc + ch);
       *row_ptr(j) = v;
     }
   }
@@ -190,7 +193,8 @@ __global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a,
   if (a.convN && run == 0 && ci.t0 + ci.L == __ldg(a.cu + ci.n + 1)) {
 #pragma unroll
     for (int j = 0; j < 3; ++j)
-      *reinterpret_cast<uint4*>(a.convN + ((size_t)ci.n * 3 + j) * Cc + ch) = *row_ptr(ci.L + j);
+      *reinterpret_cast<uint4*>(a.convN + ((size_t)state_row(a.slot, ci.n) * 3 + j) * Cc + ch) =
+          *row_ptr(ci.L + j);
   }
   const int i0 = run * 16;
   float2 hst[3][4];
@@ -832,7 +836,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
   const uint32_t lane_addr = tmem_at(tmem, (warp & 3) * 32, 0);
   const int k_row = tid & 127;  // TMEM lane = d_k index for S^T, = token index for X
   const int cs = (tid >> 7) * kCPT;  // first column of this thread inside the d_v block
-  const size_t sbase = ((size_t)n * a.Hv + h) * kD * kD;
+  const size_t sbase = ((size_t)state_row(a.slot, n) * a.Hv + h) * kD * kD;
 
   // ---- S^T initial value: lane k, column v  (state layout [v][k])
   {
@@ -1695,7 +1699,7 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   // one CTA; its width only needs to cover the sequences of one pass of the scan
   const int sched_threads = a.N <= 32 ? 32 : (a.N <= 256 ? 256 : 1024);
   gdn::chunk_schedule_kernel<<<1, sched_threads, 0, s>>>(
-      a.cu, a.N, a.ws, fused ? (int)(NC * a.Hv) : 0, a.conv0, a.convN, Cc);
+      a.cu, a.N, a.ws, fused ? (int)(NC * a.Hv) : 0, a.conv0, a.convN, a.slot, Cc);
   trace_end(s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 

@@ -153,6 +153,26 @@ int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* 
                              void* stream);
 
 /*
+ * gdn_chunk_prefill_slots -- gdn_chunk_prefill whose initial and final states live in a state
+ * pool shared with gdn_decode_step: sequence n reads and overwrites row slot_idx[n] of the pools.
+ * Source: the "Qwen3-Next" SGLang cookbook, section 3.2 (the mamba state cache of the hybrid GDN
+ * layers, one cached state per request slot, fp32 by default).
+ *   slot_idx  [N] int32 device, nullable (= identity); the slots of one call must be distinct
+ *             and inside the pools (not checked on the device).
+ *   S_pool    [slots, Hv, d, d] fp32, in/out, required when N > 0.
+ *   conv_pool [slots, K-1, Cc] (activation dtype), in/out, nullable: zero conv history, none kept.
+ * Every other argument, the workspace size and the status codes are those of gdn_chunk_prefill;
+ * the result equals gdn_chunk_prefill with S0 = SN = S_pool[slot_idx] and conv0 = convN =
+ * conv_pool[slot_idx], pool rows outside slot_idx untouched.
+ */
+int gdn_chunk_prefill_slots(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                            const void* conv_w, const float* beta, const float* g, const void* z,
+                            const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
+                            int32_t num_tokens, const int32_t* slot_idx, float* S_pool,
+                            void* conv_pool, void* out, void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, void* stream);
+
+/*
  * gdn_decode_step -- one token for each of B sequences; conv and recurrent state in place.
  * Source: as gdn_chunk_prefill with T = 1 per sequence; states resident in a slot pool, fp32
  * recurrent state as the "Qwen3-Next" SGLang cookbook's default --mamba-ssm-dtype.

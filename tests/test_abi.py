@@ -152,6 +152,23 @@ def test_block_prefill_argument_errors(L):
                                None) == gdn.GDN_OK
 
 
+def test_prefill_slots_argument_errors(L):
+    d = ctypes.byref(gdn.Dims())
+    f = L.gdn_chunk_prefill_slots
+
+    def call(dims=d, dtype=1, x=A, N=1, T=16, slot=A, pool=A, conv=A, ws=A, ws_bytes=1 << 40):
+        return f(dims, dtype, x, None, A, A, None, None, A, N, T, slot, pool, conv, A, ws, ws_bytes,
+                 None, None)
+    assert call(pool=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(pool=MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert call(conv=MIS) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dims=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(dtype=5) == gdn.GDN_ERR_UNSUPPORTED
+    assert call(ws=None) == gdn.GDN_ERR_WORKSPACE
+    assert call(x=None) == gdn.GDN_ERR_INVALID_ARG
+    assert call(N=0, T=0, pool=None, slot=None, conv=None) == gdn.GDN_OK
+
+
 def test_zero_size_calls_launch_nothing(L):
     d = ctypes.byref(gdn.Dims())
     # no sequences, no tokens: valid and a no-op
