@@ -136,7 +136,8 @@ int gdn_block_prefill(const gdn_dims* dims, int32_t hidden, const void* h, const
                       const float* S0, float* SN, const void* conv0, void* convN, void* y,
                       void* workspace, size_t workspace_bytes, int32_t* dev_status,
                       void* stream) {
-  if (!dims || hidden <= 0 || hidden % 8 != 0 || num_seqs < 0 || num_tokens < 0)
+  if (!dims || hidden <= 0 || hidden % 8 != 0 || num_seqs < 0 || num_tokens < 0 ||
+      (num_seqs == 0 && num_tokens > 0))
     return GDN_ERR_INVALID_ARG;
   const size_t need = gdn_block_prefill_workspace_size(dims, hidden, num_seqs, num_tokens);
   if (need == 0) return GDN_ERR_INVALID_ARG;

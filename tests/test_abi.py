@@ -138,6 +138,7 @@ def test_block_prefill_argument_errors(L):
     assert _block(L, d, hidden=0) == gdn.GDN_ERR_INVALID_ARG
     assert _block(L, d, hidden=260) == gdn.GDN_ERR_INVALID_ARG      # rows of 16-byte multiples
     assert _block(L, d, N=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert _block(L, d, N=0) == gdn.GDN_ERR_INVALID_ARG              # tokens, no sequences
     assert _block(L, d, h=None) == gdn.GDN_ERR_INVALID_ARG
     assert _block(L, d, y=None) == gdn.GDN_ERR_INVALID_ARG
     assert _block(L, d, a_log=None) == gdn.GDN_ERR_INVALID_ARG
