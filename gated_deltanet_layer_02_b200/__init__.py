@@ -31,7 +31,8 @@ EXPORTS = (
     "gdn_trace_reset", "gdn_trace_count", "gdn_trace_get", "gdn_debug_wait_probe",
     "gdn_chunk_prefill_static_ws", "gdn_trace_span", "gdn_decode_step_bf16_state",
     "gdn_chunk_prefill_states", "gdn_decode_multi", "gdn_block_prefill_workspace_size",
-    "gdn_block_prefill", "gdn_chunk_prefill_slots",
+    "gdn_block_prefill", "gdn_chunk_prefill_slots", "gdn_chunk_prefill_host_plan",
+    "gdn_chunk_prefill_host_workspace_size", "gdn_chunk_prefill_host",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
@@ -96,6 +97,12 @@ def lib():
             L.gdn_chunk_prefill_slots.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
                                                   i32, i32, vp, vp, vp, vp, vp, ctypes.c_size_t,
                                                   vp, vp]
+            L.gdn_chunk_prefill_host_plan.argtypes = [vp, i32, i32, i32, vp, i32]
+            L.gdn_chunk_prefill_host_plan.restype = ctypes.c_int32
+            L.gdn_chunk_prefill_host_workspace_size.argtypes = [dp, vp, i32, i32, i32]
+            L.gdn_chunk_prefill_host_workspace_size.restype = ctypes.c_size_t
+            L.gdn_chunk_prefill_host.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp,
+                                                 vp, vp, vp, i32, vp, ctypes.c_size_t, vp, vp]
             L.gdn_block_prefill_workspace_size.argtypes = [dp, i32, i32, i32]
             L.gdn_block_prefill_workspace_size.restype = ctypes.c_size_t
             L.gdn_block_prefill.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
@@ -260,6 +267,70 @@ def chunk_prefill_slots(x, beta, g, cu_seqlens, S_pool, slot_idx=None, conv_pool
     return out
 
 
+def _hptr(t, name, dtype, allow_none=True):
+    """Pointer of a host (CPU) tensor."""
+    if t is None:
+        if not allow_none:
+            raise ValueError(f"{name} is required")
+        return None
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a CPU tensor (host memory)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def host_plan(cu_seqlens, segment_tokens: int = 0):
+    """The segments gdn_chunk_prefill_host cuts a batch into: [k, 4] int32 rows
+    (first sequence, sequences, first token, tokens).  cu_seqlens: CPU int32."""
+    cu = cu_seqlens.to(torch.int32).contiguous()
+    N, T = cu.numel() - 1, int(cu[-1]) if cu.numel() else 0
+    L = lib()
+    n = L.gdn_chunk_prefill_host_plan(_hptr(cu, "cu_seqlens", torch.int32), N, T,
+                                      segment_tokens, None, 0)
+    _check("gdn_chunk_prefill_host_plan", min(n, 0))
+    segs = torch.zeros((max(n, 1), 4), dtype=torch.int32)
+    n2 = L.gdn_chunk_prefill_host_plan(_hptr(cu, "cu_seqlens", torch.int32), N, T,
+                                       segment_tokens, _hptr(segs, "segments", torch.int32), n)
+    _check("gdn_chunk_prefill_host_plan", min(n2, 0))
+    return segs[:n]
+
+
+def chunk_prefill_host(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None, SN=None,
+                       conv0=None, convN=None, out=None, workspace=None, segment_tokens: int = 0,
+                       dev_status=None, dims: Dims | None = None):
+    """chunk_prefill (bf16) with x, beta, g, z, cu_seqlens and out in HOST memory (pin them for
+    the copies to overlap the kernels); weights, states and the workspace on the device.
+    Returns (out, SN, convN); out is valid once the current stream has reached the call."""
+    dims = dims or Dims()
+    T = x.shape[0]
+    N = cu_seqlens.numel() - 1
+    Hv, d, K = dims.num_v_heads, dims.head_dim, dims.conv_kernel
+    dev = torch.device("cuda", torch.cuda.current_device())
+    bf = torch.bfloat16
+    if out is None:
+        out = torch.empty((T, Hv, d), dtype=bf, pin_memory=True)
+    if SN is None:
+        SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
+    if convN is None:
+        convN = torch.empty((N, K - 1, dims.channels), dtype=bf, device=dev)
+    cu_p = _hptr(cu_seqlens, "cu_seqlens", torch.int32, allow_none=False)
+    need = lib().gdn_chunk_prefill_host_workspace_size(ctypes.byref(dims), cu_p, N, T,
+                                                       segment_tokens)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    _check("gdn_chunk_prefill_host", lib().gdn_chunk_prefill_host(
+        ctypes.byref(dims), _hptr(x, "x", bf), _ptr(conv_w, "conv_w", bf),
+        _hptr(beta, "beta", torch.float32), _hptr(g, "g", torch.float32), _hptr(z, "z", bf),
+        _ptr(norm_w, "norm_w", bf), cu_p, N, T, _ptr(S0, "S0", torch.float32),
+        _ptr(SN, "SN", torch.float32), _ptr(conv0, "conv0", bf), _ptr(convN, "convN", bf),
+        _hptr(out, "out", bf), segment_tokens, _ptr(workspace, "workspace", torch.uint8),
+        workspace.numel(), _ptr(dev_status, "dev_status", torch.int32), _stream()))
+    return out, SN, convN
+
+
 def chunk_prefill_static_ws(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None,
                             SN=None, conv0=None, convN=None, out=None, dev_status=None,
                             want_state=True, dims: Dims | None = None):
@@ -421,6 +492,7 @@ class Trace:
 
 __all__ = ["Dims", "GdnError", "lib", "conv1d_update", "gated_rmsnorm", "chunk_prefill",
            "decode_multi", "block_prefill", "chunk_prefill_slots",
+           "chunk_prefill_host", "host_plan",
            "chunk_prefill_static_ws", "STATIC_WORKSPACE_BYTES",
            "decode_step", "prefill_workspace_size", "conv_channels", "status_string", "Trace",
            "debug_wait_probe", "EXPORTS", "LIB_PATH"]

@@ -114,6 +114,10 @@ bool dtype_ok(gdn_dtype t) { return t == GDN_F32 || t == GDN_BF16; }
 
 }  // namespace
 
+namespace gdn_host {
+int check_dims_ext(const gdn_dims* d) { return check_dims(d); }
+}  // namespace gdn_host
+
 extern "C" {
 
 int gdn_abi_version(void) { return GDN_ABI_VERSION; }

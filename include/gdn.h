@@ -153,6 +153,42 @@ int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* 
                              void* stream);
 
 /*
+ * gdn_chunk_prefill_host -- gdn_chunk_prefill (bf16) with the per-token tensors in host memory.
+ * Source: as gdn_chunk_prefill.  The packed batch is cut into segments of about segment_tokens
+ * tokens, ending at sequence ends or 128-token chunk boundaries of a sequence; the copy of one
+ * segment's inputs to the device, the layer on the previous segment and the copy of the output
+ * before that back to the host overlap on the library's two copy streams and `stream`.  A
+ * sequence cut between segments carries its fp32 state and conv history from one to the next,
+ * so the result equals one gdn_chunk_prefill call on device copies of the same inputs.
+ *   x [T, Cc], beta, g [T, Hv] fp32, z [T, Hv, d] (nullable), out [T, Hv, d]: HOST memory
+ *     (page-locked for the copies to overlap; pageable memory works, serialised).
+ *   cu_seqlens_host [N+1] int32: HOST memory, cu[0] = 0, non-decreasing, cu[N] = T.
+ *   conv_w, norm_w, S0, SN, conv0, convN, dev_status: device, as gdn_chunk_prefill.
+ *   segment_tokens: a multiple of 128, or 0 for the library's choice (T / 8 rounded up to 128,
+ *     at least 512).
+ *   workspace: device, gdn_chunk_prefill_host_workspace_size() bytes, 256-byte aligned (it
+ *     holds device copies of the per-token tensors).
+ * Asynchronous on `stream`: the host buffers may be reused, and out read, once `stream` has
+ * reached the point of the call.  Not for stream capture (the copy streams are the library's).
+ * Status codes as gdn_chunk_prefill; GDN_ERR_UNSUPPORTED unless Hv = 2 Hk and Hv % 4 == 0.
+ * gdn_chunk_prefill_host_plan writes the segments (first sequence, sequences, first token,
+ * tokens; four int32 each) into `segments` and returns their number (or a status < 0;
+ * GDN_ERR_WORKSPACE when max_segments is too small; segments may be NULL to count).
+ */
+int32_t gdn_chunk_prefill_host_plan(const int32_t* cu_seqlens_host, int32_t num_seqs,
+                                    int32_t num_tokens, int32_t segment_tokens,
+                                    int32_t* segments, int32_t max_segments);
+size_t gdn_chunk_prefill_host_workspace_size(const gdn_dims* dims, const int32_t* cu_seqlens_host,
+                                             int32_t num_seqs, int32_t num_tokens,
+                                             int32_t segment_tokens);
+int gdn_chunk_prefill_host(const gdn_dims* dims, const void* x, const void* conv_w,
+                           const float* beta, const float* g, const void* z, const void* norm_w,
+                           const int32_t* cu_seqlens_host, int32_t num_seqs, int32_t num_tokens,
+                           const float* S0, float* SN, const void* conv0, void* convN, void* out,
+                           int32_t segment_tokens, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_status, void* stream);
+
+/*
  * gdn_chunk_prefill_slots -- gdn_chunk_prefill whose initial and final states live in a state
  * pool shared with gdn_decode_step: sequence n reads and overwrites row slot_idx[n] of the pools.
  * Source: the "Qwen3-Next" SGLang cookbook, section 3.2 (the mamba state cache of the hybrid GDN
