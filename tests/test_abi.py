@@ -222,3 +222,31 @@ def test_static_workspace_entry_point_rejects_oversized_calls(L):
                                          *tail) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_chunk_prefill_static_ws(ctypes.byref(gdn.Dims(head_dim=64)), 1, A, None, A, A,
                                          None, None, A, 1, 16, *tail) == gdn.GDN_ERR_UNSUPPORTED
+
+
+def test_plain_c_consumer(L, tmp_path):
+    """include/gdn.h compiles as C99 (-pedantic) and a C program links libgdn.so and calls it."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "consumer.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "gdn.h"\n'
+        "int main(void) {\n"
+        "  gdn_dims d = {16, 32, 128, 4, 1.0f, 1e-6f, 1e-6f};\n"
+        "  int32_t cu[3] = {0, 300, 429};\n"
+        "  int32_t seg[8];\n"
+        "  int n = gdn_chunk_prefill_host_plan(cu, 2, 429, 256, seg, 2);\n"
+        '  printf("%d %d %lld %s %d %d %d %d\\n", gdn_abi_version(), n,\n'
+        "         (long long)gdn_conv_channels(&d), gdn_status_string(GDN_ERR_WORKSPACE),\n"
+        "         seg[4], seg[5], seg[6], seg[7]);\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "consumer"
+    lib_dir = os.path.dirname(gdn.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", lib_dir, "-l:libgdn.so", f"-Wl,-rpath,{lib_dir}"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out == ["1", "2", "8192", "workspace", "too", "small", "0", "2", "256", "173"]
