@@ -18,7 +18,9 @@ The kernels also rely on two facts checked here:
   * each 64-token inverse from its two 32-token diagonal inverses, both at once:
     T_h = D - D L1 D, D = blockdiag of the four 32-token inverses, L1 = the blocks (1,0) and
     (3,2) of A (exact: (L1 D)^2 = 0 inside each 64-token block);
-  * the 32-token inverses by row substitution T[l] = e_l - sum_{j<l} A[l][j] T[j].
+  * the 32-token inverses by row substitution T[l] = e_l - sum_{j<l} A[l][j] T[j];
+  * d_v column blocks of the state evolve independently (the chain's split across CTAs);
+  * the look-ahead form of the chain step, X_(c+1) = e^(G_L) W_(c+1) S_c^T + E_(c+1) U^_c.
 """
 import numpy as np
 import pytest
@@ -142,3 +144,47 @@ def test_two_level_block_inverse_assembly(g_low):
     np.testing.assert_allclose(Th[:64, :64], np.linalg.inv(np.eye(64) + A[:64, :64]),
                                rtol=1e-10, atol=1e-12)
     np.testing.assert_allclose(T, np.linalg.inv(np.eye(C) + A), rtol=1e-10, atol=1e-12)
+
+
+def _chunk_terms(Q, K, V, b, gg):
+    G = np.cumsum(gg)
+    A = b[:, None] * _masked_decay(G, True) * (K @ K.T)
+    Tm = np.linalg.inv(np.eye(len(G)) + A)
+    return G, Tm @ ((b * np.exp(G))[:, None] * K), Tm @ (b[:, None] * V)
+
+
+@pytest.mark.parametrize("g_low", [-0.05, -1.5])
+def test_look_ahead_product_of_the_chain(g_low):
+    """X of chunk c+1 from the state entering chunk c: with U^_c = diag(e^(G_L - G)) U_c and
+    E_(c+1) = W_(c+1) K_c^T (available before the chain reaches chunk c),
+    X_(c+1) = W_(c+1) S_(c+1)^T = e^(G_L) W_(c+1) S_c^T + E_(c+1) U^_c, so one product follows
+    U_c instead of two (the form measured as the look-ahead chain)."""
+    C, d = 32, 16
+    q, k, v, beta, g, S0 = _normalised_inputs(61, [2 * C], 1, 1, d, g_low)
+    k = k[:, 0] / np.linalg.norm(k[:, 0], axis=1, keepdims=True)
+    v, b, gg = v[:, 0], beta[:, 0].astype(np.float64), g[:, 0].astype(np.float64)
+    S = S0[0, 0].astype(np.float64)
+    G0, W0, Ut0 = _chunk_terms(None, k[:C], v[:C], b[:C], gg[:C])
+    G1, W1, Ut1 = _chunk_terms(None, k[C:], v[C:], b[C:], gg[C:])
+    U0 = Ut0 - W0 @ S.T
+    Uhat = np.exp(G0[-1] - G0)[:, None] * U0
+    S1 = np.exp(G0[-1]) * S + Uhat.T @ k[:C]
+    X1 = W1 @ S1.T
+    E1 = W1 @ k[:C].T
+    np.testing.assert_allclose(np.exp(G0[-1]) * (W1 @ S.T) + E1 @ Uhat, X1, rtol=1e-11,
+                               atol=1e-11)
+
+
+def test_value_column_blocks_evolve_independently():
+    """Each d_v block of the state (rows of S, columns of V and U) follows the recurrence on its
+    own: the chain may split d_v across CTAs with no exchange."""
+    lengths, d = [70], 16
+    q, k, v, beta, g, S0 = _normalised_inputs(62, lengths, 1, 1, d, -0.5)
+    qn = q[:, 0] / np.linalg.norm(q[:, 0], axis=1, keepdims=True)
+    kn = k[:, 0] / np.linalg.norm(k[:, 0], axis=1, keepdims=True)
+    b, gg, S = beta[:, 0].astype(np.float64), g[:, 0].astype(np.float64), S0[0, 0].astype(np.float64)
+    full_o, full_S = chunked_head(qn, kn, v[:, 0], b, gg, S, 16)
+    for c0 in range(0, d, 4):
+        o, Sb = chunked_head(qn, kn, v[:, 0, c0:c0 + 4], b, gg, S[c0:c0 + 4], 16)
+        np.testing.assert_allclose(o, full_o[:, c0:c0 + 4], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(Sb, full_S[c0:c0 + 4], rtol=1e-12, atol=1e-12)
