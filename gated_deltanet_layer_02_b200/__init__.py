@@ -150,6 +150,23 @@ def _ptr(t, name, dtype=None, allow_none=True):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _need(t, name, n):
+    """The C ABI takes bare pointers: refuse a tensor too small for what the call touches."""
+    if t is not None and t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call needs {n}")
+
+
+def _need_layer(dims, T, N, x=None, beta=None, g=None, z=None, out=None, conv_w=None,
+                norm_w=None, S0=None, SN=None, conv0=None, convN=None):
+    Cc, Hv, d, K = dims.channels, dims.num_v_heads, dims.head_dim, dims.conv_kernel
+    for t, name, n in ((x, "x", T * Cc), (beta, "beta", T * Hv), (g, "g", T * Hv),
+                       (z, "z", T * Hv * d), (out, "out", T * Hv * d), (conv_w, "conv_w", Cc * K),
+                       (norm_w, "norm_w", d), (S0, "S0", N * Hv * d * d),
+                       (SN, "SN", N * Hv * d * d), (conv0, "conv0", N * (K - 1) * Cc),
+                       (convN, "convN", N * (K - 1) * Cc)):
+        _need(t, name, n)
+
+
 def _act_dtype(t):
     if t.dtype == torch.bfloat16:
         return GDN_BF16
@@ -173,6 +190,11 @@ def conv1d_update(x, conv_w, cu_seqlens, conv_state_in=None, conv_state_out=None
     dt = _act_dtype(x)
     y = torch.empty_like(x) if y is None else y
     N = cu_seqlens.numel() - 1
+    Cc, K, T = dims.channels, dims.conv_kernel, x.shape[0]
+    for t, name, n in ((x, "x", T * Cc), (y, "y", T * Cc), (conv_w, "conv_w", Cc * K),
+                       (conv_state_in, "conv_state_in", N * (K - 1) * Cc),
+                       (conv_state_out, "conv_state_out", N * (K - 1) * Cc)):
+        _need(t, name, n)
     _check("gdn_conv1d_update", lib().gdn_conv1d_update(
         ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(y, "y", x.dtype),
         _ptr(conv_w, "conv_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N,
@@ -187,6 +209,9 @@ def gated_rmsnorm(o, z, w=None, eps: float = 1e-6, y=None):
     y = torch.empty_like(o) if y is None else y
     dim = o.shape[-1]
     rows = o.numel() // dim if dim else 0
+    _need(z, "z", rows * dim)
+    _need(y, "y", rows * dim)
+    _need(w, "w", dim)
     _check("gdn_gated_rmsnorm", lib().gdn_gated_rmsnorm(
         dt, _ptr(o, "o", o.dtype), _ptr(z, "z", o.dtype), _ptr(w, "w", o.dtype), float(eps),
         rows, dim, _ptr(y, "y", o.dtype), _stream()))
@@ -223,6 +248,7 @@ def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=N
         SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
     if want_state and convN is None:
         convN = torch.empty((N, K - 1, dims.channels), dtype=x.dtype, device=dev)
+    _need_layer(dims, T, N, x, beta, g, z, out, conv_w, norm_w, S0, SN, conv0, convN)
     need = prefill_workspace_size(N, T, x.dtype, dims)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
@@ -256,6 +282,11 @@ def chunk_prefill_slots(x, beta, g, cu_seqlens, S_pool, slot_idx=None, conv_pool
     if workspace is None:
         workspace = torch.empty(max(prefill_workspace_size(N, T, x.dtype, dims), 256),
                                 dtype=torch.uint8, device=x.device)
+    _need_layer(dims, T, N, x, beta, g, z, out, conv_w, norm_w)
+    if slot_idx is None:   # identity slots: rows 0 .. N-1 of the pools
+        _need(S_pool, "S_pool", N * dims.num_v_heads * dims.head_dim ** 2)
+        _need(conv_pool, "conv_pool", N * (dims.conv_kernel - 1) * dims.channels)
+    _need(slot_idx, "slot_idx", N)
     _check("gdn_chunk_prefill_slots", lib().gdn_chunk_prefill_slots(
         ctypes.byref(dims), _act_dtype(x), _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
         _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
@@ -316,6 +347,7 @@ def chunk_prefill_host(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None,
         SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
     if convN is None:
         convN = torch.empty((N, K - 1, dims.channels), dtype=bf, device=dev)
+    _need_layer(dims, T, N, x, beta, g, z, out, conv_w, norm_w, S0, SN, conv0, convN)
     cu_p = _hptr(cu_seqlens, "cu_seqlens", torch.int32, allow_none=False)
     need = lib().gdn_chunk_prefill_host_workspace_size(ctypes.byref(dims), cu_p, N, T,
                                                        segment_tokens)
@@ -352,6 +384,7 @@ def chunk_prefill_static_ws(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=
         SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
     if want_state and convN is None:
         convN = torch.empty((N, K - 1, dims.channels), dtype=x.dtype, device=dev)
+    _need_layer(dims, T, N, x, beta, g, z, out, conv_w, norm_w, S0, SN, conv0, convN)
     _check("gdn_chunk_prefill_static_ws", lib().gdn_chunk_prefill_static_ws(
         ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
         _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
@@ -372,6 +405,11 @@ def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx
     if out is None:
         out = torch.empty((B, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
     bf16_state = S is not None and S.dtype == torch.bfloat16
+    _need_layer(dims, B, 0, x, beta, g, z, out, conv_w, norm_w)
+    if slot_idx is None:   # identity slots: rows 0 .. B-1 of the pools
+        _need(S, "S", B * dims.num_v_heads * dims.head_dim ** 2)
+        _need(conv_state, "conv_state", B * (dims.conv_kernel - 1) * dims.channels)
+    _need(slot_idx, "slot_idx", B)
     name = "gdn_decode_step_bf16_state" if bf16_state else "gdn_decode_step"
     _check(name, getattr(lib(), name)(
         ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype, False),
@@ -392,6 +430,12 @@ def decode_multi(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_id
     B, k = x.shape[0], x.shape[1]
     if out is None:
         out = torch.empty((B, k, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
+    _need_layer(dims, B * k, 0, x, beta, g, z, out, conv_w, norm_w)
+    if slot_idx is None:   # identity slots: rows 0 .. B-1 of the pools
+        _need(S, "S", B * dims.num_v_heads * dims.head_dim ** 2)
+        _need(conv_state, "conv_state", B * (dims.conv_kernel - 1) * dims.channels)
+    _need(slot_idx, "slot_idx", B)
+    _need(snapshots, "snapshots", B * k * dims.num_v_heads * dims.head_dim ** 2)
     _check("gdn_decode_multi", lib().gdn_decode_multi(
         ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype, False),
         _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
@@ -417,6 +461,13 @@ def block_prefill(h, w_qkv, w_z, w_ba, a_log, dt_bias, w_out, cu_seqlens, conv_w
         SN = torch.empty((N, Hv, d, d), dtype=torch.float32, device=dev)
     if convN is None:
         convN = torch.empty((N, K - 1, dims.channels), dtype=h.dtype, device=dev)
+    Cc, HD = dims.channels, Hv * d
+    for t, name, n in ((h, "h", T * H), (y, "y", T * H), (w_qkv, "w_qkv", H * Cc),
+                       (w_z, "w_z", H * HD), (w_ba, "w_ba", H * 2 * Hv), (a_log, "a_log", Hv),
+                       (dt_bias, "dt_bias", Hv), (w_out, "w_out", HD * H)):
+        _need(t, name, n)
+    _need_layer(dims, T, N, conv_w=conv_w, norm_w=norm_w, S0=S0, SN=SN, conv0=conv0,
+                convN=convN)
     need = lib().gdn_block_prefill_workspace_size(ctypes.byref(dims), H, N, T)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)

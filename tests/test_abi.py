@@ -250,3 +250,54 @@ def test_plain_c_consumer(L, tmp_path):
                     "-L", lib_dir, "-l:libgdn.so", f"-Wl,-rpath,{lib_dir}"], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
     assert out == ["1", "2", "8192", "workspace", "too", "small", "0", "2", "256", "173"]
+
+
+def test_binding_refuses_undersized_buffers(L):
+    """The binding checks every buffer against the sizes the call touches before it hands bare
+    pointers to the library (CPU tensors: the size check comes before the device check)."""
+    import torch
+    d = gdn.Dims(2, 4)
+    T, N, Cc, Hv = 10, 1, d.channels, d.num_v_heads
+    cu = torch.tensor([0, T], dtype=torch.int32)
+    ok = dict(x=torch.zeros(T, Cc, dtype=torch.bfloat16), beta=torch.zeros(T, Hv),
+              g=torch.zeros(T, Hv))
+    with pytest.raises(ValueError, match="CUDA"):          # sizes fine: stops at the device check
+        gdn.chunk_prefill(ok["x"], ok["beta"], ok["g"], cu, dims=d)
+    with pytest.raises(ValueError, match="beta holds"):
+        gdn.chunk_prefill(ok["x"], ok["beta"][:5], ok["g"], cu, dims=d)
+    with pytest.raises(ValueError, match="x holds"):
+        gdn.chunk_prefill(ok["x"][:, :512], ok["beta"], ok["g"], cu, dims=d)
+    with pytest.raises(ValueError, match="S0 holds"):
+        gdn.chunk_prefill(ok["x"], ok["beta"], ok["g"], cu, S0=torch.zeros(1, Hv, 128, 64),
+                          dims=d)
+    with pytest.raises(ValueError, match="conv_w holds"):
+        gdn.chunk_prefill(ok["x"], ok["beta"], ok["g"], cu, dims=d,
+                          conv_w=torch.zeros(Cc, 3, dtype=torch.bfloat16))
+    B = 3
+    xs = torch.zeros(B, Cc, dtype=torch.bfloat16)
+    cw = torch.zeros(Cc, 4, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="S holds"):       # identity slots need B state rows
+        gdn.decode_step(xs, torch.zeros(B, Hv), torch.zeros(B, Hv),
+                        torch.zeros(B, 3, Cc, dtype=torch.bfloat16),
+                        torch.zeros(B - 1, Hv, 128, 128), cw, dims=d)
+    with pytest.raises(ValueError, match="slot_idx holds"):
+        gdn.decode_step(xs, torch.zeros(B, Hv), torch.zeros(B, Hv),
+                        torch.zeros(1, 3, Cc, dtype=torch.bfloat16),
+                        torch.zeros(1, Hv, 128, 128), cw, slot_idx=torch.zeros(2, dtype=torch.int32),
+                        dims=d)
+    with pytest.raises(ValueError, match="snapshots holds"):
+        gdn.decode_multi(torch.zeros(B, 2, Cc, dtype=torch.bfloat16), torch.zeros(B, 2, Hv),
+                         torch.zeros(B, 2, Hv), torch.zeros(B, 3, Cc, dtype=torch.bfloat16),
+                         torch.zeros(B, Hv, 128, 128), cw,
+                         snapshots=torch.zeros(B, 1, Hv, 128, 128), dims=d)
+    with pytest.raises(ValueError, match="z holds"):
+        gdn.gated_rmsnorm(torch.zeros(4, 128, dtype=torch.bfloat16),
+                          torch.zeros(3, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="w_out holds"):
+        H = 256
+        gdn.block_prefill(torch.zeros(T, H, dtype=torch.bfloat16),
+                          torch.zeros(H, Cc, dtype=torch.bfloat16),
+                          torch.zeros(H, Hv * 128, dtype=torch.bfloat16),
+                          torch.zeros(H, 2 * Hv, dtype=torch.bfloat16), torch.zeros(Hv),
+                          torch.zeros(Hv), torch.zeros(Hv * 128, H - 1, dtype=torch.bfloat16),
+                          cu, dims=d)
