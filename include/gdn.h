@@ -22,7 +22,10 @@
  *
  * General rules for every call:
  *   - Pointers are DEVICE pointers owned by the caller unless a comment says "host".  The
- *     library allocates no device memory and keeps no global state between calls.
+ *     library allocates no device memory of its own, except where an entry point says so
+ *     (gdn_chunk_prefill_static_ws: a static array; gdn_block_prefill: a cuBLAS handle).  Its
+ *     multi-stream paths create CUDA streams and events once per host thread and device and
+ *     keep them; no other state survives a call.
  *   - Tensors are dense, row-major, contiguous and 16-byte aligned.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *   - Return value: GDN_OK, or a negative gdn_status.  On argument errors nothing is launched
