@@ -3,14 +3,18 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one gdn_chunk_prefill of the T=4096 Qwen3-Next layer workload (16 key heads, 32 value
-heads, d = 128, bf16 activations, fp32 state, conv + SiLU + L2 norms + gated delta rule + gated
-RMSNorm, final recurrent and conv states returned), inputs resident in HBM, L2 flushed between
-timed steps.  `value` is whole-job tokens/s.  Alongside: the per-kernel roofline of the
-dominant kernel, the whole-step fractions of tensor and HBM peak, an end-to-end figure through
-the C ABI with host buffers, the decode workload (256 sequences x 64 steps, state GB/s) and the
-fp64 CPU oracle timed on this host.  N > 1 (torchrun, one process per GPU) runs independent
-replicas (the layer needs no collective): weak scaling, max time over ranks.
+Headline: one gdn_chunk_prefill of the long-context workload (one sequence of T = 262,144
+tokens, the model card's native context; 16 key heads, 32 value heads, d = 128, bf16
+activations, fp32 state; conv + SiLU + L2 norms + gated delta rule + gated RMSNorm, final
+recurrent and conv states returned), inputs resident in HBM, L2 flushed between timed steps.
+Each timed step is one replay of the step's CUDA graph, with the library's launch trace
+captured into the graph, so the per-kernel times (and the dominant kernel's roofline) come
+from the same timed replays.  `value` is whole-job tokens/s.  Alongside: the T = 4096 and the
+8-sequence variable-length prefill workloads (same figures each), an end-to-end figure of the
+headline through the C ABI with host buffers, the decode workload (256 sequences x 64 steps,
+state GB/s) and its bf16-state and 4-token variants, and the fp64 CPU oracle timed on this
+host on a bounded sample.  N > 1 (torchrun, one process per GPU) runs independent replicas
+(the layer needs no collective): weak scaling, max time over ranks.
 """
 from __future__ import annotations
 
@@ -50,7 +54,6 @@ def flops_per_token_by_kernel(w, C=CHUNK):
         "gdn_chain": 2.0 * (Hv * 2.0 * d * d),                               # W S^T, K^T U
         "gdn_out": 2.0 * (Hv * (d * d + C * d / 2.0) + Hk * C * d / 2.0),    # Q K^T, Q S^T, P U
     }
-    f["gdn_prep_chain"] = f["gdn_prep"] + f["gdn_chain"]  # the opt-in persistent kernel
     return f
 
 
@@ -61,7 +64,6 @@ def bytes_per_token_by_kernel(w):
     Hv, d = w.num_v_heads, w.head_dim
     b = {"gdn_qkv": w.channels * esz, "gdn_prep": 2 * Hv * 4, "gdn_chain": 0,
          "gdn_out": 2 * Hv * d * esz}
-    b["gdn_prep_chain"] = b["gdn_prep"]
     return b
 
 
@@ -91,8 +93,10 @@ def source_hash(family="prefill"):
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel's sources are unchanged."""
+def ncu_traffic(kernel, tokens_per_launch=None):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's sources are unchanged.
+    A prefill capture covers `capture_tokens` tokens per launch; the figure is scaled to
+    `tokens_per_launch` (the traffic of these kernels grows with the chunks they process)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
@@ -100,10 +104,13 @@ def ncu_traffic(kernel):
     except Exception:
         return None
     k = t.get("kernels", {}).get(kernel)
-    family = "decode_step" if kernel == "decode_step" else "prefill"
+    family = "decode_step" if kernel.startswith("decode") else "prefill"
     if k is None or k.get("source_hash") != source_hash(family):
         return None
-    return float(k["dram_bytes_per_launch_full_size"])
+    b = float(k["dram_bytes_per_launch"])
+    if tokens_per_launch is not None and k.get("capture_tokens"):
+        b *= tokens_per_launch / float(k["capture_tokens"])
+    return b
 
 
 # ------------------------------------------------------------------------------- clocks
@@ -166,11 +173,13 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- the arms
-def cpu_oracle_rate(w, seed, budget_s=10.0, cap_s=30.0):
-    """The fp64 oracle as it stands, on this host's cores, over whole copies of the workload
-    until at least budget_s of CPU work has run (at least one copy)."""
+def cpu_oracle_rate(w, seed, budget_s=10.0, cap_s=30.0, sample_tokens=4096):
+    """The fp64 oracle as it stands, on this host's cores, over a bounded sample of the workload:
+    the first `sample_tokens` tokens of its (first) sequence, repeated until at least budget_s
+    of CPU work has run (at least one copy)."""
     import oracle
-    inp = inputs.prefill_inputs(w, seed)
+    sample = min(sample_tokens, w.tokens)
+    inp = inputs.prefill_inputs(w, seed, lengths=(sample,))
     dims = oracle.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
     threads = oracle.default_threads()
     done, t0 = 0, time.perf_counter()
@@ -182,8 +191,8 @@ def cpu_oracle_rate(w, seed, budget_s=10.0, cap_s=30.0):
         el = time.perf_counter() - t0
         if el >= budget_s or el * (done + 1) / done > cap_s:
             break
-    return {"value": done * w.tokens / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} full copies of the {w.tokens}-token workload ({el:.1f} s)"}
+    return {"value": done * sample / el, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} runs of the first {sample} tokens of {w.name} ({el:.1f} s)"}
 
 
 def run_reference(args, w, seed, rank):
@@ -222,9 +231,73 @@ def run_reference(args, w, seed, rank):
     }
 
 
-def bench_prefill(args, w, seed, dev, gdn):
+def _graph_of(step):
+    """The step's launches captured once as a CUDA graph (the library's trace, when attached,
+    records each launch's events as event-record nodes of the graph)."""
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize()
+    return graph
+
+
+def _kernel_table(per_step, T, w, peaks):
+    """Per-kernel figures from the traced replays: per_step is a list (one per timed step) of
+    [(name, ms)] launches.  Algorithmic work per step = per-token work x T; achieved = that work
+    / the kernel's summed launch time per step (= work per launch / mean launch time for
+    equal launches)."""
+    fl, by = flops_per_token_by_kernel(w), bytes_per_token_by_kernel(w)
+    kern = {}
+    for recs in per_step:
+        for name, ms in recs:
+            k = kern.setdefault(name, {"launches": 0, "total_ms": 0.0})
+            k["launches"] += 1
+            k["total_ms"] += ms
+    n = max(1, len(per_step))
+    tot = sum(k["total_ms"] for k in kern.values()) or 1.0
+    for name, k in kern.items():
+        k["launches_per_step"] = k["launches"] / n
+        k["ms_per_step"] = k["total_ms"] / n
+        k["avg_ms"] = k["total_ms"] / k["launches"]
+        k["share"] = k["total_ms"] / tot
+        if name in fl:
+            k["tflops"] = fl[name] * T / (k["ms_per_step"] * 1e-3) / 1e12
+            k["tc_frac"] = k["tflops"] / peaks["bf16_tflops"]
+            k["gbs"] = by[name] * T / (k["ms_per_step"] * 1e-3) / 1e9
+            k["hbm_frac"] = k["gbs"] / peaks["hbm_gbs"]
+    return kern
+
+
+def _roofline(kern, T, peaks, peak_src, tokens_per_launch):
+    """Roofline of the dominant kernel (largest time per step among the layer's kernels)."""
+    cands = [k for k in kern if "tflops" in kern[k]]
+    dom = max(cands, key=lambda k_: kern[k_]["ms_per_step"])
+    dk = kern[dom]
+    if dk["hbm_frac"] > dk["tc_frac"]:
+        roof = {"bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": dk["hbm_frac"]}
+    else:
+        roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": dk["tc_frac"]}
+    tr = ncu_traffic(dom, tokens_per_launch)
+    roof.update({"kernel": dom, "traffic": tr,
+                 "traffic_note": "ncu dram read+write per launch, scaled from the capture's "
+                                 "tokens to this launch's (profiles/traffic.json)"
+                 if tr is not None else "null: no ncu capture of the current sources",
+                 "peak_source": f"{peak_src} ({'burst bf16' if roof['bound'] == 'tensor' else 'copy'})"})
+    return roof
+
+
+def bench_prefill(args, w, seed, dev, gdn, peaks, peak_src, steps, warmup, e2e=True):
+    """One prefill workload: CUDA-graph replays of the whole step (the step time), then as many
+    replays of the step captured with the library's launch trace (per-kernel CUDA events of
+    every replay), L2 flushed (256 MiB write, untimed) before each replay; optionally the
+    end-to-end figure through the C ABI with host buffers."""
+    import gated_deltanet_layer_02_b200 as _g  # noqa: F401  (the binding, already built)
+    nvtx = torch.cuda.nvtx
+    nvtx.range_push(f"prefill {w.name}: setup")
     inp = inputs.prefill_inputs(w, seed)
-    host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
     T, N = w.tokens, len(w.lengths)
@@ -236,70 +309,90 @@ def bench_prefill(args, w, seed, dev, gdn):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def step(x=d["x"], beta=d["beta"], g=d["g"], z=d["z"], cu=d["cu_seqlens"], o=out):
-        gdn.chunk_prefill(x, beta, g, cu, conv_w=d["conv_w"], z=z, norm_w=d["norm_w"], S0=d["S0"],
-                          SN=SN, convN=convN, out=o, workspace=ws, dev_status=status, dims=dims)
+    def step():
+        gdn.chunk_prefill(d["x"], d["beta"], d["g"], d["cu_seqlens"], conv_w=d["conv_w"],
+                          z=d["z"], norm_w=d["norm_w"], S0=d["S0"], SN=SN, convN=convN, out=out,
+                          workspace=ws, dev_status=status, dims=dims)
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         step()
-    torch.cuda.synchronize()
-    # Headline: the step is captured once as a CUDA graph and replayed (host launch overhead
-    # stays out of the device timeline).
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        step()
-    torch.cuda.synchronize()
-    for _ in range(args.warmup):
-        flush.zero_()
-        graph.replay()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    if dist_on():
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for i in range(args.steps):
+    nvtx.range_pop()
+
+    def timed(graph, n_steps, tr=None):
+        ms, per = [], []
+        for _ in range(warmup):
             flush.zero_()
-            ev[i][0].record()
             graph.replay()
-            ev[i][1].record()
         torch.cuda.synchronize()
+        for i in range(n_steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+            if tr is not None:
+                per.append(tr.records())
+        return ms, per
+
+    # timed region: replays of the step's graph (the headline step time)
+    graph = _graph_of(step)
     if dist_on():
         torch.distributed.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
+    torch.cuda.synchronize()
+    nvtx.range_push(f"prefill {w.name}: timed")
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        step_ms, _ = timed(graph, steps)
+    nvtx.range_pop()
+    if dist_on():
+        torch.distributed.barrier()
     del graph
-    # Per-kernel breakdown: the same steps launched eagerly with the library's launch trace
-    # (CUDA events around every kernel on the launch stream).
+    # the same step captured with the library's launch trace (an event pair around every launch,
+    # recorded by each replay; launches in a traced capture go without programmatic dependent
+    # launch), replayed as many times: the per-kernel times of the roofline
+    nvtx.range_push(f"prefill {w.name}: traced")
     tr = gdn.Trace()
-    eager_ms = []
     with tr:
-        for i in range(args.steps):
-            flush.zero_()
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record()
-            step()
-            a1.record()
-            a1.synchronize()
-            eager_ms.append(a0.elapsed_time(a1))
-    recs = tr.records()
+        tgraph = _graph_of(step)
+    traced_ms, per_step = timed(tgraph, steps, tr)
+    del tgraph
     tr.close()
+    nvtx.range_pop()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the timed steps")
-    # end to end through the C ABI with host buffers (gdn_chunk_prefill_host): the inputs'
-    # host->device copies, the layer and the output's device->host copy, overlapped segment by
-    # segment inside the call, all inside the timed region
-    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    names = ("x", "beta", "g", "z", "cu_seqlens")
-    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    res = {"workload": w.name, "tokens": T, "sequences": N, "step_ms": step_ms,
+           "traced_graph_ms_per_step": statistics.mean(traced_ms),
+           "launches_per_step": len(per_step[0]) if per_step else 0,
+           "clocks": clk.summary()}
+    nseg = max(1, sum(1 for n_, _ in per_step[0] if n_ == "gdn_prep")) if per_step else 1
+    res["kernels"] = _kernel_table(per_step, T, w, peaks)
+    res["roofline"] = _roofline(res["kernels"], T, peaks, peak_src, T / nseg)
+    if e2e:
+        nvtx.range_push(f"prefill {w.name}: e2e")
+        res["e2e"] = _bench_e2e(args, w, inp, d, dims, dev, gdn, SN, convN, status, flush)
+        nvtx.range_pop()
+    return res
+
+
+def _bench_e2e(args, w, inp, d, dims, dev, gdn, SN, convN, status, flush):
+    """End to end through the C ABI with host buffers (gdn_chunk_prefill_host): the inputs'
+    host->device copies, the layer and the output's device->host copy, overlapped segment by
+    segment inside the call, all inside the timed region."""
+    T, N = w.tokens, len(w.lengths)
+    names = ("x", "beta", "g", "z")
+    host = {k: inp[k].pin_memory() for k in names}
+    out_h = torch.empty((T, w.num_v_heads, w.head_dim), dtype=w.dtype, pin_memory=True)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names) + inp["cu_seqlens"].numel() * 4
     d2h = out_h.numel() * out_h.element_size()
     cu_h = inp["cu_seqlens"]
     hws = torch.empty(gdn.lib().gdn_chunk_prefill_host_workspace_size(
         ctypes.byref(dims), ctypes.c_void_p(cu_h.data_ptr()), N, T, 0), dtype=torch.uint8,
         device=dev)
     e2e_ms = []
-    for i in range(args.warmup + max(3, args.steps // 10)):
+    reps = max(3, min(args.steps // 10, 20)) if T <= 65536 else 3
+    for i in range(args.warmup + reps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         flush.zero_()
         a.record()
@@ -312,7 +405,9 @@ def bench_prefill(args, w, seed, dev, gdn):
             e2e_ms.append(a.elapsed_time(b))
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the end-to-end steps")
-    return step_ms, recs, clk.summary(), (statistics.mean(e2e_ms), h2d, d2h), statistics.mean(eager_ms)
+    del hws, host, out_h
+    return {"ms_per_step": statistics.mean(e2e_ms), "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": reps}
 
 
 def bench_chunk_states(args, w, seed, dev, gdn):
@@ -358,7 +453,8 @@ def bench_chunk_states(args, w, seed, dev, gdn):
 
 
 def bench_block(w, seed, dev, gdn, hidden=2048, reps=20):
-    """The token mixer (gdn_block_prefill: cuBLAS projections, gates, the layer, output
+    """The token mixer (gdn_block_prefill: tcgen05 GEMM projections with the gates fused into the
+    [b | a] projection, the layer, output
     projection) on the same sequences, hidden size 2048, eager calls with L2 flushed in between.
     flops_per_step counts the four projection GEMMs only."""
     bw = inputs.custom(w.num_k_heads, w.num_v_heads, w.head_dim, w.dtype, lengths=w.lengths)
@@ -379,19 +475,34 @@ def bench_block(w, seed, dev, gdn, hidden=2048, reps=20):
     for _ in range(3):
         step()
     torch.cuda.synchronize()
-    ms = []
+    ms, per_kernel = [], {}
+    tr = gdn.Trace()
     for _ in range(reps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        step()
-        b.record()
+        tr.reset()
+        with tr:
+            a.record()
+            step()
+            b.record()
         b.synchronize()
         ms.append(a.elapsed_time(b))
+        for name, t_ in tr.records():
+            per_kernel.setdefault(name, []).append(t_)
+    tr.close()
     t = statistics.median(ms)
-    flops = 2 * T * hidden * (w.channels + 2 * Hv * dh + 2 * Hv)
+    C, HD = w.channels, Hv * dh
+    gemm_flops = {"gemm_qkv": 2 * T * hidden * C, "gemm_z": 2 * T * hidden * HD,
+                  "gemm_ba_gates": 2 * T * hidden * 2 * Hv, "gemm_out": 2 * T * HD * hidden}
+    gemms = {}
+    for name, f in gemm_flops.items():
+        if name in per_kernel:
+            k_ms = statistics.median(per_kernel[name])
+            gemms[name] = {"ms": k_ms, "tflops": f / (k_ms * 1e-3) / 1e12}
+    flops = sum(gemm_flops.values())
     return {"workload": f"{w.name}, hidden {hidden}", "ms_per_step": t,
-            "tokens_per_s": T / (t * 1e-3), "projection_flops_per_step": flops}
+            "tokens_per_s": T / (t * 1e-3), "projection_flops_per_step": flops,
+            "gemms": gemms}
 
 
 def bench_decode_multi(w, seed, dev, gdn, k=4, reps=20):
@@ -465,20 +576,43 @@ def job_tokens_per_s(world, tokens_per_rank, ms):
     return world * tokens_per_rank / (ms * 1e-3)
 
 
+#: the headline prefill workload (the largest single-GPU configuration: one 262,144-token
+#: sequence) and the secondary prefill workloads reported beside it
+HEADLINE = 4
+SECONDARY = (1, 2)
+
+
+def _prefill_line(res, n, peaks):
+    """Whole-step figures of one prefill workload (max over ranks already applied to ms)."""
+    T, ms = res["tokens"], res["ms_per_step"]
+    w = inputs.CONFIGS[res["config_index"]]
+    fl = flops_per_token_by_kernel(w)
+    by = bytes_per_token_by_kernel(w)
+    F = sum(v for k, v in fl.items())
+    B = sum(v for k, v in by.items())
+    value = job_tokens_per_s(n, T, ms)
+    return value, {"tc_frac": F * value / n / (peaks["bf16_tflops"] * 1e12),
+                   "hbm_frac": B * value / n / (peaks["hbm_gbs"] * 1e9),
+                   "flops_per_token": F, "bytes_per_token": B, "chunk": CHUNK,
+                   "flops_per_token_chunk64": sum(flops_per_token_by_kernel(w, 64).values())}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--headline-only", action="store_true",
+                    help="only the headline prefill leg (for profiling runs)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = inputs.CONFIGS[1]
-    seed = inputs.config_seed(1)
+    w = inputs.CONFIGS[HEADLINE]
+    seed = inputs.config_seed(HEADLINE)
     if args.impl == "reference":
         res = run_reference(args, w, seed, rank)
         if res is not None:
@@ -494,82 +628,81 @@ def main():
     from gated_deltanet_layer_02_b200 import build as gdn_build
     gdn_build.build()
     import gated_deltanet_layer_02_b200 as gdn
-
-    step_ms, recs, clocks, (e2e_ms, h2d, d2h), eager_ms = bench_prefill(args, w, seed, dev, gdn)
-    ms, e2e_ms = max_over_ranks([statistics.mean(step_ms), e2e_ms], dev)
-    n = world
-    T = w.tokens
-    value = job_tokens_per_s(n, T, ms)
     peaks, peak_src = load_peaks()
+    n = world
 
-    # per-kernel breakdown of the timed steps
-    kern = {}
-    for name, t in recs:
-        k = kern.setdefault(name, {"launches": 0, "total_ms": 0.0})
-        k["launches"] += 1
-        k["total_ms"] += t
-    fl = flops_per_token_by_kernel(w)
-    by = bytes_per_token_by_kernel(w)
-    tot = sum(k["total_ms"] for k in kern.values()) or 1.0
-    for name, k in kern.items():
-        k["avg_ms"] = k["total_ms"] / k["launches"]
-        k["share"] = k["total_ms"] / tot
-        if name in fl:
-            k["tflops"] = fl[name] * T / (k["avg_ms"] * 1e-3) / 1e12
-            k["tc_frac"] = k["tflops"] / peaks["bf16_tflops"]
-            k["gbs"] = by[name] * T / (k["avg_ms"] * 1e-3) / 1e9
-            k["hbm_frac"] = k["gbs"] / peaks["hbm_gbs"]
-    dom = max((n_ for n_ in kern if n_ in fl), key=lambda n_: kern[n_]["total_ms"])
-    dk = kern[dom]
-    if dk["hbm_frac"] > dk["tc_frac"]:
-        roof = {"bound": "hbm", "achieved": dk["gbs"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": dk["hbm_frac"]}
-    else:
-        roof = {"bound": "tensor", "achieved": dk["tflops"], "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": dk["tc_frac"]}
-    roof.update({"kernel": dom, "traffic": ncu_traffic(dom),
-                 "peak_source": f"{peak_src} ({'burst bf16' if roof['bound'] == 'tensor' else 'copy'})"})
-    F = sum(v for k, v in fl.items() if k != "gdn_prep_chain")
-    B = sum(v for k, v in by.items() if k != "gdn_prep_chain")
-    step_roof = {"tc_frac": F * value / n / (peaks["bf16_tflops"] * 1e12),
-                 "hbm_frac": B * value / n / (peaks["hbm_gbs"] * 1e9),
-                 "flops_per_token": F, "bytes_per_token": B, "chunk": CHUNK,
-                 "flops_per_token_chunk64": sum(v for k, v in flops_per_token_by_kernel(w, 64).items()
-                                                if k != "gdn_prep_chain")}
+    def run_prefill(idx, steps, e2e):
+        r = bench_prefill(args, inputs.CONFIGS[idx], inputs.config_seed(idx), dev, gdn, peaks,
+                          peak_src, steps, args.warmup, e2e=e2e)
+        r["config_index"] = idx
+        r["ms_per_step"], = max_over_ranks([statistics.mean(r.pop("step_ms"))], dev)
+        if "e2e" in r:
+            r["e2e"]["ms_per_step"], = max_over_ranks([r["e2e"]["ms_per_step"]], dev)
+        return r
 
-    dec_ms, dec_bytes, dec_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev, gdn,
-                                              args.decode_steps)
-    dec_ms = max_over_ranks([dec_ms], dev)[0]
-    dec_gbs = n * dec_bytes / (dec_ms * 1e-3) / 1e9
-    # the serving option of a bf16 recurrent state (same workload, half the state bytes)
-    d16_ms, d16_bytes, d16_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev, gdn,
-                                              args.decode_steps, torch.bfloat16)
-    d16_ms = max_over_ranks([d16_ms], dev)[0]
-    d16_gbs = n * d16_bytes / (d16_ms * 1e-3) / 1e9
-    dm_ms, dm_bytes, dm_tps = bench_decode_multi(inputs.CONFIGS[3], inputs.config_seed(3), dev,
-                                                 gdn)
-    dm_ms = max_over_ranks([dm_ms], dev)[0]
-    decode = {"workload": inputs.CONFIGS[3].name, "value": dec_gbs, "unit": "GB/s",
-              "ms_per_step": dec_ms, "steps": args.decode_steps,
-              "roofline": {"bound": "hbm", "achieved": dec_gbs / n, "peak": peaks["hbm_gbs"],
-                           "unit": "GB/s", "frac": dec_gbs / n / peaks["hbm_gbs"],
-                           "traffic": ncu_traffic("decode_step"),
-                           "peak_source": f"{peak_src} (copy)"},
-              "clocks": dec_clk,
-              "bf16_state": {"value": d16_gbs, "unit": "GB/s", "ms_per_step": d16_ms,
-                             "sequence_steps_per_s": n * inputs.CONFIGS[3].batch / (d16_ms * 1e-3),
-                             "roofline": {"bound": "hbm", "achieved": d16_gbs / n,
-                                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                          "frac": d16_gbs / n / peaks["hbm_gbs"],
-                                          "traffic": None, "peak_source": f"{peak_src} (copy)"},
-                             "clocks": d16_clk},
-              "multi_token": {"tokens_per_call": 4, "ms_per_call": dm_ms,
-                              "sequence_tokens_per_s": n * inputs.CONFIGS[3].batch * 4 / (dm_ms * 1e-3),
-                              "one_token_steps_ms": 4 * dec_ms,
-                              "state_gbs": n * dm_bytes / (dm_ms * 1e-3) / 1e9}}
+    head = run_prefill(HEADLINE, args.steps, True)
+    value, step_roof = _prefill_line(head, n, peaks)
+    T = head["tokens"]
+    others = {}
+    if not args.headline_only:
+        for idx in SECONDARY:
+            r = run_prefill(idx, max(20, args.steps), False)
+            v, sr = _prefill_line(r, n, peaks)
+            r.update({"value": v, "unit": "tokens/s", "step_roofline": sr})
+            others[r["workload"]] = r
+    head_e2e = head.pop("e2e")
+    e2e = {"value": job_tokens_per_s(n, T, head_e2e["ms_per_step"]), "unit": "tokens/s",
+           "ms_per_step": head_e2e["ms_per_step"], "steps": head_e2e["steps"],
+           "h2d_bytes_per_step": head_e2e["h2d_bytes_per_step"],
+           "d2h_bytes_per_step": head_e2e["d2h_bytes_per_step"],
+           "path": "gdn_chunk_prefill_host (C ABI, pinned host buffers, copies overlapped with "
+                   "the layer segment by segment)"}
 
-    chunk_states = bench_chunk_states(args, w, seed, dev, gdn)
-    block = bench_block(w, seed, dev, gdn)
+    decode = None
+    chunk_states = block = None
+    if not args.headline_only:
+        torch.cuda.nvtx.range_push("decode")
+        dec_ms, dec_bytes, dec_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev,
+                                                  gdn, args.decode_steps)
+        dec_ms = max_over_ranks([dec_ms], dev)[0]
+        dec_gbs = n * dec_bytes / (dec_ms * 1e-3) / 1e9
+        # the serving option of a bf16 recurrent state (same workload, half the state bytes)
+        d16_ms, d16_bytes, d16_clk = bench_decode(inputs.CONFIGS[3], inputs.config_seed(3), dev,
+                                                  gdn, args.decode_steps, torch.bfloat16)
+        d16_ms = max_over_ranks([d16_ms], dev)[0]
+        d16_gbs = n * d16_bytes / (d16_ms * 1e-3) / 1e9
+        dm_ms, dm_bytes, dm_tps = bench_decode_multi(inputs.CONFIGS[3], inputs.config_seed(3),
+                                                     dev, gdn)
+        dm_ms = max_over_ranks([dm_ms], dev)[0]
+        torch.cuda.nvtx.range_pop()
+        decode = {"workload": inputs.CONFIGS[3].name, "value": dec_gbs, "unit": "GB/s",
+                  "ms_per_step": dec_ms, "steps": args.decode_steps,
+                  "roofline": {"bound": "hbm", "achieved": dec_gbs / n, "peak": peaks["hbm_gbs"],
+                               "unit": "GB/s", "frac": dec_gbs / n / peaks["hbm_gbs"],
+                               "traffic": ncu_traffic("decode_step"),
+                               "peak_source": f"{peak_src} (copy)"},
+                  "clocks": dec_clk,
+                  "bf16_state": {"value": d16_gbs, "unit": "GB/s", "ms_per_step": d16_ms,
+                                 "sequence_steps_per_s": n * inputs.CONFIGS[3].batch / (d16_ms * 1e-3),
+                                 "roofline": {"bound": "hbm", "achieved": d16_gbs / n,
+                                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                              "frac": d16_gbs / n / peaks["hbm_gbs"],
+                                              "traffic": None,
+                                              "peak_source": f"{peak_src} (copy)"},
+                                 "clocks": d16_clk},
+                  "multi_token": {"tokens_per_call": 4, "ms_per_call": dm_ms,
+                                  "sequence_tokens_per_s": n * inputs.CONFIGS[3].batch * 4 / (dm_ms * 1e-3),
+                                  "one_token_steps_ms": 4 * dec_ms,
+                                  "state_gbs": n * dm_bytes / (dm_ms * 1e-3) / 1e9,
+                                  "roofline": {"bound": "hbm",
+                                               "achieved": dm_bytes / (dm_ms * 1e-3) / 1e9,
+                                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                               "frac": dm_bytes / (dm_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                               "traffic": None,
+                                               "peak_source": f"{peak_src} (copy)"}}}
+        w1 = inputs.CONFIGS[1]
+        chunk_states = bench_chunk_states(args, w1, inputs.config_seed(1), dev, gdn)
+        block = bench_block(w1, inputs.config_seed(1), dev, gdn)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -577,20 +710,22 @@ def main():
 
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": n, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16",
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; Qwen3-Next GDN layer shapes)",
         "config": {"workload": w.name, "global_batch": n, "seq_len": T,
                    "parallelism": "replicas" if n == 1 else f"replicas x{n}",
-                   "l2": "flushed between timed steps (256 MiB write, untimed)",
-                   "launch": "CUDA graph replay of the whole step",
+                   "l2": "flushed between timed steps (256 MiB write, untimed); inputs 8.7 GB "
+                         "> L2 as well",
+                   "launch": "CUDA graph replay of the whole step; per-kernel times from as many "
+                             "replays of the same step captured with the library's launch trace "
+                             "(event-record nodes around every launch)",
                    "chunk": CHUNK, "heads": [w.num_k_heads, w.num_v_heads], "head_dim": 128},
-        "roofline": roof, "step_roofline": step_roof, "kernels": kern,
-        "e2e": {"value": job_tokens_per_s(n, T, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": len(recs), "eager_ms_per_step": eager_ms,
-        "clocks": clocks, "decode": decode, "chunk_states": chunk_states, "block": block,
-        "cpu_baseline": cpu,
+        "roofline": head["roofline"], "step_roofline": step_roof, "kernels": head["kernels"],
+        "traced_graph_ms_per_step": head["traced_graph_ms_per_step"],
+        "e2e": e2e, "gpu_launches": head["launches_per_step"] * args.steps,
+        "clocks": head["clocks"], "prefill_configs": others, "decode": decode,
+        "chunk_states": chunk_states, "block": block, "cpu_baseline": cpu,
     }
     if rank == 0:
         print(json.dumps(res), flush=True)

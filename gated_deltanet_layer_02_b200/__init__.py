@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
 
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
-    GDN_ERR_WORKSPACE = 0, -1, -2, -3, -4, -5
+    GDN_ERR_WORKSPACE, GDN_ERR_BOUNDS = 0, -1, -2, -3, -4, -5, -6
 GDN_F32, GDN_BF16 = 0, 1
 
 #: every symbol include/gdn.h declares
@@ -32,11 +32,22 @@ EXPORTS = (
     "gdn_chunk_prefill_static_ws", "gdn_trace_span", "gdn_decode_step_bf16_state",
     "gdn_chunk_prefill_states", "gdn_decode_multi", "gdn_block_prefill_workspace_size",
     "gdn_block_prefill", "gdn_chunk_prefill_slots", "gdn_chunk_prefill_host_plan",
-    "gdn_chunk_prefill_host_workspace_size", "gdn_chunk_prefill_host",
+    "gdn_chunk_prefill_host_workspace_size", "gdn_chunk_prefill_host", "gdn_debug_set",
+    "gdn_chunk_prefill_pages",
 )
 
 #: size of the library-owned scratch used by chunk_prefill_static_ws (GDN_STATIC_WORKSPACE_BYTES)
 STATIC_WORKSPACE_BYTES = 64 << 20
+
+
+GDN_FAULT_NONE, GDN_FAULT_SKIP_CHAIN_LOAD = 0, 1
+
+
+class DebugOptions(ctypes.Structure):
+    """gdn_debug_options (see gdn.h): test and debug controls of the calling host thread."""
+    _fields_ = [("wait_limit_us", ctypes.c_uint32), ("segment_chunks", ctypes.c_int32),
+                ("chain_split", ctypes.c_int32), ("fault", ctypes.c_int32),
+                ("fault_chunk", ctypes.c_int32)]
 
 
 class GdnError(RuntimeError):
@@ -63,6 +74,74 @@ class Dims(ctypes.Structure):
 
 _lib = None
 _lock = threading.Lock()
+LIB_CHECKED_PATH = os.path.join(_HERE, "libgdn_checked.so")
+
+
+def _configure(L):
+    """Sets the ctypes signatures of every entry point on a loaded libgdn (or its checked
+    variant) and checks that each declared symbol resolves."""
+    vp, i32, dp = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(Dims)
+    L.gdn_abi_version.restype = ctypes.c_int
+    L.gdn_conv_channels.argtypes = [dp]
+    L.gdn_conv_channels.restype = ctypes.c_int64
+    L.gdn_status_string.argtypes = [ctypes.c_int]
+    L.gdn_status_string.restype = ctypes.c_char_p
+    L.gdn_conv1d_update.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, i32, i32, vp, vp, vp]
+    L.gdn_gated_rmsnorm.argtypes = [ctypes.c_int, vp, vp, vp, ctypes.c_float, i32, i32, vp, vp]
+    L.gdn_chunk_prefill_workspace_size.argtypes = [dp, ctypes.c_int, i32, i32]
+    L.gdn_chunk_prefill_workspace_size.restype = ctypes.c_size_t
+    L.gdn_chunk_prefill.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, i32, i32,
+                                    vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
+    L.gdn_chunk_prefill_states.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                           i32, i32, vp, vp, vp, vp, vp, vp, vp,
+                                           ctypes.c_size_t, vp, vp]
+    L.gdn_chunk_prefill_pages.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, i32,
+                                          i32, vp, vp, vp, vp, vp, i32, vp, vp,
+                                          ctypes.c_size_t, vp, vp]
+    L.gdn_decode_step.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                  i32, vp, vp, vp]
+    L.gdn_decode_step_bf16_state.argtypes = L.gdn_decode_step.argtypes
+    L.gdn_decode_multi.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                   i32, i32, i32, vp, vp, vp, vp]
+    L.gdn_chunk_prefill_slots.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                          i32, i32, vp, i32, vp, vp, vp, vp,
+                                          ctypes.c_size_t, vp, vp]
+    L.gdn_chunk_prefill_host_plan.argtypes = [vp, i32, i32, i32, vp, i32]
+    L.gdn_chunk_prefill_host_plan.restype = ctypes.c_int32
+    L.gdn_chunk_prefill_host_workspace_size.argtypes = [dp, vp, i32, i32, i32]
+    L.gdn_chunk_prefill_host_workspace_size.restype = ctypes.c_size_t
+    L.gdn_chunk_prefill_host.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp,
+                                         vp, vp, vp, i32, vp, ctypes.c_size_t, vp, vp]
+    L.gdn_block_prefill_workspace_size.argtypes = [dp, i32, i32, i32]
+    L.gdn_block_prefill_workspace_size.restype = ctypes.c_size_t
+    L.gdn_block_prefill.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
+                                    i32, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
+    L.gdn_trace_create.argtypes = [ctypes.POINTER(vp)]
+    L.gdn_trace_destroy.argtypes = [vp]
+    L.gdn_trace_attach.argtypes = [vp]
+    L.gdn_trace_reset.argtypes = [vp]
+    L.gdn_trace_count.argtypes = [vp]
+    L.gdn_trace_get.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_char_p),
+                                ctypes.POINTER(ctypes.c_float)]
+    L.gdn_trace_span.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_float),
+                                 ctypes.POINTER(ctypes.c_float)]
+    L.gdn_debug_wait_probe.argtypes = [vp, ctypes.c_uint32, vp]
+    L.gdn_debug_set.argtypes = [ctypes.POINTER(DebugOptions)]
+    L.gdn_chunk_prefill_static_ws.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
+                                              i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    for name in EXPORTS:  # every declared symbol must resolve
+        getattr(L, name)
+    return L
+
+
+def lib_checked():
+    """The bounds-check build (libgdn_checked.so, built with
+    `python -m gated_deltanet_layer_02_b200.build --bounds-check`), loaded beside libgdn.so for
+    tests: the same entry points, kernels compiled with -DGDN_BOUNDS_CHECK."""
+    if not os.path.exists(LIB_CHECKED_PATH):
+        raise RuntimeError(f"{LIB_CHECKED_PATH} is missing: build it with "
+                           "`python -m gated_deltanet_layer_02_b200.build --bounds-check`")
+    return _configure(ctypes.CDLL(LIB_CHECKED_PATH))
 
 
 def lib():
@@ -73,55 +152,7 @@ def lib():
             if not os.path.exists(LIB_PATH):
                 raise RuntimeError(f"{LIB_PATH} is missing: build it with "
                                    "`python -m gated_deltanet_layer_02_b200.build`")
-            L = ctypes.CDLL(LIB_PATH)
-            vp, i32, dp = ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(Dims)
-            L.gdn_abi_version.restype = ctypes.c_int
-            L.gdn_conv_channels.argtypes = [dp]
-            L.gdn_conv_channels.restype = ctypes.c_int64
-            L.gdn_status_string.argtypes = [ctypes.c_int]
-            L.gdn_status_string.restype = ctypes.c_char_p
-            L.gdn_conv1d_update.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, i32, i32, vp, vp, vp]
-            L.gdn_gated_rmsnorm.argtypes = [ctypes.c_int, vp, vp, vp, ctypes.c_float, i32, i32, vp, vp]
-            L.gdn_chunk_prefill_workspace_size.argtypes = [dp, ctypes.c_int, i32, i32]
-            L.gdn_chunk_prefill_workspace_size.restype = ctypes.c_size_t
-            L.gdn_chunk_prefill.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, i32, i32,
-                                            vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
-            L.gdn_chunk_prefill_states.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
-                                                   i32, i32, vp, vp, vp, vp, vp, vp, vp,
-                                                   ctypes.c_size_t, vp, vp]
-            L.gdn_decode_step.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
-                                          vp, vp]
-            L.gdn_decode_step_bf16_state.argtypes = L.gdn_decode_step.argtypes
-            L.gdn_decode_multi.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                           i32, i32, vp, vp, vp]
-            L.gdn_chunk_prefill_slots.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
-                                                  i32, i32, vp, vp, vp, vp, vp, ctypes.c_size_t,
-                                                  vp, vp]
-            L.gdn_chunk_prefill_host_plan.argtypes = [vp, i32, i32, i32, vp, i32]
-            L.gdn_chunk_prefill_host_plan.restype = ctypes.c_int32
-            L.gdn_chunk_prefill_host_workspace_size.argtypes = [dp, vp, i32, i32, i32]
-            L.gdn_chunk_prefill_host_workspace_size.restype = ctypes.c_size_t
-            L.gdn_chunk_prefill_host.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp,
-                                                 vp, vp, vp, i32, vp, ctypes.c_size_t, vp, vp]
-            L.gdn_block_prefill_workspace_size.argtypes = [dp, i32, i32, i32]
-            L.gdn_block_prefill_workspace_size.restype = ctypes.c_size_t
-            L.gdn_block_prefill.argtypes = [dp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32,
-                                            i32, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp]
-            L.gdn_trace_create.argtypes = [ctypes.POINTER(vp)]
-            L.gdn_trace_destroy.argtypes = [vp]
-            L.gdn_trace_attach.argtypes = [vp]
-            L.gdn_trace_reset.argtypes = [vp]
-            L.gdn_trace_count.argtypes = [vp]
-            L.gdn_trace_get.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_char_p),
-                                        ctypes.POINTER(ctypes.c_float)]
-            L.gdn_trace_span.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_float),
-                                         ctypes.POINTER(ctypes.c_float)]
-            L.gdn_debug_wait_probe.argtypes = [vp, ctypes.c_uint32, vp]
-            L.gdn_chunk_prefill_static_ws.argtypes = [dp, ctypes.c_int, vp, vp, vp, vp, vp, vp, vp,
-                                                      i32, i32, vp, vp, vp, vp, vp, vp, vp]
-            for name in EXPORTS:  # every declared symbol must resolve
-                getattr(L, name)
-            _lib = L
+            _lib = _configure(ctypes.CDLL(LIB_PATH))
     return _lib
 
 
@@ -165,6 +196,15 @@ def _need_layer(dims, T, N, x=None, beta=None, g=None, z=None, out=None, conv_w=
                        (SN, "SN", N * Hv * d * d), (conv0, "conv0", N * (K - 1) * Cc),
                        (convN, "convN", N * (K - 1) * Cc)):
         _need(t, name, n)
+
+
+def _pool_rows(S, conv_state, dims):
+    """Rows of a state pool pair: whole [Hv, d, d] states in S that have a conv history row."""
+    per_S = dims.num_v_heads * dims.head_dim ** 2
+    rows = S.numel() // per_S if S is not None else 0
+    if conv_state is not None:
+        rows = min(rows, conv_state.numel() // ((dims.conv_kernel - 1) * dims.channels))
+    return rows
 
 
 def _act_dtype(t):
@@ -228,13 +268,15 @@ def prefill_workspace_size(num_seqs: int, num_tokens: int, dtype=torch.bfloat16,
 
 def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None, SN=None,
                   conv0=None, convN=None, out=None, workspace=None, dev_status=None,
-                  want_state=True, dims: Dims | None = None, chunk_states=None):
+                  want_state=True, dims: Dims | None = None, chunk_states=None,
+                  page_states=None, page_size: int = 128):
     """The whole layer over packed sequences.  Returns (out, SN, convN).
 
     x [T, Cc], beta/g [T, Hv] fp32, z [T, Hv, d] or None, cu_seqlens [N+1] int32 (device),
     S0 [N, Hv, d, d] fp32 or None, conv0 [N, K-1, Cc] or None.  chunk_states [C, Hv, d, d] fp32
     (C = sum of ceil(L_n / 128)) receives the state after every 128-token chunk
-    (gdn_chunk_prefill_states).
+    (gdn_chunk_prefill_states); page_states [P, Hv, d, d] (P = sum of ceil(L_n / page_size))
+    the state after every page of 64 or 128 tokens (gdn_chunk_prefill_pages).
     """
     dims = dims or Dims()
     dt = _act_dtype(x)
@@ -260,7 +302,10 @@ def chunk_prefill(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=N
             _ptr(out, "out", x.dtype))
     tail = (_ptr(workspace, "workspace", torch.uint8), workspace.numel(),
             _ptr(dev_status, "dev_status", torch.int32), _stream())
-    if chunk_states is None:
+    if page_states is not None:
+        _check("gdn_chunk_prefill_pages", lib().gdn_chunk_prefill_pages(
+            *head, int(page_size), _ptr(page_states, "page_states", torch.float32), *tail))
+    elif chunk_states is None:
         _check("gdn_chunk_prefill", lib().gdn_chunk_prefill(*head, *tail))
     else:
         _check("gdn_chunk_prefill_states", lib().gdn_chunk_prefill_states(
@@ -273,7 +318,8 @@ def chunk_prefill_slots(x, beta, g, cu_seqlens, S_pool, slot_idx=None, conv_pool
                         dev_status=None, dims: Dims | None = None):
     """chunk_prefill with the states in pools shared with decode_step: sequence n starts from
     and overwrites S_pool[slot_idx[n]] ([slots, Hv, d, d] fp32) and conv_pool[slot_idx[n]]
-    ([slots, K-1, Cc]).  Slots must be distinct.  Returns out [T, Hv, d]."""
+    ([slots, K-1, Cc]).  Slots must be distinct; a slot outside [0, slots) is skipped on the
+    device and reported in dev_status (GDN_ERR_INVALID_ARG).  Returns out [T, Hv, d]."""
     dims = dims or Dims()
     T = x.shape[0]
     N = cu_seqlens.numel() - 1
@@ -283,15 +329,15 @@ def chunk_prefill_slots(x, beta, g, cu_seqlens, S_pool, slot_idx=None, conv_pool
         workspace = torch.empty(max(prefill_workspace_size(N, T, x.dtype, dims), 256),
                                 dtype=torch.uint8, device=x.device)
     _need_layer(dims, T, N, x, beta, g, z, out, conv_w, norm_w)
-    if slot_idx is None:   # identity slots: rows 0 .. N-1 of the pools
-        _need(S_pool, "S_pool", N * dims.num_v_heads * dims.head_dim ** 2)
-        _need(conv_pool, "conv_pool", N * (dims.conv_kernel - 1) * dims.channels)
+    num_slots = _pool_rows(S_pool, conv_pool, dims)
+    if slot_idx is None and num_slots < N:   # identity slots: rows 0 .. N-1 of the pools
+        raise ValueError(f"the pools hold {num_slots} rows; the call needs {N}")
     _need(slot_idx, "slot_idx", N)
     _check("gdn_chunk_prefill_slots", lib().gdn_chunk_prefill_slots(
         ctypes.byref(dims), _act_dtype(x), _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype),
         _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
         _ptr(norm_w, "norm_w", x.dtype), _ptr(cu_seqlens, "cu_seqlens", torch.int32), N, T,
-        _ptr(slot_idx, "slot_idx", torch.int32), _ptr(S_pool, "S_pool", torch.float32),
+        _ptr(slot_idx, "slot_idx", torch.int32), num_slots, _ptr(S_pool, "S_pool", torch.float32),
         _ptr(conv_pool, "conv_pool", x.dtype), _ptr(out, "out", x.dtype),
         _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
         _ptr(dev_status, "dev_status", torch.int32), _stream()))
@@ -396,9 +442,10 @@ def chunk_prefill_static_ws(x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=
 
 
 def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx=None,
-                out=None, dims: Dims | None = None):
+                out=None, dev_status=None, dims: Dims | None = None):
     """One token per sequence; conv_state and S are updated in place.  Returns out [B, Hv, d].
-    S may be fp32 (gdn_decode_step) or bf16 (gdn_decode_step_bf16_state)."""
+    S may be fp32 (gdn_decode_step) or bf16 (gdn_decode_step_bf16_state).  A slot outside the
+    pools is skipped on the device and reported in dev_status (GDN_ERR_INVALID_ARG)."""
     dims = dims or Dims()
     dt = _act_dtype(x)
     B = x.shape[0]
@@ -406,9 +453,9 @@ def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx
         out = torch.empty((B, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
     bf16_state = S is not None and S.dtype == torch.bfloat16
     _need_layer(dims, B, 0, x, beta, g, z, out, conv_w, norm_w)
-    if slot_idx is None:   # identity slots: rows 0 .. B-1 of the pools
-        _need(S, "S", B * dims.num_v_heads * dims.head_dim ** 2)
-        _need(conv_state, "conv_state", B * (dims.conv_kernel - 1) * dims.channels)
+    num_slots = _pool_rows(S, conv_state, dims)
+    if slot_idx is None and num_slots < B:   # identity slots: rows 0 .. B-1 of the pools
+        raise ValueError(f"the state pools hold {num_slots} rows; the call needs {B}")
     _need(slot_idx, "slot_idx", B)
     name = "gdn_decode_step_bf16_state" if bf16_state else "gdn_decode_step"
     _check(name, getattr(lib(), name)(
@@ -416,12 +463,13 @@ def decode_step(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx
         _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
         _ptr(norm_w, "norm_w", x.dtype), _ptr(conv_state, "conv_state", x.dtype),
         _ptr(S, "S", torch.bfloat16 if bf16_state else torch.float32),
-        _ptr(slot_idx, "slot_idx", torch.int32), B, _ptr(out, "out", x.dtype), _stream()))
+        _ptr(slot_idx, "slot_idx", torch.int32), num_slots, B, _ptr(out, "out", x.dtype),
+        _ptr(dev_status, "dev_status", torch.int32), _stream()))
     return out
 
 
 def decode_multi(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_idx=None,
-                 out=None, snapshots=None, dims: Dims | None = None):
+                 out=None, snapshots=None, dev_status=None, dims: Dims | None = None):
     """k tokens per sequence (x [B, k, Cc]); conv_state and S (fp32) are updated in place.
     Returns out [B, k, Hv, d]; snapshots [B, k, Hv, d, d] fp32 receives the state after each
     token when given."""
@@ -431,17 +479,18 @@ def decode_multi(x, beta, g, conv_state, S, conv_w, z=None, norm_w=None, slot_id
     if out is None:
         out = torch.empty((B, k, dims.num_v_heads, dims.head_dim), dtype=x.dtype, device=x.device)
     _need_layer(dims, B * k, 0, x, beta, g, z, out, conv_w, norm_w)
-    if slot_idx is None:   # identity slots: rows 0 .. B-1 of the pools
-        _need(S, "S", B * dims.num_v_heads * dims.head_dim ** 2)
-        _need(conv_state, "conv_state", B * (dims.conv_kernel - 1) * dims.channels)
+    num_slots = _pool_rows(S, conv_state, dims)
+    if slot_idx is None and num_slots < B:   # identity slots: rows 0 .. B-1 of the pools
+        raise ValueError(f"the state pools hold {num_slots} rows; the call needs {B}")
     _need(slot_idx, "slot_idx", B)
     _need(snapshots, "snapshots", B * k * dims.num_v_heads * dims.head_dim ** 2)
     _check("gdn_decode_multi", lib().gdn_decode_multi(
         ctypes.byref(dims), dt, _ptr(x, "x", x.dtype), _ptr(conv_w, "conv_w", x.dtype, False),
         _ptr(beta, "beta", torch.float32), _ptr(g, "g", torch.float32), _ptr(z, "z", x.dtype),
         _ptr(norm_w, "norm_w", x.dtype), _ptr(conv_state, "conv_state", x.dtype),
-        _ptr(S, "S", torch.float32), _ptr(slot_idx, "slot_idx", torch.int32), B, k,
-        _ptr(out, "out", x.dtype), _ptr(snapshots, "snapshots", torch.float32), _stream()))
+        _ptr(S, "S", torch.float32), _ptr(slot_idx, "slot_idx", torch.int32), num_slots, B, k,
+        _ptr(out, "out", x.dtype), _ptr(snapshots, "snapshots", torch.float32),
+        _ptr(dev_status, "dev_status", torch.int32), _stream()))
     return out
 
 
@@ -482,6 +531,26 @@ def block_prefill(h, w_qkv, w_z, w_ba, a_log, dt_bias, w_out, cu_seqlens, conv_w
         _ptr(y, "y", bf), _ptr(workspace, "workspace", torch.uint8), workspace.numel(),
         _ptr(dev_status, "dev_status", torch.int32), _stream()))
     return y, SN, convN
+
+
+class debug_options:
+    """Context manager around gdn_debug_set: the library calls of this host thread inside the
+    block use the given settings; leaving the block restores the defaults.
+
+        with gdn.debug_options(segment_chunks=2, chain_split=4):
+            gdn.chunk_prefill(...)
+    """
+
+    def __init__(self, wait_limit_us=0, segment_chunks=0, chain_split=0, fault=GDN_FAULT_NONE,
+                 fault_chunk=0):
+        self.opts = DebugOptions(wait_limit_us, segment_chunks, chain_split, fault, fault_chunk)
+
+    def __enter__(self):
+        _check("gdn_debug_set", lib().gdn_debug_set(ctypes.byref(self.opts)))
+        return self
+
+    def __exit__(self, *exc):
+        lib().gdn_debug_set(None)
 
 
 def debug_wait_probe(dev_status, limit_us: int):
@@ -546,4 +615,4 @@ __all__ = ["Dims", "GdnError", "lib", "conv1d_update", "gated_rmsnorm", "chunk_p
            "chunk_prefill_host", "host_plan",
            "chunk_prefill_static_ws", "STATIC_WORKSPACE_BYTES",
            "decode_step", "prefill_workspace_size", "conv_channels", "status_string", "Trace",
-           "debug_wait_probe", "EXPORTS", "LIB_PATH"]
+           "debug_wait_probe", "debug_options", "DebugOptions", "EXPORTS", "LIB_PATH"]

@@ -1,10 +1,12 @@
 """Build libgdn.so in-tree for sm_100a with nvcc (no JIT cache, nothing installed).
 
-    python -m gated_deltanet_layer_02_b200.build [--force]
+    python -m gated_deltanet_layer_02_b200.build [--force] [--bounds-check]
 
 Each .cu under csrc/ is compiled to an object in csrc/_build/ (rebuilt when it or a header is
 newer), then linked into gated_deltanet_layer_02_b200/libgdn.so with the CUDA runtime linked
-statically.
+statically.  ``--bounds-check`` builds the checked variant instead: every source compiled with
+-DGDN_BOUNDS_CHECK into csrc/_build_checked/ and linked into libgdn_checked.so (index checks
+in the kernels that record GDN_ERR_BOUNDS in the caller's status word and skip the access).
 """
 from __future__ import annotations
 
@@ -20,6 +22,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(CSRC, "_build")
 LIB = os.path.join(HERE, "libgdn.so")
+BUILD_CHECKED = os.path.join(CSRC, "_build_checked")
+LIB_CHECKED = os.path.join(HERE, "libgdn_checked.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -45,20 +49,22 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, bounds_check: bool = False) -> str:
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    build_dir, lib_path = (BUILD_CHECKED, LIB_CHECKED) if bounds_check else (BUILD, LIB)
+    flags = FLAGS + (["-DGDN_BOUNDS_CHECK"] if bounds_check else [])
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = _headers()
     jobs = []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         if force or _stale(obj, [src] + headers):
             jobs.append((src, obj))
 
     def compile_one(job):
         src, obj = job
-        cmd = [nvcc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        cmd = [nvcc, *ARCH, *flags, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -70,16 +76,17 @@ def build(force: bool = False, verbose: bool = False) -> str:
         for msg in ex.map(compile_one, jobs):
             if verbose and msg:
                 sys.stderr.write(msg)
-    objs = [os.path.join(BUILD, os.path.basename(s)[:-3] + ".o") for s in sources]
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".{os.getpid()}.tmp"
+    objs = [os.path.join(build_dir, os.path.basename(s)[:-3] + ".o") for s in sources]
+    if force or jobs or _stale(lib_path, objs):
+        tmp = lib_path + f".{os.getpid()}.tmp"
         cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr}")
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                bounds_check="--bounds-check" in sys.argv))

@@ -16,7 +16,7 @@ cudaError_t launch_conv1d(bool bf16, const void* x, void* y, const void* w, cons
                           cudaStream_t s);
 cudaError_t launch_conv_state_out(bool bf16, const void* x, const int32_t* cu, int N, int Cc,
                                   const void* st_in, void* st_out, const int32_t* slot,
-                                  cudaStream_t s);
+                                  int num_slots, int32_t* status, cudaStream_t s);
 cudaError_t launch_gated_rmsnorm(bool bf16, const void* o, const void* z, const void* w, float eps,
                                  int rows, int dim, void* y, cudaStream_t s);
 cudaError_t launch_decode(bool bf16, bool state_bf16, const gdn::DecodeArgs& a, cudaStream_t s);
@@ -44,6 +44,16 @@ namespace gdn_host {
 static thread_local gdn_trace* t_trace = nullptr;
 static thread_local bool t_open = false;
 
+// Records `ev` on `s`.  Inside a stream capture the record becomes an event-record node of the
+// graph (cudaEventRecordExternal), so every replay of the graph records the event again and the
+// launch times can be read after each replay.
+static cudaError_t record_event(cudaEvent_t ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    return cudaEventRecordWithFlags(ev, s, cudaEventRecordExternal);
+  return cudaEventRecord(ev, s);
+}
+
 void trace_begin(const char* name, cudaStream_t s) {
   gdn_trace* tr = t_trace;
   t_open = false;
@@ -59,14 +69,16 @@ void trace_begin(const char* name, cudaStream_t s) {
   }
   TraceRec& r = tr->recs[tr->used];
   r.name = name;
-  if (cudaEventRecord(r.start, s) == cudaSuccess) t_open = true;
+  if (record_event(r.start, s) == cudaSuccess) t_open = true;
 }
+
+bool trace_attached() { return t_trace != nullptr; }
 
 void trace_end(cudaStream_t s) {
   gdn_trace* tr = t_trace;
   if (!tr || !t_open) return;
   t_open = false;
-  if (cudaEventRecord(tr->recs[tr->used].stop, s) == cudaSuccess) tr->used++;
+  if (record_event(tr->recs[tr->used].stop, s) == cudaSuccess) tr->used++;
 }
 }  // namespace gdn_host
 
@@ -116,6 +128,9 @@ bool dtype_ok(gdn_dtype t) { return t == GDN_F32 || t == GDN_BF16; }
 
 namespace gdn_host {
 int check_dims_ext(const gdn_dims* d) { return check_dims(d); }
+
+static thread_local gdn_debug_options t_debug = {};
+const gdn_debug_options& debug_opts() { return t_debug; }
 }  // namespace gdn_host
 
 extern "C" {
@@ -134,6 +149,7 @@ const char* gdn_status_string(int status) {
     case GDN_ERR_CUDA: return "CUDA error";
     case GDN_ERR_TIMEOUT: return "device wait timed out";
     case GDN_ERR_WORKSPACE: return "workspace too small";
+    case GDN_ERR_BOUNDS: return "index check failed (bounds-check build)";
     default: return "unknown status";
   }
 }
@@ -186,13 +202,14 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
                         int32_t num_tokens, const float* S0, float* SN, const void* conv0,
                         void* convN, void* out, void* workspace, size_t workspace_bytes,
                         int32_t* dev_status, float* chunk_states, const int32_t* slot,
-                        void* stream) {
+                        int32_t num_slots, void* stream, bool page64 = false) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return GDN_ERR_UNSUPPORTED;
   if (num_seqs < 0 || num_tokens < 0) return GDN_ERR_INVALID_ARG;
   if (num_seqs == 0 && num_tokens > 0) return GDN_ERR_INVALID_ARG;
   if (num_seqs > 0 && !cu_seqlens) return GDN_ERR_INVALID_ARG;
+  if (slot && num_slots <= 0 && num_seqs > 0) return GDN_ERR_INVALID_ARG;
   if (num_tokens > 0 && (!x || !beta || !g || !out)) return GDN_ERR_INVALID_ARG;
   const void* ptrs[] = {x, conv_w, beta, g, z, norm_w, S0, SN, conv0, convN, out, chunk_states};
   for (const void* p : ptrs)
@@ -220,6 +237,8 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
     a.conv0 = static_cast<const float*>(conv0);
     a.out = static_cast<float*>(out);
     a.slot = slot;
+    a.status = dev_status;
+    a.num_slots = num_slots;
     a.N = num_seqs;
     a.Hk = dims->num_k_heads;
     a.Hv = dims->num_v_heads;
@@ -229,7 +248,7 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
     cudaError_t e = gdn_host::launch_recurrent_f32(a, s);
     if (e == cudaSuccess && convN)
       e = gdn_host::launch_conv_state_out(false, x, cu_seqlens, num_seqs, Cc, conv0, convN, slot,
-                                          s);
+                                          num_slots, dev_status, s);
     return map_cuda(e);
   }
   gdn::PrefillArgs a{};
@@ -245,8 +264,15 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
   a.conv0 = static_cast<const __nv_bfloat16*>(conv0);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.chunk_states = chunk_states;
+  a.page64 = page64 ? 1 : 0;
   a.slot = slot;
   a.status = dev_status;
+  a.num_slots = num_slots;
+  {
+    const gdn_debug_options& dbg = gdn_host::debug_opts();
+    a.wait_ns = dbg.wait_limit_us ? (uint64_t)dbg.wait_limit_us * 1000ull : gdn::kWaitLimitNs;
+    a.fault_chunk = dbg.fault == GDN_FAULT_SKIP_CHAIN_LOAD ? dbg.fault_chunk : -1;
+  }
   a.N = num_seqs;
   a.T = num_tokens;
   a.Hk = dims->num_k_heads;
@@ -261,7 +287,8 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
   a.convN = separate_conv_state ? nullptr : static_cast<__nv_bfloat16*>(convN);
   cudaError_t e = gdn_host::launch_prefill_tc(a, workspace, s);
   if (e == cudaSuccess && separate_conv_state)
-    e = gdn_host::launch_conv_state_out(true, x, cu_seqlens, num_seqs, Cc, conv0, convN, slot, s);
+    e = gdn_host::launch_conv_state_out(true, x, cu_seqlens, num_seqs, Cc, conv0, convN, slot,
+                                        num_slots, dev_status, s);
   return map_cuda(e);
 }
 
@@ -273,7 +300,7 @@ int gdn_chunk_prefill(const gdn_dims* dims, gdn_dtype dtype, const void* x, cons
                       void* stream) {
   return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
                       num_tokens, S0, SN, conv0, convN, out, workspace, workspace_bytes,
-                      dev_status, nullptr, nullptr, stream);
+                      dev_status, nullptr, nullptr, num_seqs, stream);
 }
 
 int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* x,
@@ -286,19 +313,34 @@ int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* 
   if (num_tokens > 0 && !chunk_states) return GDN_ERR_INVALID_ARG;
   return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
                       num_tokens, S0, SN, conv0, convN, out, workspace, workspace_bytes,
-                      dev_status, chunk_states, nullptr, stream);
+                      dev_status, chunk_states, nullptr, num_seqs, stream);
+}
+
+int gdn_chunk_prefill_pages(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                            const void* conv_w, const float* beta, const float* g, const void* z,
+                            const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
+                            int32_t num_tokens, const float* S0, float* SN, const void* conv0,
+                            void* convN, void* out, int32_t page_size, float* page_states,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream) {
+  if (page_size != 64 && page_size != 128) return GDN_ERR_UNSUPPORTED;
+  if (num_tokens > 0 && !page_states) return GDN_ERR_INVALID_ARG;
+  return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
+                      num_tokens, S0, SN, conv0, convN, out, workspace, workspace_bytes,
+                      dev_status, page_states, nullptr, num_seqs, stream, page_size == 64);
 }
 
 int gdn_chunk_prefill_slots(const gdn_dims* dims, gdn_dtype dtype, const void* x,
                             const void* conv_w, const float* beta, const float* g, const void* z,
                             const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
-                            int32_t num_tokens, const int32_t* slot_idx, float* S_pool,
-                            void* conv_pool, void* out, void* workspace, size_t workspace_bytes,
-                            int32_t* dev_status, void* stream) {
+                            int32_t num_tokens, const int32_t* slot_idx, int32_t num_slots,
+                            float* S_pool, void* conv_pool, void* out, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
   if (num_seqs > 0 && !S_pool) return GDN_ERR_INVALID_ARG;
+  if (num_slots < 0 || (!slot_idx && num_slots < num_seqs)) return GDN_ERR_INVALID_ARG;
   return prefill_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, cu_seqlens, num_seqs,
                       num_tokens, S_pool, S_pool, conv_pool, conv_pool, out, workspace,
-                      workspace_bytes, dev_status, nullptr, slot_idx, stream);
+                      workspace_bytes, dev_status, nullptr, slot_idx, num_slots, stream);
 }
 
 }  // extern "C"
@@ -307,11 +349,12 @@ namespace {
 int decode_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
                 const float* beta, const float* g, const void* z, const void* norm_w,
                 void* conv_state, void* S, bool state_bf16, const int32_t* slot_idx,
-                int32_t batch, void* out, void* stream) {
+                int32_t num_slots, int32_t batch, void* out, int32_t* dev_status, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return GDN_ERR_UNSUPPORTED;
   if (batch < 0) return GDN_ERR_INVALID_ARG;
+  if (num_slots < 0 || (!slot_idx && num_slots < batch)) return GDN_ERR_INVALID_ARG;
   if (batch > 0 && (!x || !conv_w || !beta || !g || !conv_state || !S || !out))
     return GDN_ERR_INVALID_ARG;
   const void* ptrs[] = {x, conv_w, beta, g, z, norm_w, conv_state, S, out};
@@ -329,6 +372,8 @@ int decode_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void
   a.S = S;
   a.slot_idx = slot_idx;
   a.out = out;
+  a.status = dev_status;
+  a.num_slots = num_slots;
   a.B = batch;
   a.Hk = dims->num_k_heads;
   a.Hv = dims->num_v_heads;
@@ -344,20 +389,22 @@ extern "C" {
 
 int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
                     const float* beta, const float* g, const void* z, const void* norm_w,
-                    void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
-                    void* out, void* stream) {
+                    void* conv_state, float* S, const int32_t* slot_idx, int32_t num_slots,
+                    int32_t batch, void* out, int32_t* dev_status, void* stream) {
   return decode_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, conv_state, S, false, slot_idx,
-                     batch, out, stream);
+                     num_slots, batch, out, dev_status, stream);
 }
 
 int gdn_decode_multi(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
                      const float* beta, const float* g, const void* z, const void* norm_w,
-                     void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
-                     int32_t tokens, void* out, float* snapshots, void* stream) {
+                     void* conv_state, float* S, const int32_t* slot_idx, int32_t num_slots,
+                     int32_t batch, int32_t tokens, void* out, float* snapshots,
+                     int32_t* dev_status, void* stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (!dtype_ok(dtype)) return GDN_ERR_UNSUPPORTED;
   if (batch < 0 || tokens < 0) return GDN_ERR_INVALID_ARG;
+  if (num_slots < 0 || (!slot_idx && num_slots < batch)) return GDN_ERR_INVALID_ARG;
   if (tokens > 8) return GDN_ERR_UNSUPPORTED;
   if (batch > 0 && tokens > 0 && (!x || !conv_w || !beta || !g || !conv_state || !S || !out))
     return GDN_ERR_INVALID_ARG;
@@ -376,6 +423,8 @@ int gdn_decode_multi(const gdn_dims* dims, gdn_dtype dtype, const void* x, const
   a.S = S;
   a.slot_idx = slot_idx;
   a.out = out;
+  a.status = dev_status;
+  a.num_slots = num_slots;
   a.B = batch;
   a.Hk = dims->num_k_heads;
   a.Hv = dims->num_v_heads;
@@ -389,9 +438,10 @@ int gdn_decode_multi(const gdn_dims* dims, gdn_dtype dtype, const void* x, const
 int gdn_decode_step_bf16_state(const gdn_dims* dims, gdn_dtype dtype, const void* x,
                                const void* conv_w, const float* beta, const float* g,
                                const void* z, const void* norm_w, void* conv_state, void* S,
-                               const int32_t* slot_idx, int32_t batch, void* out, void* stream) {
+                               const int32_t* slot_idx, int32_t num_slots, int32_t batch,
+                               void* out, int32_t* dev_status, void* stream) {
   return decode_impl(dims, dtype, x, conv_w, beta, g, z, norm_w, conv_state, S, true, slot_idx,
-                     batch, out, stream);
+                     num_slots, batch, out, dev_status, stream);
 }
 
 int gdn_trace_create(gdn_trace** out) {
@@ -444,6 +494,21 @@ int gdn_trace_span(gdn_trace* trace, int32_t i, float* start_ms, float* end_ms) 
   if (cudaEventElapsedTime(start_ms, r0.start, r.start) != cudaSuccess ||
       cudaEventElapsedTime(end_ms, r0.start, r.stop) != cudaSuccess)
     return GDN_ERR_CUDA;
+  return GDN_OK;
+}
+
+int gdn_debug_set(const gdn_debug_options* opts) {
+  if (!opts) {
+    gdn_host::t_debug = gdn_debug_options{};
+    return GDN_OK;
+  }
+  const bool split_ok = opts->chain_split == 0 || opts->chain_split == 1 ||
+                        opts->chain_split == 2 || opts->chain_split == 4;
+  if (opts->wait_limit_us > 10000000u || opts->segment_chunks < 0 || !split_ok ||
+      (opts->fault != GDN_FAULT_NONE && opts->fault != GDN_FAULT_SKIP_CHAIN_LOAD) ||
+      opts->fault_chunk < 0)
+    return GDN_ERR_INVALID_ARG;
+  gdn_host::t_debug = *opts;
   return GDN_OK;
 }
 

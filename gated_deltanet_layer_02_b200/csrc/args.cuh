@@ -6,8 +6,12 @@
 namespace gdn {
 
 // Row of a state pool that holds the states of sequence n: slot[n], or n without a slot map.
-__device__ __forceinline__ int state_row(const int32_t* slot, int n) {
-  return slot ? __ldg(slot + n) : n;
+// A slot outside [0, num_slots) gives -1: the caller then reads that sequence's initial states
+// as zero, writes none of its states and reports GDN_ERR_INVALID_ARG.
+__device__ __forceinline__ int state_row(const int32_t* slot, int n, int num_slots) {
+  if (!slot) return n;
+  const int r = __ldg(slot + n);
+  return (r >= 0 && r < num_slots) ? r : -1;
 }
 
 struct DecodeArgs {
@@ -21,6 +25,8 @@ struct DecodeArgs {
   void* S;  // fp32 or bf16 (see the decode kernel's state type)
   const int32_t* slot_idx;
   void* out;
+  int32_t* status;  // device status word (first error wins), or NULL
+  int num_slots;    // rows of the state pools (slot_idx entries must lie in [0, num_slots))
   int B, Hk, Hv;
   float q_scale, l2_eps, norm_eps;
 };
@@ -38,6 +44,8 @@ struct RecArgs {
   const float* conv0;
   float* out;
   const int32_t* slot;  // [N] state-pool row of each sequence (S0, SN, conv0), or NULL (= n)
+  int32_t* status;
+  int num_slots;
   int N, Hk, Hv;
   float q_scale, l2_eps, norm_eps;
 };
@@ -49,14 +57,13 @@ struct ChunkInfo {
 struct Workspace {
   ChunkInfo* chunks;     // [NCmax]
   int32_t* seq_first;    // [N+1] first chunk of each sequence (prefix sum), [N] = total
+  int32_t* page_first;   // [N+1] first 64-token page of each sequence (prefix sum)
   __nv_bfloat16* Qw;     // [NCmax][Hk][128][128]
   __nv_bfloat16* Kw;     // [NCmax][Hk][128][128]
   __nv_bfloat16* Ww;     // [NCmax][Hv][128][128]
   __nv_bfloat16* Uw;     // [NCmax][Hv][128][128]  U~ from prep, overwritten with U by chain
   __nv_bfloat16* Sw;     // [NCmax][Hv][128 (d_k)][128 (d_v)]  S^T entering each chunk
   float* Gw;             // [NCmax][Hv][128]  cumulative log decay inside the chunk
-  int* ready;            // [NCmax][Hv]  prep published (chunk, value head); zeroed per call
-  int* counter;          // next prep unit of the persistent workers; zeroed per call
 };
 
 struct PrefillArgs {
@@ -73,9 +80,16 @@ struct PrefillArgs {
   __nv_bfloat16* convN;  // written by the q/k/v kernel (and the chunk table for empty sequences)
                          // when set; NULL when the caller wants none or it aliases conv0
   __nv_bfloat16* out;
-  float* chunk_states;  // [chunks][Hv][d_v][d_k] fp32: state after each chunk, or NULL
+  float* chunk_states;  // [entries][Hv][d_v][d_k] fp32: state after each chunk (or each
+                        // 64-token page with page64), or NULL
+  int page64;           // states every 64 tokens instead of every chunk
   const int32_t* slot;  // [N] state-pool row of each sequence (S0, SN, conv0, convN), or NULL
   int32_t* status;
+  uint64_t wait_ns;     // bound of every device wait (ns); a wait that runs out reports
+                        // GDN_ERR_TIMEOUT
+  int fault_chunk;      // debug fault injection: the first chain CTA skips the W load of this
+                        // chunk (-1: none)
+  int num_slots;        // rows of the state pools when `slot` is set
   int N, T, Hk, Hv, nsplit;
   float q_scale, l2_eps, norm_eps;
   Workspace ws;

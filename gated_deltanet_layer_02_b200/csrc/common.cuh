@@ -75,6 +75,19 @@ __device__ __forceinline__ void report_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Index checks of the bounds-check build (-DGDN_BOUNDS_CHECK, libgdn_checked.so): a failed
+// check records GDN_ERR_BOUNDS in the caller's status word and the guarded access is skipped.
+// In the normal build GDN_IN_BOUNDS is the constant true and costs nothing.
+__device__ __forceinline__ bool bounds_ok(bool cond, int32_t* status) {
+  if (!cond) report_status(status, GDN_ERR_BOUNDS);
+  return cond;
+}
+#ifdef GDN_BOUNDS_CHECK
+#define GDN_IN_BOUNDS(cond, status) (::gdn::bounds_ok((cond), (status)))
+#else
+#define GDN_IN_BOUNDS(cond, status) (true)
+#endif
+
 }  // namespace gdn
 
 // ---------------------------------------------------------------- host-side launch helpers
@@ -82,4 +95,9 @@ namespace gdn_host {
 // Brackets a launch with trace events when a trace is attached to this host thread.
 void trace_begin(const char* name, cudaStream_t s);
 void trace_end(cudaStream_t s);
+// True while a trace is attached to this host thread (its launches go without programmatic
+// dependent launch, so that each kernel's events bracket that kernel alone).
+bool trace_attached();
+// Debug and test controls set with gdn_debug_set for the calling host thread (defaults: zeros).
+const gdn_debug_options& debug_opts();
 }  // namespace gdn_host

@@ -84,12 +84,19 @@ __global__ void __launch_bounds__(128) conv_state_out_kernel(const T* __restrict
                                                              const int32_t* __restrict__ cu, int N,
                                                              int Cc, const T* state_in,
                                                              T* state_out,
-                                                             const int32_t* __restrict__ slot) {
+                                                             const int32_t* __restrict__ slot,
+                                                             int num_slots, int32_t* status) {
   const int c = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   const int n = blockIdx.y;
   if (c >= Cc || n >= N) return;
   const int s = __ldg(cu + n), L = __ldg(cu + n + 1) - s;
-  const size_t row = (size_t)state_row(slot, n) * 3;
+  if (!GDN_IN_BOUNDS(s >= 0 && L >= 0, status)) return;
+  const int srow = state_row(slot, n, num_slots);
+  if (srow < 0) {  // slot out of range: no access to the pool
+    if (c == 0) report_status(status, GDN_ERR_INVALID_ARG);
+    return;
+  }
+  const size_t row = (size_t)srow * 3;
   float r[3][8];
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
@@ -130,7 +137,8 @@ static cudaError_t conv1d_impl(const void* x, void* y, const void* w, const int3
     trace_begin("conv_state_out", s);
     gdn::conv_state_out_kernel<T><<<grid, 128, 0, s>>>(static_cast<const T*>(x), cu, N, Cc,
                                                        static_cast<const T*>(st_in),
-                                                       static_cast<T*>(st_out), nullptr);
+                                                       static_cast<T*>(st_out), nullptr, N,
+                                                       nullptr);
     trace_end(s);
     return cudaGetLastError();
   }
@@ -146,18 +154,19 @@ cudaError_t launch_conv1d(bool bf16, const void* x, void* y, const void* w, cons
 
 cudaError_t launch_conv_state_out(bool bf16, const void* x, const int32_t* cu, int N, int Cc,
                                   const void* st_in, void* st_out, const int32_t* slot,
-                                  cudaStream_t s) {
+                                  int num_slots, int32_t* status, cudaStream_t s) {
   if (!st_out || N == 0) return cudaSuccess;
   dim3 grid((Cc / 8 + 127) / 128, N);
   trace_begin("conv_state_out", s);
   if (bf16)
     gdn::conv_state_out_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), cu, N, Cc,
-        static_cast<const __nv_bfloat16*>(st_in), static_cast<__nv_bfloat16*>(st_out), slot);
+        static_cast<const __nv_bfloat16*>(st_in), static_cast<__nv_bfloat16*>(st_out), slot, num_slots, status);
   else
     gdn::conv_state_out_kernel<float><<<grid, 128, 0, s>>>(static_cast<const float*>(x), cu, N,
                                                            Cc, static_cast<const float*>(st_in),
-                                                           static_cast<float*>(st_out), slot);
+                                                           static_cast<float*>(st_out), slot, num_slots,
+                                                           status);
   trace_end(s);
   return cudaGetLastError();
 }

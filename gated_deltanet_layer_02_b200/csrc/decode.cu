@@ -69,8 +69,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
   const int hk = blockIdx.x % a.Hk;
   const int R = a.Hv / a.Hk;
   const int Cc = (2 * a.Hk + a.Hv) * d;
-  const int slot = a.slot_idx ? __ldg(a.slot_idx + b) : b;
+  const int slot = state_row(a.slot_idx, b, a.num_slots);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (slot < 0) {  // slot out of range: the sequence is skipped, its outputs are not written
+    if (tid == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
+    return;
+  }
 
   __shared__ float y_s[(2 + kMaxR) * d];  // q | k | v_0..v_{R-1} after conv
   __shared__ float o_s[kMaxR * d];
@@ -223,8 +227,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_multi_kernel(DecodeArgs
   const int hk = blockIdx.x % a.Hk;
   const int R = a.Hv / a.Hk;
   const int Cc = (2 * a.Hk + a.Hv) * d;
-  const int slot = a.slot_idx ? __ldg(a.slot_idx + b) : b;
+  const int slot = state_row(a.slot_idx, b, a.num_slots);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (slot < 0) {  // slot out of range: the sequence is skipped, its outputs are not written
+    if (tid == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
+    return;
+  }
   extern __shared__ float dsm[];
   float* y_s = dsm;                          // [k][(2 + R) d]: q | k | v_0..v_{R-1}
   float* o_s = y_s + k * (2 + R) * d;        // [k][R d]

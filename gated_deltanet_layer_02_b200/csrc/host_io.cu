@@ -221,9 +221,17 @@ int gdn_chunk_prefill_host(const gdn_dims* dims, const void* x, const void* conv
   cudaError_t e = io_streams(2 * segs.size() + 2, &io);
   if (e != cudaSuccess) return GDN_ERR_CUDA;
   cudaEvent_t ev_start = io->ev[0], ev_end = io->ev[1];
+  // After a failure with copies already queued, `stream` still joins both copy streams, so that
+  // work the caller queues on it afterwards (freeing or reusing the host buffers) waits for
+  // every copy in flight (best effort: a failing runtime may refuse these calls as well).
+  auto fail = [&](int code) {
+    if (cudaEventRecord(ev_start, io->h2d) == cudaSuccess) cudaStreamWaitEvent(s, ev_start, 0);
+    if (cudaEventRecord(ev_end, io->d2h) == cudaSuccess) cudaStreamWaitEvent(s, ev_end, 0);
+    return code;
+  };
 #define GDN_TRY(call)                          \
   do {                                         \
-    if ((e = (call)) != cudaSuccess) return GDN_ERR_CUDA; \
+    if ((e = (call)) != cudaSuccess) return fail(GDN_ERR_CUDA); \
   } while (0)
   // copies start after the caller's earlier work on `stream` (it may still use this workspace)
   GDN_TRY(cudaEventRecord(ev_start, s));
@@ -261,7 +269,7 @@ int gdn_chunk_prefill_host(const gdn_dims* dims, const void* x, const void* conv
                            sg.ntok, dS + sg.n0 * sstride, dS + sg.n0 * sstride,
                            dconv + sg.n0 * cstride, dconv + sg.n0 * cstride, dout + t0 * Hv * dh,
                            w + l.layer, l.layer_bytes, dev_status, s);
-    if (rc != GDN_OK) return rc;
+    if (rc != GDN_OK) return fail(rc);
     GDN_TRY(cudaEventRecord(ev_done, s));
     GDN_TRY(cudaStreamWaitEvent(io->d2h, ev_done, 0));
     GDN_TRY(cudaMemcpyAsync(hout + t0 * Hv * dh, dout + t0 * Hv * dh, nt * Hv * dh * 2,

@@ -24,14 +24,16 @@ __global__ void __launch_bounds__(256) recurrent_f32_kernel(RecArgs a) {
   __shared__ float red_q[4], red_k[4], red_o[8];
 
   const int s = __ldg(a.cu + n), e = __ldg(a.cu + n + 1);
+  const int srow = state_row(a.slot, n, a.num_slots);  // -1: slot out of range, no state access
+  if (srow < 0 && tid == 0 && h == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
   // conv history (threads < 128): rows t-3, t-2, t-1 of channel tid of q, k, v
   float hq[3] = {0, 0, 0}, hkk[3] = {0, 0, 0}, hv[3] = {0, 0, 0};
   float wq[4], wk[4], wv[4];
   if (tid < d) {
-    if (a.conv0) {
+    if (a.conv0 && srow >= 0) {
 #pragma unroll
       for (int j = 0; j < 3; ++j) {
-        const float* row = a.conv0 + ((size_t)state_row(a.slot, n) * 3 + j) * Cc;
+        const float* row = a.conv0 + ((size_t)srow * 3 + j) * Cc;
         hq[j] = row[cq + tid];
         hkk[j] = row[ck + tid];
         hv[j] = row[cv + tid];
@@ -48,11 +50,11 @@ __global__ void __launch_bounds__(256) recurrent_f32_kernel(RecArgs a) {
   }
   // state rows of this warp
   float st[kRows][4];
-  const size_t sbase = ((size_t)state_row(a.slot, n) * a.Hv + h) * d * d;
+  const size_t sbase = ((size_t)(srow < 0 ? 0 : srow) * a.Hv + h) * d * d;
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
     const int v = warp * kRows + r;
-    if (a.S0) {
+    if (a.S0 && srow >= 0) {
       float4 p = *reinterpret_cast<const float4*>(a.S0 + sbase + (size_t)v * d + 4 * lane);
       st[r][0] = p.x; st[r][1] = p.y; st[r][2] = p.z; st[r][3] = p.w;
     } else {
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(256) recurrent_f32_kernel(RecArgs a) {
       a.out[((size_t)t * a.Hv + h) * d + tid] = o;
     }
   }
-  if (a.SN) {
+  if (a.SN && srow >= 0) {
 #pragma unroll
     for (int r = 0; r < kRows; ++r) {
       const int v = warp * kRows + r;

@@ -40,51 +40,77 @@ constexpr uint32_t kTile = 16384;  // one [128][64] bf16 row tile
 
 
 // ------------------------------------------------------------------------------ schedule
-__global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, Workspace ws,
-                                      int nready, const __nv_bfloat16* conv0,
-                                      __nv_bfloat16* convN, const int32_t* slot, int Cc) {
-  // publication flags and work counter of the persistent prep + chain kernel
-  for (int k = threadIdx.x; k < nready; k += blockDim.x) ws.ready[k] = 0;
-  if (threadIdx.x == 0 && nready > 0) *ws.counter = 0;
-  // single CTA, sequential prefix over sequences in blocks of blockDim
-  __shared__ int carry;
-  __shared__ int part[1024];
-  if (threadIdx.x == 0) carry = 0;
+__global__ void chunk_schedule_kernel(const int32_t* __restrict__ cu, int N, int T,
+                                      Workspace ws, const __nv_bfloat16* conv0,
+                                      __nv_bfloat16* convN, const int32_t* slot, int num_slots,
+                                      int Cc, int32_t* status) {
+  // single CTA: prefix sums over sequences (in blocks of blockDim) of their 128-token chunks
+  // and of their 64-token pages, then the chunk entries written in parallel
+  __shared__ int carry, carry_p;
+  __shared__ int part[1024], part_p[1024];
+  if (threadIdx.x == 0) carry = carry_p = 0;
   __syncthreads();
   for (int base = 0; base < N; base += blockDim.x) {
     const int n = base + threadIdx.x;
-    int cnt = 0;
-    if (n < N) cnt = (cu[n + 1] - cu[n] + kC - 1) / kC;
+    int cnt = 0, pages = 0;
+    // bounds-check build: a sequence whose cu_seqlens entries are out of order or past T gets
+    // no chunks (and GDN_ERR_BOUNDS)
+    if (n < N && GDN_IN_BOUNDS(cu[n] >= 0 && cu[n + 1] >= cu[n] && cu[n + 1] <= T, status)) {
+      cnt = (cu[n + 1] - cu[n] + kC - 1) / kC;
+      pages = (cu[n + 1] - cu[n] + 63) / 64;
+    }
     part[threadIdx.x] = cnt;
+    part_p[threadIdx.x] = pages;
     __syncthreads();
-    for (int off = 1; off < (int)blockDim.x; off <<= 1) {  // inclusive scan
-      int v = threadIdx.x >= (unsigned)off ? part[threadIdx.x - off] : 0;
+    for (int off = 1; off < (int)blockDim.x; off <<= 1) {  // inclusive scans
+      const bool in = threadIdx.x >= (unsigned)off;
+      const int v = in ? part[threadIdx.x - off] : 0, vp = in ? part_p[threadIdx.x - off] : 0;
       __syncthreads();
       part[threadIdx.x] += v;
+      part_p[threadIdx.x] += vp;
       __syncthreads();
     }
-    const int first = carry + part[threadIdx.x] - cnt;
     if (n < N) {
-      ws.seq_first[n] = first;
-      for (int ci = 0; ci < cnt; ++ci) {
-        ChunkInfo info;
-        info.n = n;
-        info.t0 = cu[n] + ci * kC;
-        info.L = min(kC, cu[n + 1] - info.t0);
-        info.pad = ci;
-        ws.chunks[first + ci] = info;
-      }
+      ws.seq_first[n] = carry + part[threadIdx.x] - cnt;
+      ws.page_first[n] = carry_p + part_p[threadIdx.x] - pages;
     }
     __syncthreads();
-    if (threadIdx.x == blockDim.x - 1) carry += part[threadIdx.x];
+    if (threadIdx.x == blockDim.x - 1) {
+      carry += part[threadIdx.x];
+      carry_p += part_p[threadIdx.x];
+    }
     __syncthreads();
   }
-  if (threadIdx.x == 0) ws.seq_first[N] = carry;
+  if (threadIdx.x == 0) {
+    ws.seq_first[N] = carry;
+    ws.page_first[N] = carry_p;
+  }
+  __syncthreads();  // seq_first (global, written by this CTA) is visible to all its threads
+  // chunk entries: chunk k belongs to the last sequence n with seq_first[n] <= k
+  const int total = carry;
+  for (int k = threadIdx.x; k < total; k += blockDim.x) {
+    int lo = 0, hi = N;  // seq_first[lo] <= k < seq_first[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (ws.seq_first[mid] <= k) lo = mid; else hi = mid;
+    }
+    ChunkInfo info;
+    info.n = lo;
+    info.t0 = cu[lo] + (k - ws.seq_first[lo]) * kC;
+    info.L = min(kC, cu[lo + 1] - info.t0);
+    info.pad = k - ws.seq_first[lo];
+    ws.chunks[k] = info;
+  }
   // final conv history of empty sequences (the q/k/v kernel writes the others): the initial one
   if (convN) {
     for (int n = 0; n < N; ++n) {
       if (cu[n + 1] != cu[n]) continue;
-      const size_t row = (size_t)state_row(slot, n) * 3 * Cc;
+      const int srow = state_row(slot, n, num_slots);
+      if (srow < 0) {
+        if (threadIdx.x == 0) report_status(status, GDN_ERR_INVALID_ARG);
+        continue;
+      }
+      const size_t row = (size_t)srow * 3 * Cc;
       for (int k = threadIdx.x; k < 3 * Cc; k += blockDim.x)
         convN[row + k] = conv0 ? conv0[row + k] : __float2bfloat16(0.f);
     }
@@ -135,6 +161,9 @@ __global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a,
   pdl_wait();  // the chunk table, and the end of every reader of the previous call's tiles
   if (c >= a.ws.seq_first[a.N]) return;
   const ChunkInfo ci = a.ws.chunks[c];
+  if (!GDN_IN_BOUNDS(ci.n >= 0 && ci.n < a.N && ci.t0 >= 0 && ci.L > 0 && ci.L <= kC &&
+                         ci.t0 + ci.L <= a.T, a.status))
+    return;
   const int tid = threadIdx.x, vec = tid & 15, run = tid >> 4;
   const int Hk = a.Hk, Hv = a.Hv;
   const int Cc = (2 * Hk + Hv) * kD;
@@ -170,30 +199,32 @@ __global__ void __launch_bounds__(128, 5) gdn_qkv_kernel(PrefillArgs a,
   uint8_t* box = sm + (vec >> 3) * kXBox;
   const uint32_t chunk = vec & 7;
   auto row_ptr = [&](int r) { return reinterpret_cast<uint4*>(box + sw128_off(r, chunk)); };
-  const bool ok = mbar_wait(bar, 0);
+  const bool ok = mbar_wait(bar, 0, a.wait_ns);
   pdl_trigger();
   if (!ok) {
     if (tid == 0) report_status(a.status, GDN_ERR_TIMEOUT);
     return;
   }
+  // state-pool row of the sequence (-1: its slot is out of range, no pool access)
+  const int srow = state_row(a.slot, ci.n, a.num_slots);
+  if (srow < 0 && tid == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
   // first chunk of a sequence: the 3 rows before it come from the conv state (or are zero)
   if (ci.t0 == seq_start && run == 0) {
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (a.conv0)
-        v = *reinterpret_cast<const uint4*>(
-            a.conv0 + ((size_t)state_row(a.slot, ci.n) * 3 + j) * Cc + ch);
+      if (a.conv0 && srow >= 0)
+        v = *reinterpret_cast<const uint4*>(a.conv0 + ((size_t)srow * 3 + j) * Cc + ch);
       *row_ptr(j) = v;
     }
   }
   __syncthreads();
   // last chunk of its sequence: the final conv history is the box's rows L .. L+2 (the three
   // inputs before the sequence end, conv state rows included when L < 3)
-  if (a.convN && run == 0 && ci.t0 + ci.L == __ldg(a.cu + ci.n + 1)) {
+  if (a.convN && srow >= 0 && run == 0 && ci.t0 + ci.L == __ldg(a.cu + ci.n + 1)) {
 #pragma unroll
     for (int j = 0; j < 3; ++j)
-      *reinterpret_cast<uint4*>(a.convN + ((size_t)state_row(a.slot, ci.n) * 3 + j) * Cc + ch) =
+      *reinterpret_cast<uint4*>(a.convN + ((size_t)srow * 3 + j) * Cc + ch) =
           *row_ptr(ci.L + j);
   }
   const int i0 = run * 16;
@@ -320,13 +351,11 @@ struct PrepCtl {
 // One (chunk c, value head h) unit of prep on a CTA whose barriers are initialised and whose 256
 // TMEM columns are allocated.  `par` is the parity of this unit on bar_k, bar_v and bar_w (one
 // completion each per unit; bar completes six times, so its parity starts at 0 every unit).
-// With `ready` set, W, U~ and G are published for the chain: once the TMA stores have completed,
-// thread 0 sets ready[c * Hv + h] with release semantics.  Returns false after a wait ran out
-// (the status word is set; the CTA must not start another unit).
+// Returns false after a wait ran out (the status word is set).
 __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMap& mapK,
                                           const CUtensorMap& mapV, const CUtensorMap& mapW,
-                                          int c, int h, uint8_t* sm, uint32_t tmem, uint32_t par,
-                                          int* ready) {
+                                          int c, int h, uint8_t* sm, uint32_t tmem,
+                                          uint32_t par) {
   const PrepCtl ctl(sm);
   float* G_s = ctl.G_s;
   float* B_s = ctl.B_s;
@@ -337,6 +366,8 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
   uint64_t* bar = ctl.bar;
   uint64_t* bar_w = ctl.bar_w;
   const ChunkInfo ci = a.ws.chunks[c];
+  if (!GDN_IN_BOUNDS(ci.t0 >= 0 && ci.L > 0 && ci.L <= kC && ci.t0 + ci.L <= a.T, a.status))
+    return false;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int quarter = warp & 3, wg = warp >> 2;
   const int Hv = a.Hv;
@@ -386,7 +417,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
   bool ok = true;
   // ---------------- gram K K^T
   if (tid == 0) {
-    ok = mbar_wait(bar_k, par);
+    ok = mbar_wait(bar_k, par, a.wait_ns);
     tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -397,7 +428,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
     }
   }
   if (__syncthreads_or(!ok)) goto done;
-  ok = mbar_wait(bar, phase);
+  ok = mbar_wait(bar, phase, a.wait_ns);
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
@@ -535,7 +566,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
                   t > 0);
     mma_commit(bar);
   }
-  ok = mbar_wait(bar, phase);
+  ok = mbar_wait(bar, phase, a.wait_ns);
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
@@ -565,7 +596,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
                t > 0);
     mma_commit(bar);
   }
-  ok = mbar_wait(bar, phase);
+  ok = mbar_wait(bar, phase, a.wait_ns);
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
@@ -594,7 +625,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
                idesc_bf16(128, 64, false, true), kk > 0);
     mma_commit(bar);
   }
-  ok = mbar_wait(bar, phase);
+  ok = mbar_wait(bar, phase, a.wait_ns);
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
@@ -623,7 +654,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
                idesc_bf16(128, 64, false, true), kk > 0);
     mma_commit(bar);
   }
-  ok = mbar_wait(bar, phase);
+  ok = mbar_wait(bar, phase, a.wait_ns);
   phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
@@ -680,7 +711,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
       mma_bf16(tmem + kColW, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sK, kk, kTile), id, kk > 0);
     mma_commit(bar_w);
     pdl_trigger();
-    ok = mbar_wait(bar_v, par);
+    ok = mbar_wait(bar_v, par, a.wait_ns);
     tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -688,7 +719,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
         mma_bf16(tmem + kColU, desc_kmajor(sTB, kk, kTile), desc_mnmajor(sV, kk, kTile), id, kk > 0);
       mma_commit(bar);
     } else {
-      mbar_wait(bar_w, par);  // let the W products finish before the CTA gives up its TMEM
+      mbar_wait(bar_w, par, a.wait_ns);  // let the W products finish before the CTA gives up its TMEM
     }
   }
   if (__syncthreads_or(!ok)) goto done;
@@ -697,7 +728,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
     const int i = quarter * 32 + lane, half = wg;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
-      ok = mbar_wait(m == 0 ? bar_w : bar, m == 0 ? par : phase);
+      ok = mbar_wait(m == 0 ? bar_w : bar, m == 0 ? par : phase, a.wait_ns);
       if (__syncthreads_or(!ok)) goto done;
       tc_fence_after();
       uint8_t* tile = sm + (m == 0 ? kPrepKs : kPrepR2);
@@ -720,16 +751,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
         bulk_commit();
       }
     }
-    if (tid == 0) {
-      if (ready) {
-        bulk_wait_all();             // W and U~ are in global memory
-        fence_proxy_async_global();  // ... for the TMA loads of the chain as well
-        __threadfence();
-        st_release_gpu(ready + c * Hv + h, 1);
-      } else {
-        bulk_wait_reads();  // the writes complete before the kernel is seen to end
-      }
-    }
+    if (tid == 0) bulk_wait_reads();  // the writes complete before the kernel is seen to end
   }
 done:
   // every exit reaches this point on all threads (each early exit follows a block-wide vote)
@@ -760,7 +782,7 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *ctl.tslot;
-  prep_unit(a, mapK, mapV, mapW, c, h, sm, tmem, 0, nullptr);
+  prep_unit(a, mapK, mapV, mapW, c, h, sm, tmem, 0);
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x < 32) tmem_dealloc(tmem, 256);
@@ -773,7 +795,9 @@ __global__ void __launch_bounds__(256, 2) gdn_prep_kernel(PrefillArgs a,
 // when the sequence ends there, else to carry_out.  Shared memory: W tile(s), one K tile and one
 // bf16 operand tile that holds S_b^T for X and then U^ for the state update (X has consumed S_b
 // by the time U^ is written).  It stays near 100 KB so that a prep or out CTA fits beside it.
-template <int DV, int WS = (DV > 64 ? 1 : 2)>
+// With MID (64-token pages), a second operand tile holds the first half of the chunk's U^ for
+// the state in the middle of the chunk, and a third TMEM region accumulates it.
+template <int DV, bool MID = false, int WS = (DV > 64 ? 1 : 2)>
 struct ChainCfg {
   static_assert(DV == 32 || DV == 64 || DV == 128, "d_v block");
   static_assert(WS == 1 || WS == 2, "W stages");
@@ -783,18 +807,18 @@ struct ChainCfg {
   static constexpr uint32_t kWStages = WS;                      // W tiles in flight
   static constexpr uint32_t kK = kWStages * 2 * kTile;          // K tile pair
   static constexpr uint32_t kOp = kK + 2 * kTile;               // S_b^T, then U^
-  static constexpr uint32_t kEnd = kOp + kOpTiles * kTile;
+  static constexpr uint32_t kOpMid = kOp + kOpTiles * kTile;    // first-half U^ (MID)
+  static constexpr uint32_t kEnd = kOpMid + (MID ? kOpTiles * kTile : 0);
   static constexpr uint32_t kSmem = kEnd + 1024 + 256;
-  static constexpr uint32_t kTmemCols = 2 * DV;                 // S^T | X
+  static constexpr uint32_t kTmemCols = MID ? (DV == 32 ? 128 : DV == 64 ? 256 : 512)
+                                            : 2 * DV;           // S^T | X (| S_mid^T)
 };
 
-// The chain of CTA `bid` = (sequence, value head, d_v block).  With `ready` set (persistent
-// prep + chain kernel), thread 0 waits for prep to publish each chunk before loading it.
-template <int DV, int WS>
+// The chain of CTA `bid` = (sequence, value head, d_v block).
+template <int DV, bool MID>
 __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorMap& mapW,
-                                           const CUtensorMap& mapK, int bid, uint8_t* sm,
-                                           const int* ready) {
-  using Cfg = ChainCfg<DV, WS>;
+                                           const CUtensorMap& mapK, int bid, uint8_t* sm) {
+  using Cfg = ChainCfg<DV, MID>;
   // the chain's own threads (the first Cfg::kThreads of the block) synchronise on barrier 1
 #define CSYNC() bar_sync_n(1, Cfg::kThreads)
 #define CSYNC_OR(x) bar_or_n(1, Cfg::kThreads, (x))
@@ -809,8 +833,10 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
   const int n = bid / (nsplit * a.Hv);
   const int hk = h / (a.Hv / a.Hk);
   const int tid = threadIdx.x, warp = tid >> 5;
-  pdl_wait();  // W, U~, G of this call (unless `ready`), and the carry of the previous launch
+  pdl_wait();  // W, U~, G of this call, and the carry of the previous launch
   const int s_first = a.ws.seq_first[n], s_end = a.ws.seq_first[n + 1];
+  if (!GDN_IN_BOUNDS(s_first >= 0 && s_end >= s_first && s_end <= a.T / kC + a.N, a.status))
+    return;
   const int first = max(s_first, a.c0);
   const int nch = min(s_end, a.c1) - first;
   // an empty sequence belongs to the launch whose range holds its position in the chunk table
@@ -831,17 +857,25 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
   CSYNC();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t colS = 0, colX = Cfg::kTmemCols / 2;
+  const uint32_t colS = 0, colX = DV, colM = 2 * DV;
   constexpr int kCPT = Cfg::kCPT, kGroups = kCPT / 32;
   const uint32_t lane_addr = tmem_at(tmem, (warp & 3) * 32, 0);
   const int k_row = tid & 127;  // TMEM lane = d_k index for S^T, = token index for X
   const int cs = (tid >> 7) * kCPT;  // first column of this thread inside the d_v block
-  const size_t sbase = ((size_t)state_row(a.slot, n) * a.Hv + h) * kD * kD;
+  const int srow = state_row(a.slot, n, a.num_slots);  // -1: slot out of range
+  if (srow < 0 && tid == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
+  const size_t sbase = ((size_t)(srow < 0 ? 0 : srow) * a.Hv + h) * kD * kD;
+  // state outputs after chunks (and, with MID, after the first 64 tokens of a chunk): entry of
+  // the state after chunk j of this sequence, and of the one in its middle
+  const int page_first = MID ? a.ws.page_first[n] : 0;
+  auto end_entry = [&](int c, int L) {
+    return MID ? page_first + 2 * (c - s_first) + (L > 64 ? 1 : 0) : c;
+  };
 
   // ---- S^T initial value: lane k, column v  (state layout [v][k])
   {
     const float* src = from_carry ? a.carry_in + (size_t)h * kD * kD
-                                  : (a.S0 ? a.S0 + sbase : nullptr);
+                                  : (a.S0 && srow >= 0 ? a.S0 + sbase : nullptr);
 #pragma unroll
     for (int gi = 0; gi < kGroups; ++gi) {
       float v[32];
@@ -854,8 +888,16 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     }
     tmem_st_wait();
   }
+  // thread 0's count of loads issued and waited for, to drain them after a failed wait; a W
+  // load left out on purpose (debug fault injection: the first chain CTA skips the load of chunk
+  // a.fault_chunk, so that its bounded wait runs out) is never waited for in the drain
+  int w_issued = 0, w_done = 0, k_issued = 0, k_done = 0, w_skipped = -1;
   auto issue_w = [&](int ci) {
     const int c = first + ci;
+    if (bid == 0 && c == a.fault_chunk) {
+      w_skipped = ci;
+      return;
+    }
     const int st = Cfg::kWStages == 1 ? 0 : (ci & 1);
     uint8_t* dst = sm + st * 2 * kTile;
     mbar_arrive_expect_tx(bar_w + st, 2 * kTile);
@@ -871,21 +913,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     tma_load_2d(dst, &mapK, bar_k, 0, row);
     tma_load_2d(dst + kTile, &mapK, bar_k, 64, row);
   };
-  // thread 0's count of loads issued and waited for, to drain them after a failed wait
-  int w_issued = 0, w_done = 0, k_issued = 0, k_done = 0;
   bool mma_pending = false;
-  bool flag_ok = true;
-  int flag_next = 0;  // thread 0: relaxed read of the next chunk's flag
-  if (ready && nch > 0) {
-    if (tid == 0) flag_ok = wait_flag(ready + first * a.Hv + h);
-    if (CSYNC_OR(!flag_ok)) {
-      if (tid == 0) report_status(a.status, GDN_ERR_TIMEOUT);
-      tc_fence_before();
-      CSYNC();
-      if (warp == 0) tmem_dealloc(tmem, Cfg::kTmemCols);
-      return;
-    }
-  }
   if (tid == 0 && nch > 0) {
     issue_w(0);
     issue_k(0);
@@ -899,36 +927,28 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
   constexpr int kVec = kCPT / 8;
   uint4 ut_cur[kVec], ut_nxt[kVec];
   float Gi_cur = 0.f, Gl_cur = 0.f, Gi_nxt = 0.f, Gl_nxt = 0.f;
-  auto load_chunk_rows = [&](int ci, uint4 (&ut)[kVec], float& Gi, float& Gl) {
+  float Gm_cur = 0.f, Gm_nxt = 0.f;  // G after token 63 (MID)
+  int L_cur = 0, L_nxt = 0;          // tokens in the chunk (state outputs)
+  auto load_chunk_rows = [&](int ci, uint4 (&ut)[kVec], float& Gi, float& Gl, float& Gm,
+                             int& L) {
     const int c = first + ci;
     const float* Gc = a.ws.Gw + ((size_t)c * a.Hv + h) * kC;
     Gi = Gc[k_row];
     Gl = Gc[kC - 1];
+    if (MID) Gm = Gc[63];
+    if (a.chunk_states) L = a.ws.chunks[c].L;
     const uint4* src = reinterpret_cast<const uint4*>(
         a.ws.Uw + (((size_t)c * a.Hv + h) * kC + k_row) * kD + v0 + cs);
 #pragma unroll
     for (int q = 0; q < kVec; ++q) ut[q] = src[q];
   };
-  if (nch > 0) load_chunk_rows(0, ut_cur, Gi_cur, Gl_cur);
+  if (nch > 0) load_chunk_rows(0, ut_cur, Gi_cur, Gl_cur, Gm_cur, L_cur);
   for (int ci = 0; ci < nch; ++ci) {
     const int c = first + ci;
     const int wst = Cfg::kWStages == 1 ? 0 : (ci & 1);
     const uint32_t wphase = Cfg::kWStages == 1 ? (ci & 1) : ((ci >> 1) & 1);
-    // the next chunk's prep must be published before any of its loads (thread 0 issues the W
-    // load; every thread reads its U~ rows after the barrier below)
-    if (ready && tid == 0 && ci + 1 < nch) {
-      // the flag of chunk c + 1 was read (relaxed) one step ago; if it was set, an acquire
-      // fence completes the synchronisation, otherwise wait for it
-      if (flag_next != 0) {
-        fence_acq_rel_gpu();
-        fence_proxy_async_global();
-      } else {
-        flag_ok = wait_flag(ready + (c + 1) * a.Hv + h);
-      }
-      flag_next = ci + 2 < nch ? ld_relaxed_gpu(ready + (c + 2) * a.Hv + h) : 1;
-    }
     __syncwarp();  // warp 0 reconverges before its TMEM loads
-    if (Cfg::kWStages == 2 && tid == 0 && ci + 1 < nch && flag_ok) {
+    if (Cfg::kWStages == 2 && tid == 0 && ci + 1 < nch) {
       issue_w(ci + 1);
       ++w_issued;
     }
@@ -939,10 +959,16 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     const float gam = __expf(Gl_cur);
     __nv_bfloat16* Srow = a.ws.Sw + (((size_t)c * a.Hv + h) * kD + k_row) * kD + v0 + cs;
     float sreg[kGroups][32];
+    float smid[MID ? kGroups : 1][32];  // e^(G_63) S_c^T, the decayed part of the middle state
 #pragma unroll
     for (int gi = 0; gi < kGroups; ++gi) {
       tmem_ld32(lane_addr + colS + cs + gi * 32, sreg[gi]);
       tmem_ld_wait();
+      if constexpr (MID) {
+        const float gm = __expf(Gm_cur);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) smid[gi][e] = gm * sreg[gi][e];
+      }
 
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -966,7 +992,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     CSYNC();
     // ---- X = W S_b^T  (M = 128 tokens, N = DV, K = d_k)
     if (tid == 0) {
-      ok = flag_ok && mbar_wait(bar_w + wst, wphase);
+      ok = mbar_wait(bar_w + wst, wphase, a.wait_ns);
       tc_fence_after();
       if (ok) {
         ++w_done;
@@ -996,9 +1022,9 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
       }
       tmem_st_wait();
     }
-    if (ci + 1 < nch) load_chunk_rows(ci + 1, ut_nxt, Gi_nxt, Gl_nxt);
+    if (ci + 1 < nch) load_chunk_rows(ci + 1, ut_nxt, Gi_nxt, Gl_nxt, Gm_nxt, L_nxt);
     if ((failed = CSYNC_OR(!ok))) break;
-    ok = mbar_wait(bar_mma, mma_phase);
+    ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
     if ((failed = CSYNC_OR(!ok))) break;
     mma_phase ^= 1;
     mma_pending = false;
@@ -1013,6 +1039,9 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     __nv_bfloat16* Urow = a.ws.Uw + (((size_t)c * a.Hv + h) * kC + k_row) * kD + v0 + cs;
     {
       const float dec = __expf(Gl_cur - Gi_cur);
+      // MID: the first 64 tokens of U, decayed to token 63, for the state in the middle of the
+      // chunk (rows 64..127 of that operand are never read)
+      const float decm = MID && k_row < 64 ? __expf(Gm_cur - Gi_cur) : 0.f;
 #pragma unroll
       for (int gi = 0; gi < kGroups; ++gi) {
         float v[32];
@@ -1033,6 +1062,11 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
 #pragma unroll
           for (int e = 0; e < 8; ++e) h8[e] = u8[e] * dec;
           st_row8_bf16(OP, kTile, k_row, (cs >> 3) + vq, h8);
+          if (MID && k_row < 64) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) h8[e] = u8[e] * decm;
+            st_row8_bf16(sm + Cfg::kOpMid, kTile, k_row, (cs >> 3) + vq, h8);
+          }
           if constexpr (!kOverlap) {
             float w8[8];
 #pragma unroll
@@ -1047,7 +1081,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     CSYNC();
     // ---- S^T += K^T U^  (M = d_k, N = DV, K = tokens)
     if (tid == 0) {
-      ok = mbar_wait(bar_k, ci & 1);
+      ok = mbar_wait(bar_k, ci & 1, a.wait_ns);
       tc_fence_after();
       if (ok) {
         ++k_done;
@@ -1056,6 +1090,15 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16(tmem + colS, desc_mnmajor(sK, kk, kTile), desc_mnmajor(sU, kk, kTile),
                    idesc_bf16(128, DV, true, true), 1);
+        if (MID && L_cur > 64) {
+          // S_mid^T = e^(G_63) S_c^T + K[0:64]^T U^mid: the product over tokens 0..63 here,
+          // the decayed state added at the readout
+          const uint32_t sUm = smem_u32(sm + Cfg::kOpMid);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16(tmem + colM, desc_mnmajor(sK, kk, kTile), desc_mnmajor(sUm, kk, kTile),
+                     idesc_bf16(128, DV, true, true), kk > 0);
+        }
         mma_commit(bar_mma);
         mma_pending = true;
       }
@@ -1071,14 +1114,15 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
       }
     }
     if ((failed = CSYNC_OR(!ok))) break;
-    ok = mbar_wait(bar_mma, mma_phase);
+    ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
     if ((failed = CSYNC_OR(!ok))) break;
     mma_phase ^= 1;
     mma_pending = false;
     tc_fence_after();
     if (a.chunk_states) {
       // the state after chunk c (fp32, layout [v][k]), for prefix and branch caching
-      float* cst = a.chunk_states + (((size_t)c * a.Hv + h) * kD + v0 + cs) * kD + k_row;
+      float* cst = a.chunk_states +
+                   (((size_t)end_entry(c, L_cur) * a.Hv + h) * kD + v0 + cs) * kD + k_row;
 #pragma unroll
       for (int gi = 0; gi < kGroups; ++gi) {
         float v[32];
@@ -1086,6 +1130,18 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) cst[(gi * 32 + e) * kD] = v[e];
+      }
+      if (MID && L_cur > 64) {
+        // and the state after the chunk's first 64 tokens (the entry before the chunk end's)
+        float* mst = cst - (size_t)a.Hv * kD * kD;
+#pragma unroll
+        for (int gi = 0; gi < kGroups; ++gi) {
+          float v[32];
+          tmem_ld32(lane_addr + colM + cs + gi * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mst[(gi * 32 + e) * kD] = v[e] + smid[MID ? gi : 0][e];
+        }
       }
     }
     // the update has consumed K and the operand tile
@@ -1097,8 +1153,11 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     for (int q = 0; q < kVec; ++q) ut_cur[q] = ut_nxt[q];
     Gi_cur = Gi_nxt;
     Gl_cur = Gl_nxt;
+    Gm_cur = Gm_nxt;
+    L_cur = L_nxt;
   }
-  float* dst = to_carry ? a.carry_out + (size_t)h * kD * kD : (a.SN ? a.SN + sbase : nullptr);
+  float* dst = to_carry ? a.carry_out + (size_t)h * kD * kD
+                        : (a.SN && srow >= 0 ? a.SN + sbase : nullptr);
   if (!failed && dst) {
 #pragma unroll
     for (int gi = 0; gi < kGroups; ++gi) {
@@ -1114,10 +1173,11 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     // give loads and products still in flight a bounded time to land before the CTA's shared
     // memory and TMEM are released
     for (int j = w_done; j < w_issued; ++j)
-      mbar_wait(bar_w + (Cfg::kWStages == 1 ? 0 : (j & 1)),
-                Cfg::kWStages == 1 ? (j & 1) : ((j >> 1) & 1));
-    for (int j = k_done; j < k_issued; ++j) mbar_wait(bar_k, j & 1);
-    if (mma_pending) mbar_wait(bar_mma, mma_phase);
+      if (j != w_skipped)
+        mbar_wait(bar_w + (Cfg::kWStages == 1 ? 0 : (j & 1)),
+                Cfg::kWStages == 1 ? (j & 1) : ((j >> 1) & 1), a.wait_ns);
+    for (int j = k_done; j < k_issued; ++j) mbar_wait(bar_k, j & 1, a.wait_ns);
+    if (mma_pending) mbar_wait(bar_mma, mma_phase, a.wait_ns);
   }
   tc_fence_before();
   CSYNC();
@@ -1126,7 +1186,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
 #undef CSYNC_OR
 }
 
-template <int DV>
+template <int DV, bool MID>
 __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(PrefillArgs a,
                                                            const __grid_constant__ CUtensorMap mapW,
                                                            const __grid_constant__ CUtensorMap mapK) {
@@ -1134,59 +1194,7 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   pdl_trigger();
-  chain_body<DV, ChainCfg<DV>::kWStages>(a, mapW, mapK, blockIdx.x, sm, nullptr);
-}
-
-// ------------------------------------------------------------------------ prep + chain
-// One persistent launch of prep and chain, for a chunk table with few chains: CTAs below
-// `nchain` run one chain each (d_v blocks of DV columns); every other CTA is a prep worker that
-// takes (chunk, value head) units in chunk-major order from a device counter and publishes each
-// unit with a flag the chain waits for.  Workers never wait on the chains, so the chains make
-// progress as long as a worker holds an SM slot, which a grid of (SM slots) CTAs with fewer
-// chains than slots guarantees; every wait is bounded in any case.  The flags and the counter
-// are zeroed by the chunk-table kernel of the same call.
-// The chain role keeps a single W buffer here, so that two CTAs of either role fit on an SM.
-template <int DV>
-constexpr uint32_t fused_smem() {
-  return ChainCfg<DV, 1>::kSmem > kPrepSmem ? ChainCfg<DV, 1>::kSmem : kPrepSmem;
-}
-
-template <int DV>
-__global__ void __launch_bounds__(256, 2) gdn_prep_chain_kernel(
-    PrefillArgs a, const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
-    const __grid_constant__ CUtensorMap mapW, int nchain) {
-  static_assert(ChainCfg<DV, 1>::kThreads <= 256, "block size");
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
-  if ((int)blockIdx.x < nchain) {
-    // a chain uses the first ChainCfg::kThreads threads; the others leave at once
-    if ((int)threadIdx.x < ChainCfg<DV, 1>::kThreads)
-      chain_body<DV, 1>(a, mapW, mapK, blockIdx.x, sm, a.ws.ready);
-    return;
-  }
-  const PrepCtl ctl(sm);
-  const int tid = threadIdx.x;
-  pdl_wait();  // the chunk table
-  const int units = a.ws.seq_first[a.N] * a.Hv;
-  if (tid == 128) ctl.init();
-  if (tid < 32) tmem_alloc(ctl.tslot, 256);
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *ctl.tslot;
-  uint32_t par = 0;
-  while (true) {
-    if (tid == 0) *ctl.unit = atomicAdd(a.ws.counter, 1);
-    __syncthreads();
-    const int u = *ctl.unit;
-    if (u >= units) break;
-    if (!prep_unit(a, mapK, mapV, mapW, u / a.Hv, u % a.Hv, sm, tmem, par, a.ws.ready)) break;
-    par ^= 1;
-    __syncthreads();  // shared memory and the unit slot are reused
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (tid < 32) tmem_dealloc(tmem, 256);
+  chain_body<DV, MID>(a, mapW, mapK, blockIdx.x, sm);
 }
 
 // ----------------------------------------------------------------------------------- out
@@ -1226,6 +1234,10 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
     return;
   }
   const ChunkInfo ci = a.ws.chunks[c];
+  if (!GDN_IN_BOUNDS(ci.t0 >= 0 && ci.L > 0 && ci.L <= kC && ci.t0 + ci.L <= a.T, a.status)) {
+    pdl_wait();
+    return;
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int quarter = warp & 3, half = warp >> 2;
   const int i = quarter * 32 + lane;  // token row of this thread
@@ -1273,7 +1285,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
   uint32_t mma_phase = 0;
   // ---- Q K^T
   if (tid == 0) {
-    ok = mbar_wait(bar_qk, 0);
+    ok = mbar_wait(bar_qk, 0, a.wait_ns);
     tc_fence_after();
     if (ok) {
 #pragma unroll
@@ -1284,7 +1296,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
     }
   }
   if (__syncthreads_or(!ok)) goto done;
-  ok = mbar_wait(bar_mma, mma_phase);
+  ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
   mma_phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
@@ -1351,7 +1363,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
   __syncthreads();
   // ---- O = Q^ S^T + P U   (A operands from TMEM)
   if (tid == 0) {
-    ok = mbar_wait(bar_s, 0) && mbar_wait(bar_u, 0);
+    ok = mbar_wait(bar_s, 0, a.wait_ns) && mbar_wait(bar_u, 0, a.wait_ns);
     tc_fence_after();
     if (ok) {
       constexpr uint32_t id = idesc_bf16(128, 128, false, true);
@@ -1365,7 +1377,7 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
     }
   }
   if (__syncthreads_or(!ok)) goto done;
-  ok = mbar_wait(bar_mma, mma_phase);
+  ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
   mma_phase ^= 1;
   if (__syncthreads_or(!ok)) goto done;
   tc_fence_after();
@@ -1427,21 +1439,11 @@ using gdn::kD;
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-static int env_int(const char* name, int dflt) {
-  const char* v = getenv(name);
-  if (!v || !*v) return dflt;
-  char* end = nullptr;
-  const long x = strtol(v, &end, 10);
-  return (end && *end == 0 && x >= 0 && x < (1 << 20)) ? (int)x : dflt;
-}
-
 // Launch with programmatic stream serialisation: the kernel may start while the previous kernel
 // in the stream drains, and waits for it with griddepcontrol.wait before touching its outputs.
-// GDN_PDL=0 turns this off (plain stream order).
 template <typename... KArgs, typename... Args>
 static cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                             cudaStream_t s, Args&&... args) {
-  static const bool enabled = env_int("GDN_PDL", 1) != 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -1451,7 +1453,7 @@ static cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 bl
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = (pdl && enabled) ? 1 : 0;
+  cfg.numAttrs = (pdl && !trace_attached()) ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -1461,8 +1463,8 @@ static cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 bl
 // the sequential chain overlaps the parallel kernels instead of following them.  The parallel
 // kernels already fill every SM (two CTAs each, bound by shared memory), so the overlap only
 // pays where the chain is long: by default the table is cut only from 512 chunks on, into
-// segments of 64.  GDN_SEGMENT_CHUNKS=<n> sets the segment length (a value at or above the
-// chunk count gives a single launch of each kernel).
+// segments of 64.  The debug option segment_chunks sets the segment length (a value at or above
+// the chunk count gives a single launch of each kernel).
 struct SegPlan {
   int nseg, seg;
 };
@@ -1470,7 +1472,7 @@ struct SegPlan {
 static SegPlan seg_plan(int N, int T) {
   const int NC = T / kC + N;
   if (T == 0 || NC <= 1) return {1, NC > 0 ? NC : 1};
-  int target = env_int("GDN_SEGMENT_CHUNKS", 0);
+  int target = debug_opts().segment_chunks;
   if (target <= 0) target = NC >= 512 ? 64 : NC;
   int nseg = (NC + target - 1) / target;
   if (nseg < 1) nseg = 1;
@@ -1480,7 +1482,7 @@ static SegPlan seg_plan(int N, int T) {
 }
 
 struct WsLayout {
-  size_t chunks, seq_first, Qw, Kw, Ww, Uw, Sw, Gw, ready, carry, total;
+  size_t chunks, seq_first, page_first, Qw, Kw, Ww, Uw, Sw, Gw, carry, total;
 };
 
 static WsLayout ws_layout(int N, int T, int Hk, int Hv) {
@@ -1491,13 +1493,13 @@ static WsLayout ws_layout(int N, int T, int Hk, int Hv) {
   size_t o = 0;
   l.chunks = o; o = align_up(o + NC * sizeof(gdn::ChunkInfo), 1024);
   l.seq_first = o; o = align_up(o + (size_t)(N + 1) * 4, 1024);
+  l.page_first = o; o = align_up(o + (size_t)(N + 1) * 4, 1024);
   l.Qw = o; o = align_up(o + NC * Hk * tile, 1024);
   l.Kw = o; o = align_up(o + NC * Hk * tile, 1024);
   l.Ww = o; o = align_up(o + NC * Hv * tile, 1024);
   l.Uw = o; o = align_up(o + NC * Hv * tile, 1024);
   l.Sw = o; o = align_up(o + NC * Hv * tile, 1024);
   l.Gw = o; o = align_up(o + NC * Hv * kC * 4, 1024);
-  l.ready = o; o = align_up(o + NC * Hv * 4 + 4, 1024);  // flags, then the work counter
   // one fp32 [Hv][d][d] state per segment boundary (at most one sequence crosses each)
   l.carry = o; o = align_up(o + (size_t)(p.nseg - 1) * Hv * kD * kD * 4, 1024);
   l.total = o;
@@ -1545,26 +1547,26 @@ static bool make_map_x(CUtensorMap* m, const void* base, int T, int Cc) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DV>
+template <int DV, bool MID>
 static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW,
                                 const CUtensorMap& mK, cudaStream_t s, bool pdl) {
-  using Cfg = gdn::ChainCfg<DV>;
+  using Cfg = gdn::ChainCfg<DV, MID>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(gdn::gdn_chain_kernel<DV>,
+    cudaError_t e = cudaFuncSetAttribute(gdn::gdn_chain_kernel<DV, MID>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   trace_begin("gdn_chain", s);
-  cudaError_t e = launch_k(pdl, gdn::gdn_chain_kernel<DV>, dim3(a.N * a.Hv * a.nsplit),
+  cudaError_t e = launch_k(pdl, gdn::gdn_chain_kernel<DV, MID>, dim3(a.N * a.Hv * a.nsplit),
                            dim3(Cfg::kThreads), Cfg::kSmem, s, a, mW, mK);
   trace_end(s);
   return e;
 }
 
 int choose_nsplit(int N, int Hv) {
-  const int forced = env_int("GDN_CHAIN_SPLIT", 0);
+  const int forced = debug_opts().chain_split;
   if (forced == 1 || forced == 2 || forced == 4) return forced;
   const int units = N * Hv;
   if (units >= 148) return 1;
@@ -1616,40 +1618,13 @@ static cudaError_t pipe_streams(PipeStreams** out) {
   return cudaSuccess;
 }
 
-// Grid of the persistent prep + chain kernel: two CTAs per SM.  Its shape (256 threads of at most
-// 128 registers, about 100 KB of shared memory) is built to fit twice on an SM; with fewer
-// resident, the chains (low block indices) still leave slots to the workers, only fewer.
-static cudaError_t fused_slots(int* grid) {
-  static_assert(gdn::fused_smem<32>() + 1024 <= 232448 / 2, "two CTAs per SM");
-  constexpr int kMaxDev = 64;
-  static int cached[kMaxDev] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-  if (!cached[dev]) {
-    if ((e = cudaFuncSetAttribute(gdn::gdn_prep_chain_kernel<32>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  gdn::fused_smem<32>())) != cudaSuccess ||
-        (e = cudaFuncSetAttribute(gdn::gdn_prep_chain_kernel<32>,
-                                  cudaFuncAttributePreferredSharedMemoryCarveout,
-                                  cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
-      return e;
-    int nsm = 0;
-    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-      return e;
-    cached[dev] = 2 * nsm;
-  }
-  *grid = cached[dev];
-  return cudaSuccess;
-}
-
 cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t s) {
   const WsLayout l = ws_layout(a.N, a.T, a.Hk, a.Hv);
   const SegPlan plan = seg_plan(a.N, a.T);
   uint8_t* w = static_cast<uint8_t*>(workspace);
   a.ws.chunks = reinterpret_cast<gdn::ChunkInfo*>(w + l.chunks);
   a.ws.seq_first = reinterpret_cast<int32_t*>(w + l.seq_first);
+  a.ws.page_first = reinterpret_cast<int32_t*>(w + l.page_first);
   a.ws.Qw = reinterpret_cast<__nv_bfloat16*>(w + l.Qw);
   a.ws.Kw = reinterpret_cast<__nv_bfloat16*>(w + l.Kw);
   a.ws.Ww = reinterpret_cast<__nv_bfloat16*>(w + l.Ww);
@@ -1657,8 +1632,6 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   a.ws.Sw = reinterpret_cast<__nv_bfloat16*>(w + l.Sw);
   a.ws.Gw = reinterpret_cast<float*>(w + l.Gw);
   const size_t NC = (size_t)a.T / kC + (size_t)a.N + 1;
-  a.ws.ready = reinterpret_cast<int*>(w + l.ready);
-  a.ws.counter = a.ws.ready + NC * a.Hv;
   float* carry = reinterpret_cast<float*>(w + l.carry);
   const size_t carry_stride = (size_t)a.Hv * kD * kD;
   CUtensorMap mQ, mK, mW, mU, mS, mX;
@@ -1683,27 +1656,15 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     attr = true;
   }
   cudaError_t e;
-  // Persistent prep + chain (one launch), opt-in with GDN_FUSED=1: one chain CTA per (sequence,
-  // value head, 32-column block), the other SM slots as prep workers.  It hides the chain
-  // behind prep, but a chain step sharing its SM with a worker (and acquiring the ready flag)
-  // takes about twice as long as alone, so at the Qwen3-Next shape with T = 4096 it measured
-  // slower than the separate launches (177 us against 64 + 64 us); off by default.
-  int fused_grid = 0, nchain = 0;
-  if (plan.nseg <= 1 && a.T > 0 && env_int("GDN_FUSED", 0) != 0) {
-    if ((e = fused_slots(&fused_grid)) != cudaSuccess) return e;
-    nchain = a.N * a.Hv * 4;
-    if (2 * nchain > fused_grid) fused_grid = 0;
-  }
-  const bool fused = fused_grid > 0;
   trace_begin("chunk_schedule", s);
   // one CTA; its width only needs to cover the sequences of one pass of the scan
-  const int sched_threads = a.N <= 32 ? 32 : (a.N <= 256 ? 256 : 1024);
+  const int sched_work = std::max(a.N, a.T / kC);
+  const int sched_threads = sched_work <= 32 ? 32 : (sched_work <= 256 ? 256 : 1024);
   gdn::chunk_schedule_kernel<<<1, sched_threads, 0, s>>>(
-      a.cu, a.N, a.ws, fused ? (int)(NC * a.Hv) : 0, a.conv0, a.convN, a.slot, Cc);
+      a.cu, a.N, a.T, a.ws, a.conv0, a.convN, a.slot, a.num_slots, Cc, a.status);
   trace_end(s);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  // one segment's kernels on the given streams
   // one segment's kernels on the given streams; `pdl` where each follows the previous kernel
   // of the same stream with no other dependency in between
   auto launch_parallel_front = [&](const gdn::PrefillArgs& sa, cudaStream_t st,
@@ -1721,10 +1682,17 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     return e2;
   };
   auto launch_chain_any = [&](gdn::PrefillArgs sa, cudaStream_t st, bool pdl) -> cudaError_t {
+    if (sa.page64) {
+      switch (sa.nsplit) {
+        case 4: return launch_chain<32, true>(sa, mW, mK, st, pdl);
+        case 2: return launch_chain<64, true>(sa, mW, mK, st, pdl);
+        default: sa.nsplit = 1; return launch_chain<128, true>(sa, mW, mK, st, pdl);
+      }
+    }
     switch (sa.nsplit) {
-      case 4: return launch_chain<32>(sa, mW, mK, st, pdl);
-      case 2: return launch_chain<64>(sa, mW, mK, st, pdl);
-      default: sa.nsplit = 1; return launch_chain<128>(sa, mW, mK, st, pdl);
+      case 4: return launch_chain<32, false>(sa, mW, mK, st, pdl);
+      case 2: return launch_chain<64, false>(sa, mW, mK, st, pdl);
+      default: sa.nsplit = 1; return launch_chain<128, false>(sa, mW, mK, st, pdl);
     }
   };
   auto launch_out = [&](const gdn::PrefillArgs& sa, cudaStream_t st, bool pdl) -> cudaError_t {
@@ -1736,24 +1704,6 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   };
 
   const int NCmax = a.T / kC + a.N;
-  if (fused) {
-    a.c0 = 0;
-    a.c1 = NCmax;
-    a.carry_in = nullptr;
-    a.carry_out = nullptr;
-    a.nsplit = 4;
-    trace_begin("gdn_qkv", s);
-    e = launch_k(true, gdn::gdn_qkv_kernel, dim3(2 * a.Hk + a.Hv, NCmax), dim3(128), gdn::kQkvSmem,
-                 s, a, mX);
-    trace_end(s);
-    if (e != cudaSuccess) return e;
-    trace_begin("gdn_prep_chain", s);
-    e = launch_k(true, gdn::gdn_prep_chain_kernel<32>, dim3(fused_grid), dim3(256),
-                 gdn::fused_smem<32>(), s, a, mK, mU, mW, nchain);
-    trace_end(s);
-    if (e != cudaSuccess) return e;
-    return launch_out(a, s, true);
-  }
   if (plan.nseg <= 1) {
     a.c0 = 0;
     a.c1 = NCmax;

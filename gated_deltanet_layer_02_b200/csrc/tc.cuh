@@ -18,8 +18,9 @@
 
 namespace gdn {
 
-// Upper bound of every device-side wait, in ns of %globaltimer.  A wait that runs out sets the
-// kernel's status word to GDN_ERR_TIMEOUT and the CTA abandons its work.
+// Default upper bound of every device-side wait, in ns of %globaltimer (a call may set another
+// through its arguments).  A wait that runs out sets the kernel's status word to
+// GDN_ERR_TIMEOUT and the CTA abandons its work.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -59,13 +60,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// Bounded wait for phase `parity` of `bar`.  Returns false after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Bounded wait for phase `parity` of `bar`.  Returns false after limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
     __nanosleep(20);
   }
 }
@@ -86,18 +88,6 @@ __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
-// Bounded wait until *flag is non-zero (acquire), then a proxy fence so that TMA loads issued
-// afterwards see what the flag publishes.  Returns false after kWaitLimitNs.
-__device__ __forceinline__ bool wait_flag(const int* flag) {
-  const uint64_t t0 = global_timer_ns();
-  while (ld_acquire_gpu(flag) == 0) {
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(64);
-  }
-  fence_proxy_async_global();
-  return true;
-}
-
 // 2-D tiled TMA load, completion signalled on `bar` (transaction bytes).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y) {

@@ -23,9 +23,10 @@
  * General rules for every call:
  *   - Pointers are DEVICE pointers owned by the caller unless a comment says "host".  The
  *     library allocates no device memory of its own, except where an entry point says so
- *     (gdn_chunk_prefill_static_ws: a static array; gdn_block_prefill: a cuBLAS handle).  Its
- *     multi-stream paths create CUDA streams and events once per host thread and device and
- *     keep them; no other state survives a call.
+ *     (gdn_chunk_prefill_static_ws: a static array).  Its multi-stream paths create CUDA
+ *     streams and events once per host thread and device and keep them; debug settings
+ *     (gdn_debug_set) and an attached trace are per host thread; no other state survives a
+ *     call.
  *   - Tensors are dense, row-major, contiguous and 16-byte aligned.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *   - Return value: GDN_OK, or a negative gdn_status.  On argument errors nothing is launched
@@ -45,15 +46,19 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2
 
 typedef enum gdn_status {
   GDN_OK = 0,
-  GDN_ERR_INVALID_ARG = -1, /* null/misaligned pointer, negative size, bad cu_seqlens shape */
+  GDN_ERR_INVALID_ARG = -1, /* null/misaligned pointer, negative size, bad cu_seqlens shape;
+                               on the device: a slot index outside its pool */
   GDN_ERR_UNSUPPORTED = -2, /* shape or dtype this build does not implement */
   GDN_ERR_CUDA = -3,        /* a CUDA runtime call or kernel launch failed */
   GDN_ERR_TIMEOUT = -4,     /* written to dev_status by a device wait that ran out */
-  GDN_ERR_WORKSPACE = -5    /* workspace missing or smaller than *_workspace_size() */
+  GDN_ERR_WORKSPACE = -5,   /* workspace missing or smaller than *_workspace_size() */
+  GDN_ERR_BOUNDS = -6       /* bounds-check build only (libgdn_checked.so, compiled with
+                               -DGDN_BOUNDS_CHECK): a kernel index check failed and the access
+                               was skipped; never reported by the normal build */
 } gdn_status;
 
 typedef enum gdn_dtype { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -156,6 +161,30 @@ int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* 
                              void* stream);
 
 /*
+ * gdn_chunk_prefill_pages -- gdn_chunk_prefill_states for a cache page of 64 or 128 tokens.
+ * Source: the "Qwen3-Next" SGLang cookbook, section 3.2, radix cache for the hybrid layers: its
+ * example serves with --page-size 64, and the page size must divide the linear-attention
+ * kernel's chunk or be a multiple of it; with this library's 128-token chunk, pages of 64 need
+ * the state in the middle of every chunk as well.
+ *   page_size     64 or 128 (GDN_ERR_UNSUPPORTED otherwise).  128: the result of
+ *                 gdn_chunk_prefill_states.
+ *   page_states   [P, Hv, d, d] fp32, P = sum over sequences of ceil(L_n / page_size): entry p is
+ *                 the state after page p, pages numbered sequence by sequence (sequence n's page
+ *                 j covers its tokens [page_size j, min(page_size (j + 1), L_n))); the entry of a
+ *                 sequence's last page equals its final state.  Required when num_tokens > 0.
+ * With 64, the chain adds for each chunk of more than 64 tokens the state after its first 64:
+ * e^(G_63) S_c + K[0:64]^T diag(e^(G_63 - G_i)) U[0:64] (the chunk's own U, fp32 accumulation).
+ * bf16 only.  Other arguments, the workspace size and the status codes: gdn_chunk_prefill.
+ */
+int gdn_chunk_prefill_pages(const gdn_dims* dims, gdn_dtype dtype, const void* x,
+                            const void* conv_w, const float* beta, const float* g, const void* z,
+                            const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
+                            int32_t num_tokens, const float* S0, float* SN, const void* conv0,
+                            void* convN, void* out, int32_t page_size, float* page_states,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream);
+
+/*
  * gdn_chunk_prefill_host -- gdn_chunk_prefill (bf16) with the per-token tensors in host memory.
  * Source: as gdn_chunk_prefill.  The packed batch is cut into segments of about segment_tokens
  * tokens, ending at sequence ends or 128-token chunk boundaries of a sequence; the copy of one
@@ -172,7 +201,9 @@ int gdn_chunk_prefill_states(const gdn_dims* dims, gdn_dtype dtype, const void* 
  *   workspace: device, gdn_chunk_prefill_host_workspace_size() bytes, 256-byte aligned (it
  *     holds device copies of the per-token tensors).
  * Asynchronous on `stream`: the host buffers may be reused, and out read, once `stream` has
- * reached the point of the call.  Not for stream capture (the copy streams are the library's).
+ * reached the point of the call.  This holds on error returns too: copies queued before the
+ * error still read or write the host buffers, and `stream` waits for them.  Not for stream
+ * capture (the copy streams are the library's).
  * Status codes as gdn_chunk_prefill; GDN_ERR_UNSUPPORTED unless Hv = 2 Hk and Hv % 4 == 0.
  * gdn_chunk_prefill_host_plan writes the segments (first sequence, sequences, first token,
  * tokens; four int32 each) into `segments` and returns their number (or a status < 0;
@@ -196,8 +227,11 @@ int gdn_chunk_prefill_host(const gdn_dims* dims, const void* x, const void* conv
  * pool shared with gdn_decode_step: sequence n reads and overwrites row slot_idx[n] of the pools.
  * Source: the "Qwen3-Next" SGLang cookbook, section 3.2 (the mamba state cache of the hybrid GDN
  * layers, one cached state per request slot, fp32 by default).
- *   slot_idx  [N] int32 device, nullable (= identity); the slots of one call must be distinct
- *             and inside the pools (not checked on the device).
+ *   slot_idx  [N] int32 device, nullable (= identity); the slots of one call must be distinct.
+ *   num_slots rows of the pools (>= N when slot_idx is NULL).  The kernels check every slot
+ *             against it: a sequence whose slot lies outside [0, num_slots) starts from zero
+ *             states, writes no state and sets dev_status to GDN_ERR_INVALID_ARG (its outputs
+ *             are computed from the zero states); no pool row outside the range is touched.
  *   S_pool    [slots, Hv, d, d] fp32, in/out, required when N > 0.
  *   conv_pool [slots, K-1, Cc] (activation dtype), in/out, nullable: zero conv history, none kept.
  * Every other argument, the workspace size and the status codes are those of gdn_chunk_prefill;
@@ -207,9 +241,9 @@ int gdn_chunk_prefill_host(const gdn_dims* dims, const void* x, const void* conv
 int gdn_chunk_prefill_slots(const gdn_dims* dims, gdn_dtype dtype, const void* x,
                             const void* conv_w, const float* beta, const float* g, const void* z,
                             const void* norm_w, const int32_t* cu_seqlens, int32_t num_seqs,
-                            int32_t num_tokens, const int32_t* slot_idx, float* S_pool,
-                            void* conv_pool, void* out, void* workspace, size_t workspace_bytes,
-                            int32_t* dev_status, void* stream);
+                            int32_t num_tokens, const int32_t* slot_idx, int32_t num_slots,
+                            float* S_pool, void* conv_pool, void* out, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
  * gdn_decode_step -- one token for each of B sequences; conv and recurrent state in place.
@@ -218,13 +252,16 @@ int gdn_chunk_prefill_slots(const gdn_dims* dims, gdn_dtype dtype, const void* x
  *   x [B, Cc], beta/g [B, Hv] fp32, z [B, Hv, d] nullable, conv_w [Cc, K] (required),
  *   norm_w [d] nullable, conv_state [slots, K-1, Cc] in/out, S [slots, Hv, d, d] fp32 in/out,
  *   slot_idx [B] int32 device, nullable (= identity); slots of one call must be distinct.
+ *   num_slots  rows of conv_state and S (>= B when slot_idx is NULL).  A sequence whose slot lies
+ *     outside [0, num_slots) is skipped on the device: no state access, its out rows are not
+ *     written, and dev_status (int32, nullable) is set to GDN_ERR_INVALID_ARG.
  *   out [B, Hv, d].
  * One pass over the state: it is read once and written once.
  */
 int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
                     const float* beta, const float* g, const void* z, const void* norm_w,
-                    void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
-                    void* out, void* stream);
+                    void* conv_state, float* S, const int32_t* slot_idx, int32_t num_slots,
+                    int32_t batch, void* out, int32_t* dev_status, void* stream);
 
 /*
  * gdn_block_prefill -- the token mixer of a Gated DeltaNet decoder layer: input projections,
@@ -237,9 +274,10 @@ int gdn_decode_step(const gdn_dims* dims, gdn_dtype dtype, const void* x, const 
  *   a), all row-major (input x output); a_log, dt_bias [Hv] fp32; w_out [Hv d, H]; y [T, H].
  *   conv_w, norm_w, cu_seqlens, S0, SN, conv0, convN, dev_status: as gdn_chunk_prefill.
  *   workspace: at least gdn_block_prefill_workspace_size() bytes, 256-byte aligned.
- * The four projections are plain GEMMs (fp32 accumulation) and run in cuBLAS, loaded on the
- * first call (GDN_ERR_UNSUPPORTED when it cannot be loaded); cuBLAS creates one handle per
- * device and host thread on that first call (not inside a stream capture).
+ * The four projections run on the library's own tcgen05 GEMM (bf16 operands, fp32
+ * accumulation in TMEM): the [b | a] projection computes the gates in its epilogue (beta and g
+ * never leave the GEMM as b and a); the q|k|v, z and output projections round to bf16.
+ * GDN_ERR_UNSUPPORTED when 2 Hv > 64 (the gate GEMM's tile width).
  */
 size_t gdn_block_prefill_workspace_size(const gdn_dims* dims, int32_t hidden, int32_t num_seqs,
                                         int32_t num_tokens);
@@ -258,7 +296,8 @@ int gdn_block_prefill(const gdn_dims* dims, int32_t hidden, const void* h, const
  * 0..k-1 in order (the same fp32 arithmetic per token): outputs of every token, conv and
  * recurrent state after token k-1.  The state rows are read and written once for all k tokens.
  *   x [B, k, Cc], beta/g [B, k, Hv] fp32, z [B, k, Hv, d] nullable, out [B, k, Hv, d];
- *   conv_w, norm_w, conv_state, S (fp32), slot_idx as gdn_decode_step; 0 <= k <= 8
+ *   conv_w, norm_w, conv_state, S (fp32), slot_idx, num_slots, dev_status as gdn_decode_step;
+ *   0 <= k <= 8
  *   (GDN_ERR_UNSUPPORTED above 8; k = 0 or B = 0 launch nothing).
  *   snapshots [B, k, Hv, d, d] fp32, nullable: the recurrent state after each token, indexed by
  *     position in the call (not by slot), for a caller that accepts only the first m tokens
@@ -267,8 +306,9 @@ int gdn_block_prefill(const gdn_dims* dims, int32_t hidden, const void* h, const
  */
 int gdn_decode_multi(const gdn_dims* dims, gdn_dtype dtype, const void* x, const void* conv_w,
                      const float* beta, const float* g, const void* z, const void* norm_w,
-                     void* conv_state, float* S, const int32_t* slot_idx, int32_t batch,
-                     int32_t tokens, void* out, float* snapshots, void* stream);
+                     void* conv_state, float* S, const int32_t* slot_idx, int32_t num_slots,
+                     int32_t batch, int32_t tokens, void* out, float* snapshots,
+                     int32_t* dev_status, void* stream);
 
 /*
  * gdn_decode_step_bf16_state -- gdn_decode_step with the recurrent state stored in bf16.
@@ -282,7 +322,8 @@ int gdn_decode_multi(const gdn_dims* dims, gdn_dtype dtype, const void* x, const
 int gdn_decode_step_bf16_state(const gdn_dims* dims, gdn_dtype dtype, const void* x,
                                const void* conv_w, const float* beta, const float* g,
                                const void* z, const void* norm_w, void* conv_state, void* S,
-                               const int32_t* slot_idx, int32_t batch, void* out, void* stream);
+                               const int32_t* slot_idx, int32_t num_slots, int32_t batch,
+                               void* out, int32_t* dev_status, void* stream);
 
 /*
  * gdn_chunk_prefill_static_ws -- gdn_chunk_prefill for callers that cannot allocate device
@@ -299,6 +340,9 @@ int gdn_decode_step_bf16_state(const gdn_dims* dims, gdn_dtype dtype, const void
  *     1,791 tokens, or fewer tokens spread over more sequences).
  *   - The first call on each device looks the array's device address up (cudaGetSymbolAddress,
  *     with that device current) and caches it; make that first call before any stream capture.
+ *     The cached address belongs to the device context of that first call: do not call this
+ *     entry point again after a cudaDeviceReset (or any reset of the primary context) in the
+ *     same process.
  *   - All calls share the one array and it keeps the previous call's contents (nothing in it
  *     needs to start at zero).  Calls that overlap on the GPU (different streams, or different
  *     host threads on one device) race on it and must be serialised by the caller.
@@ -317,6 +361,9 @@ int gdn_chunk_prefill_static_ws(const gdn_dims* dims, gdn_dtype dtype, const voi
  * attached to the calling host thread, every kernel the library launches from that thread is
  * bracketed by two CUDA events recorded on the launch stream.  After synchronising, read the
  * per-launch device times.  A trace holds up to 4096 launches; further ones are not recorded.
+ * Launches made while the stream is being captured into a CUDA graph get their two events as
+ * event-record nodes of that graph: each replay records them again, so after a replay (and a
+ * synchronisation) gdn_trace_get returns the times of that replay's launches.
  */
 typedef struct gdn_trace gdn_trace;
 int gdn_trace_create(gdn_trace** out);         /* host object, owned by the caller */
@@ -329,6 +376,37 @@ int gdn_trace_get(gdn_trace* trace, int32_t i, const char** name, float* ms);
 /* Start and end of launch i in ms after the start of launch 0 of the same trace (launches on
  * different streams overlap on this common time line).  Synchronises on both end events. */
 int gdn_trace_span(gdn_trace* trace, int32_t i, float* start_ms, float* end_ms);
+
+/*
+ * gdn_debug_set -- debug and test controls, not needed for normal use.  The settings apply to
+ * the calls the calling host thread makes afterwards (the library copies *opts); NULL restores
+ * the defaults (all fields zero).  Workspace sizes depend on segment_chunks: query them with
+ * the same settings as the call.
+ *   wait_limit_us  bound of every device wait of the prefill kernels, in microseconds (0: 2 s).
+ *                  A wait that runs out writes GDN_ERR_TIMEOUT to dev_status, lets the copies
+ *                  and products it has in flight land, frees its TMEM and ends its CTA.
+ *   segment_chunks length in 128-token chunks of the segments the bf16 prefill pipelines over
+ *                  its streams (0: the library's choice, 64 from 512 chunks on, else one).
+ *   chain_split    d_v blocks per state in the sequential chain kernel: 1, 2 or 4 (0: the
+ *                  library's choice).
+ *   fault          GDN_FAULT_NONE, or GDN_FAULT_SKIP_CHAIN_LOAD: the first CTA of the chain
+ *                  kernel does not issue the load of chunk fault_chunk's W tile (chunk index of
+ *                  the call's table, sequence by sequence), so its bounded wait for that tile
+ *                  runs out.  Used to test the timeout path with no GPU fault: the call then
+ *                  reports GDN_ERR_TIMEOUT in dev_status and its outputs are undefined.
+ *   fault_chunk    see fault.
+ * Returns GDN_OK, or GDN_ERR_INVALID_ARG for an out-of-range field (settings unchanged).
+ */
+#define GDN_FAULT_NONE 0
+#define GDN_FAULT_SKIP_CHAIN_LOAD 1
+typedef struct gdn_debug_options {
+  uint32_t wait_limit_us;
+  int32_t segment_chunks;
+  int32_t chain_split;
+  int32_t fault;
+  int32_t fault_chunk;
+} gdn_debug_options;
+int gdn_debug_set(const gdn_debug_options* opts);
 
 /*
  * gdn_debug_wait_probe -- test aid for the bounded device waits: launches one CTA that waits

@@ -66,9 +66,9 @@ def _load():
             lib.orc_conv1d_silu.argtypes = [ip, vp, vp, vp, ip, ip, ip, ip, vp, vp, vp]
             lib.orc_gated_rmsnorm.argtypes = [ip, vp, vp, vp, ctypes.c_double, ip, ip, vp]
             lib.orc_prefill.argtypes = [ctypes.POINTER(_Dims), ip, vp, vp, vp, vp, vp, vp, vp, ip,
-                                        ip, vp, vp, ctypes.c_longlong, vp, vp, vp, ip]
+                                        ip, vp, vp, ctypes.c_longlong, vp, vp, vp, vp, vp, ip]
             lib.orc_decode_step.argtypes = [ctypes.POINTER(_Dims), ip, vp, vp, vp, vp, vp, vp, vp,
-                                            vp, vp, ip, vp, ip]
+                                            vp, vp, ip, vp, vp, vp, ip]
             for f in (lib.orc_conv1d_silu, lib.orc_gated_rmsnorm, lib.orc_prefill,
                       lib.orc_decode_step):
                 f.restype = ctypes.c_int
@@ -185,11 +185,13 @@ def gated_rmsnorm(o, z, w, eps):
 
 
 def prefill(dims: Dims, x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None, S0=None,
-            conv0=None, out_t0: int = 0, want_state: bool = True, nthreads: int | None = None):
+            conv0=None, out_t0: int = 0, want_state: bool = True, nthreads: int | None = None,
+            with_scales: bool = False):
     """Full layer over packed sequences (see gdn_oracle.c for the definition).
 
     Returns (out [T - out_t0, Hv, d], SN [N, Hv, d, d] or None, convN [N, K-1, Cc] or None),
-    all fp64 numpy arrays.
+    all fp64 numpy arrays.  With ``with_scales`` two more arrays follow: the element scales of
+    out and the state magnitudes M (the error scales of the gdn_oracle.c header).
     """
     keep = []
     cx, px = _act(x, keep)
@@ -204,16 +206,18 @@ def prefill(dims: Dims, x, beta, g, cu_seqlens, conv_w=None, z=None, norm_w=None
     out = np.zeros((T - out_t0, Hv, d), np.float64)
     SN = np.zeros((N, Hv, d, d), np.float64) if want_state else None
     convN = np.zeros((N, K - 1, dims.channels), np.float64) if want_state else None
+    out_scale = np.zeros_like(out) if with_scales else None
+    SN_scale = np.zeros((N, Hv, d, d), np.float64) if with_scales else None
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p) if a is not None else None  # noqa: E731
     c_dims = dims._c()
     rc = _load().orc_prefill(
         ctypes.byref(c_dims), code, px, pw, _f32(beta, keep), _f32(g, keep), pz, pn,
-        _i32(cu_seqlens, keep), N, T, _f32(S0, keep), pc, int(out_t0),
-        out.ctypes.data_as(ctypes.c_void_p),
-        SN.ctypes.data_as(ctypes.c_void_p) if SN is not None else None,
-        convN.ctypes.data_as(ctypes.c_void_p) if convN is not None else None,
-        int(nthreads or default_threads()))
+        _i32(cu_seqlens, keep), N, T, _f32(S0, keep), pc, int(out_t0), ptr(out), ptr(SN),
+        ptr(convN), ptr(out_scale), ptr(SN_scale), int(nthreads or default_threads()))
     if rc != 0:
         raise ValueError(f"orc_prefill failed: {rc}")
+    if with_scales:
+        return out, SN, convN, out_scale, SN_scale
     return out, SN, convN
 
 
@@ -232,11 +236,13 @@ def block_gates(ba, a_log, dt_bias):
 
 
 def block_prefill(dims: Dims, h, w_qkv, w_z, w_ba, a_log, dt_bias, w_out, cu_seqlens,
-                  conv_w=None, norm_w=None, S0=None, conv0=None, nthreads: int | None = None):
+                  conv_w=None, norm_w=None, S0=None, conv0=None, nthreads: int | None = None,
+                  with_scales: bool = False):
     """The token mixer of a decoder layer in fp64: x = h W_qkv, z = h W_z, [b | a] = h W_ba,
     the gates of block_gates, the layer (prefill) and y = o W_out.  Weights are [in, out].
     Returns (y [T, H], SN, convN) as fp64 numpy; the gates enter the layer rounded to fp32
-    (its beta and g are fp32 inputs)."""
+    (its beta and g are fp32 inputs).  With ``with_scales`` the element scales of y (the
+    layer's output scales carried through |W_out|) and the state magnitudes follow."""
     f64 = lambda t: np.asarray(t.detach().cpu().double().numpy() if isinstance(t, torch.Tensor)
                                else t, np.float64)
     hh = f64(h)
@@ -245,20 +251,30 @@ def block_prefill(dims: Dims, h, w_qkv, w_z, w_ba, a_log, dt_bias, w_out, cu_seq
     z = hh @ f64(w_z)
     beta, g = block_gates(hh @ f64(w_ba), f64(a_log), f64(dt_bias))
     to64 = lambda t: None if t is None else torch.from_numpy(f64(t))
-    o, SN, convN = prefill(dims, torch.from_numpy(x), beta.astype(np.float32),
-                           g.astype(np.float32), cu_seqlens, conv_w=to64(conv_w),
-                           z=torch.from_numpy(z), norm_w=to64(norm_w), S0=S0, conv0=to64(conv0),
-                           nthreads=nthreads)
-    y = o.reshape(T, dims.num_v_heads * dims.head_dim) @ f64(w_out)
+    res = prefill(dims, torch.from_numpy(x), beta.astype(np.float32),
+                  g.astype(np.float32), cu_seqlens, conv_w=to64(conv_w),
+                  z=torch.from_numpy(z), norm_w=to64(norm_w), S0=S0, conv0=to64(conv0),
+                  nthreads=nthreads, with_scales=with_scales)
+    o, SN, convN = res[:3]
+    HD = dims.num_v_heads * dims.head_dim
+    y = o.reshape(T, HD) @ f64(w_out)
+    if with_scales:
+        y_scale = res[3].reshape(T, HD) @ np.abs(f64(w_out))
+        return y, SN, convN, y_scale, res[4]
     return y, SN, convN
 
 
 def decode_step(dims: Dims, x, beta, g, conv_state, S, conv_w=None, z=None, norm_w=None,
-                slot_idx=None, nthreads: int | None = None):
+                slot_idx=None, nthreads: int | None = None, M=None):
     """One decode token per sequence; conv_state [slots, K-1, Cc] and S [slots, Hv, d, d] are
-    fp64 numpy arrays updated in place.  Returns out [B, Hv, d] fp64."""
+    fp64 numpy arrays updated in place.  Returns out [B, Hv, d] fp64.
+
+    With ``M`` (fp64 like S; start it as |S|) the state magnitude of the gdn_oracle.c header is
+    carried in place as well, and the call returns (out, element scales of out)."""
     assert conv_state.dtype == np.float64 and conv_state.flags.c_contiguous
     assert S.dtype == np.float64 and S.flags.c_contiguous
+    if M is not None:
+        assert M.dtype == np.float64 and M.flags.c_contiguous and M.shape == S.shape
     keep = []
     cx, px = _act(x, keep)
     cw, pw = _act(conv_w, keep)
@@ -267,12 +283,15 @@ def decode_step(dims: Dims, x, beta, g, conv_state, S, conv_w=None, z=None, norm
     code = _same_dtype([cx, cw, cz, cn])
     B = x.shape[0]
     out = np.zeros((B, dims.num_v_heads, dims.head_dim), np.float64)
+    out_scale = np.zeros_like(out) if M is not None else None
     c_dims = dims._c()
     rc = _load().orc_decode_step(
         ctypes.byref(c_dims), code, px, pw, _f32(beta, keep), _f32(g, keep), pz, pn,
         conv_state.ctypes.data_as(ctypes.c_void_p), S.ctypes.data_as(ctypes.c_void_p),
         _i32(slot_idx, keep), B, out.ctypes.data_as(ctypes.c_void_p),
+        M.ctypes.data_as(ctypes.c_void_p) if M is not None else None,
+        out_scale.ctypes.data_as(ctypes.c_void_p) if out_scale is not None else None,
         int(nthreads or default_threads()))
     if rc != 0:
         raise ValueError(f"orc_decode_step failed: {rc}")
-    return out
+    return out if M is None else (out, out_scale)

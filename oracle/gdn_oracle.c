@@ -35,6 +35,25 @@
  *   - gated norm: y = o / sqrt(mean(o^2) + norm_eps) * w * silu(z), per (token, value head),
  *     w is the effective weight (a zero-centred caller passes 1 + w).
  *
+ * Error scales (optional outputs, used by the tests to set element-wise tolerances).  Every
+ * quantity gets a magnitude: the same computation with every term replaced by its absolute
+ * value, so that nothing cancels.  The conv output y = silu(sum_i w_i x_i) gets
+ * ym = 1.1 sum_i |w_i| |x_i| (1.1 bounds the slope of SiLU; ym >= |y|), or |x| with the conv
+ * off; q and k get ym / |y~| after the L2 norm, v keeps ym.  Writing km, qm, vm for those, the
+ * state runs
+ *        M_t = alpha_t M_{t-1} + beta_t (vm_t + alpha_t |S_{t-1}| km_t) km_t^T,   M_0 = |S_0|
+ * (|.| element-wise; the kv_mem term uses the actual state, so M stays finite like S).  By the
+ * triangle inequality M_t >= |S_t| element-wise.  The scale of output element o_t[v] is
+ * c_t[v] = sum_k M_t[v][k] qm_t[k] (>= |o_t[v]|): the size of the terms the dot product adds
+ * up.  For the gated RMSNorm y = o r w silu(z), r = 1 / sqrt(m + eps), m = mean(o^2), a change
+ * of each o[u] by c[u] moves y[v] by at most (to first order)
+ *        s[v] = |w[v] silu(z[v])| r (c[v] + |o[v]| sum_u |o[u]| c[u] / (d (m + eps))),
+ * which is the scale reported for normalised outputs.  Rounding an input or an intermediate of
+ * the recurrence by a relative epsilon changes an element by a multiple of epsilon times its
+ * scale, not of epsilon times its value: elements that are small sums of large terms (a query
+ * nearly orthogonal to the state, a row whose RMSNorm divides by a small norm) carry large
+ * scales.  The scales are outputs only; they change nothing in out, SN or convN.
+ *
  * All inputs are converted exactly to fp64 (bf16 and fp32 values are exactly representable).
  * Independent (sequence, value head) units run on host threads; within a unit the arithmetic
  * is the sequential per-token recurrence above, in the order written.
@@ -153,6 +172,9 @@ typedef struct {
     long long out_t0;
     double *out;           /* [T - out_t0][Hv][d] */
     double *SN;            /* [N][Hv][d][d] or NULL */
+    double *out_scale;     /* [T - out_t0][Hv][d] or NULL: element scales of out */
+    double *SN_scale;      /* [N][Hv][d][d] or NULL: the magnitude M at the end */
+    double *Md;            /* decode: [slots][Hv][d][d] magnitude, in/out, or NULL */
     const int32_t *slot;   /* decode: state slot of each sequence, or NULL */
     int next;              /* shared work counter */
     pthread_mutex_t mu;
@@ -182,12 +204,24 @@ static void run_unit(unit_job *jb, int unit) {
     double *v = (double *)malloc(sizeof(double) * d), *o = (double *)malloc(sizeof(double) * d);
     double *u = (double *)malloc(sizeof(double) * d), *kv = (double *)malloc(sizeof(double) * d);
     double *yq = (double *)malloc(sizeof(double) * 3 * d);
+    /* error scales: magnitudes of the conv outputs and of q, k, v, magnitude M of the state,
+       |S| km and the output scales c */
+    const int scales = jb->out_scale || jb->SN_scale || jb->Md;
+    double *ym = scales ? (double *)malloc(sizeof(double) * 3 * d) : NULL;
+    double *M = scales ? (double *)calloc((size_t)d * d, sizeof(double)) : NULL;
+    double *ak = scales ? (double *)malloc(sizeof(double) * d) : NULL;
+    double *cs = scales ? (double *)malloc(sizeof(double) * d) : NULL;
 
     const size_t sbase = ((size_t)slot * Hv + h) * (size_t)d * d;
     if (jb->S0)
         for (size_t i = 0; i < (size_t)d * d; ++i) S[i] = (double)jb->S0[sbase + i];
     if (jb->S0d)
         for (size_t i = 0; i < (size_t)d * d; ++i) S[i] = jb->S0d[sbase + i];
+    if (scales) {
+        for (size_t i = 0; i < (size_t)d * d; ++i) M[i] = fabs(S[i]);
+        if (jb->Md)
+            for (size_t i = 0; i < (size_t)d * d; ++i) M[i] = jb->Md[sbase + i];
+    }
     /* conv history for the three channel groups, oldest row first */
     for (int j = 0; j < K - 1; ++j)
         for (int gi = 0; gi < 3; ++gi)
@@ -206,18 +240,26 @@ static void run_unit(unit_job *jb, int unit) {
             for (int c = 0; c < d; ++c) {
                 double xc = ld_any(jb->x, jb->dtype, (size_t)t * Cc + chans[gi] + c);
                 double yv;
+                double mag = fabs(xc);
                 if (jb->conv_w) {
                     const size_t wrow = (size_t)(chans[gi] + c) * K;
-                    double acc = 0.0;
-                    for (int i = 0; i < K - 1; ++i)
-                        acc += ld_any(jb->conv_w, jb->dtype, wrow + i) *
-                               hist[((size_t)i * 3 + gi) * d + c];
-                    acc += ld_any(jb->conv_w, jb->dtype, wrow + K - 1) * xc;
+                    double acc = 0.0, am = 0.0;
+                    for (int i = 0; i < K - 1; ++i) {
+                        const double wi = ld_any(jb->conv_w, jb->dtype, wrow + i);
+                        const double hi = hist[((size_t)i * 3 + gi) * d + c];
+                        acc += wi * hi;
+                        am += fabs(wi) * fabs(hi);
+                    }
+                    const double wl = ld_any(jb->conv_w, jb->dtype, wrow + K - 1);
+                    acc += wl * xc;
+                    am += fabs(wl) * fabs(xc);
                     yv = silu(acc);
+                    mag = 1.1 * am;
                 } else {
                     yv = xc;
                 }
                 yq[gi * d + c] = yv;
+                if (scales) ym[gi * d + c] = mag;
             }
         for (int j = 0; j + 1 < K - 1; ++j)
             for (int i = 0; i < 3 * d; ++i) hist[(size_t)j * 3 * d + i] = hist[(size_t)(j + 1) * 3 * d + i];
@@ -239,11 +281,23 @@ static void run_unit(unit_job *jb, int unit) {
             k[c] = yq[d + c] * rk;
             v[c] = yq[2 * d + c];
         }
+        if (scales)  /* magnitudes of q, k, v in place of the conv magnitudes */
+            for (int c = 0; c < d; ++c) {
+                ym[c] *= rq;
+                ym[d + c] *= rk;
+            }
 
         /* 3. gated delta rule, one token */
         const double alpha = exp((double)jb->g[(size_t)t * Hv + h]);
         const double beta = (double)jb->beta[(size_t)t * Hv + h];
         for (size_t i = 0; i < (size_t)d * d; ++i) S[i] *= alpha;       /* S <- alpha S      */
+        if (scales) {                                   /* |alpha S_{t-1}| km, before the write */
+            for (int r = 0; r < d; ++r) {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c) acc += fabs(S[(size_t)r * d + c]) * ym[d + c];
+                ak[r] = acc;
+            }
+        }
         for (int r = 0; r < d; ++r) {                                      /* kv_mem = S k      */
             double acc = 0.0;
             for (int c = 0; c < d; ++c) acc += S[(size_t)r * d + c] * k[c];
@@ -257,25 +311,49 @@ static void run_unit(unit_job *jb, int unit) {
             for (int c = 0; c < d; ++c) acc += S[(size_t)r * d + c] * q[c];
             o[r] = acc;
         }
+        if (scales) {                         /* M <- alpha M + beta (vm + |alpha S| km) km^T */
+            for (int r = 0; r < d; ++r) {
+                const double a = beta * (ym[2 * d + r] + ak[r]);
+                for (int c = 0; c < d; ++c)
+                    M[(size_t)r * d + c] = alpha * M[(size_t)r * d + c] + a * ym[d + c];
+            }
+            for (int r = 0; r < d; ++r) {                              /* c = M qm           */
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c) acc += M[(size_t)r * d + c] * ym[c];
+                cs[r] = acc;
+            }
+        }
 
         /* 4. z-gated RMSNorm */
         if (jb->z) {
-            double ss = 0.0;
-            for (int r = 0; r < d; ++r) ss += o[r] * o[r];
-            double inv = 1.0 / sqrt(ss / d + dm->norm_eps);
+            double ss = 0.0, oc = 0.0;
+            for (int r = 0; r < d; ++r) {
+                ss += o[r] * o[r];
+                if (scales) oc += fabs(o[r]) * cs[r];
+            }
+            const double m_eps = ss / d + dm->norm_eps;
+            double inv = 1.0 / sqrt(m_eps);
             for (int r = 0; r < d; ++r) {
                 double wr = jb->norm_w ? ld_any(jb->norm_w, jb->dtype, (size_t)r) : 1.0;
                 double zr = ld_any(jb->z, jb->dtype, ((size_t)t * Hv + h) * d + r);
+                if (scales)   /* first-order change of the normalised element (header) */
+                    cs[r] = fabs(wr * silu(zr)) * inv * (cs[r] + fabs(o[r]) * oc / (d * m_eps));
                 o[r] = o[r] * inv * wr * silu(zr);
             }
         }
         if ((long long)t >= jb->out_t0) {
             double *dst = jb->out + (((size_t)(t - jb->out_t0)) * Hv + h) * d;
             memcpy(dst, o, sizeof(double) * d);
+            if (jb->out_scale)
+                memcpy(jb->out_scale + (((size_t)(t - jb->out_t0)) * Hv + h) * d, cs,
+                       sizeof(double) * d);
         }
     }
     if (jb->SN) memcpy(jb->SN + sbase, S, sizeof(double) * (size_t)d * d);
+    if (jb->SN_scale) memcpy(jb->SN_scale + sbase, M, sizeof(double) * (size_t)d * d);
+    if (jb->Md) memcpy(jb->Md + sbase, M, sizeof(double) * (size_t)d * d);
     free(S); free(hist); free(q); free(k); free(v); free(o); free(u); free(kv); free(yq);
+    free(M); free(ak); free(cs); free(ym);
 }
 
 static void *worker(void *arg) {
@@ -336,11 +414,13 @@ static void conv_final(const orc_dims *dm, int dtype, const void *x, const int32
 /*   cu_seqlens [N+1], S0 [N][Hv][d][d] fp32 or NULL, conv0 [N][K-1][Cc] dtype or NULL.          */
 /*   out [T-out_t0][Hv][d] fp64: outputs of tokens t >= out_t0 only.                            */
 /*   SN [N][Hv][d][d] fp64 or NULL; convN [N][K-1][Cc] fp64 or NULL.                            */
+/*   out_scale [T-out_t0][Hv][d], SN_scale [N][Hv][d][d] fp64 or NULL: the error scales of the   */
+/*   header (element scales of out, magnitude M of the final states).                          */
 /* ------------------------------------------------------------------------------------------ */
 int orc_prefill(const orc_dims *dm, int dtype, const void *x, const void *conv_w, const float *beta,
                 const float *g, const void *z, const void *norm_w, const int32_t *cu_seqlens, int N,
                 int T, const float *S0, const void *conv0, long long out_t0, double *out, double *SN,
-                double *convN, int nthreads) {
+                double *convN, double *out_scale, double *SN_scale, int nthreads) {
     if (!dims_ok(dm) || N < 0 || T < 0 || out_t0 < 0 || out_t0 > T) return -1;
     if (N > 0 && (cu_seqlens[0] != 0 || cu_seqlens[N] != T)) return -1;
     for (int n = 0; n < N; ++n)
@@ -350,6 +430,7 @@ int orc_prefill(const orc_dims *dm, int dtype, const void *x, const void *conv_w
     jb.dm = dm; jb.dtype = dtype; jb.x = x; jb.conv_w = conv_w; jb.z = z; jb.norm_w = norm_w;
     jb.beta = beta; jb.g = g; jb.cu_seqlens = cu_seqlens; jb.N = N; jb.T = T; jb.S0 = S0;
     jb.conv0 = conv0; jb.out_t0 = out_t0; jb.out = out; jb.SN = SN;
+    jb.out_scale = out_scale; jb.SN_scale = SN_scale;
     run_units(&jb, nthreads);
     if (convN) conv_final(dm, dtype, x, cu_seqlens, N, conv0, NULL, NULL, convN);
     return 0;
@@ -360,11 +441,13 @@ int orc_prefill(const orc_dims *dm, int dtype, const void *x, const void *conv_w
 /*   x [B][Cc] dtype, beta/g [B][Hv] fp32, z [B][Hv][d] dtype or NULL.                           */
 /*   conv_state [slots][K-1][Cc] fp64 in/out, S [slots][Hv][d][d] fp64 in/out,                   */
 /*   slot_idx [B] or NULL (sequence b uses slot b).  out [B][Hv][d] fp64.                         */
+/*   M [slots][Hv][d][d] fp64 in/out or NULL: the state magnitude of the header, carried across  */
+/*   steps like S (start from |S|); out_scale [B][Hv][d] fp64 (used only with M).                */
 /* ------------------------------------------------------------------------------------------ */
 int orc_decode_step(const orc_dims *dm, int dtype, const void *x, const void *conv_w,
                     const float *beta, const float *g, const void *z, const void *norm_w,
                     double *conv_state, double *S, const int32_t *slot_idx, int B, double *out,
-                    int nthreads) {
+                    double *M, double *out_scale, int nthreads) {
     if (!dims_ok(dm) || B < 0) return -1;
     const int K = dm->conv_kernel, Cc = 2 * dm->num_k_heads * dm->head_dim + dm->num_v_heads * dm->head_dim;
     int32_t *cu = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B + 1));
@@ -375,6 +458,7 @@ int orc_decode_step(const orc_dims *dm, int dtype, const void *x, const void *co
     jb.dm = dm; jb.dtype = dtype; jb.x = x; jb.conv_w = conv_w; jb.z = z; jb.norm_w = norm_w;
     jb.beta = beta; jb.g = g; jb.cu_seqlens = cu; jb.N = B; jb.T = B; jb.S0d = S;
     jb.conv0d = conv_state; jb.out_t0 = 0; jb.out = out; jb.SN = S; jb.slot = slot_idx;
+    jb.Md = M; jb.out_scale = M ? out_scale : NULL;
     run_units(&jb, nthreads);
     /* new conv history of each slot: drop the oldest row, append this token's input
        (all units have finished reading the old history at this point) */

@@ -1,5 +1,8 @@
 """Helpers shared by the GPU parity tests: run the CUDA path through the binding and the
 fp64 oracle on the same seeded CPU tensors, and compare."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -7,15 +10,25 @@ import oracle
 import gated_deltanet_layer_02_b200 as gdn
 from gated_deltanet_layer_02_b200 import build as gdn_build
 
-#: Tolerances.  fp32 activations: max-abs error <= 1e-4.  bf16 activations: relative RMS
-#: error ||gpu - oracle||_2 / ||oracle||_2 <= 2e-2 per tensor (outputs and final states
-#: separately).  The max-abs / rms reading is not used for bf16: rounding the exact result to
-#: bf16 already exceeds it on heavy-tailed normalised outputs (tests/test_tolerance_reading.py).
-#: A guard against localised errors that an RMS can hide: at most 0.2% of the elements may be
-#: off by more than 0.1 * rms(oracle).
+#: Tolerances, all element-wise.
+#:  * fp32 activations: max |gpu - oracle| <= 1e-4 on outputs and states.
+#:  * bf16 activations: every element within 2e-2 of its error scale, plus one bf16 rounding
+#:    of the value for bf16 tensors:   |gpu - oracle| <= 2e-2 * scale + 2^-8 * |oracle|
+#:    (2^-8 only for bf16 results; fp32 recurrent states get 2e-2 * scale alone).  The scale of
+#:    an element is the oracle's own measure of the terms that form it (gdn_oracle.c header:
+#:    the magnitude M of the state recurrence, M |q| for an output, carried through the gated
+#:    RMSNorm), so a small element made of large cancelling terms gets the tolerance of those
+#:    terms.  Checks without such a scale (conv, standalone RMSNorm, conv history) use the
+#:    tensor's RMS.  On top, the relative RMS error of the tensor must stay <= 2e-2.
+#:    Why not 2e-2 * rms(oracle) + 2^-8 |oracle|: one bf16 rounding of the normalised q and k
+#:    (the tensor-core operands) already moves the exact output by more than that on some
+#:    elements (tests/test_tolerance_reading.py), so that bound measures the conditioning of
+#:    the problem rather than the implementation.
+#: Each check's figures go to the test output and, with GDN_PARITY_LOG=<file>, to a JSON-lines
+#: log.
 TOL_F32_ABS = 1e-4
-TOL_BF16_REL_RMS = 2e-2
-GUARD_FRAC, GUARD_LEVEL = 2e-3, 0.1
+TOL_BF16_REL = 2e-2
+BF16_ULP_REL = 2.0 ** -8
 
 _built = False
 
@@ -49,10 +62,21 @@ def gpu_prefill(w, inp, dev_status=None, **kw):
     return out, SN, convN
 
 
+class Ref(tuple):
+    """(out, SN, convN) of the oracle, unpacking like a 3-tuple, with the error scales of the
+    out and SN elements as attributes (out_scale, SN_scale)."""
+
+    def __new__(cls, out, SN, convN, out_scale=None, SN_scale=None):
+        r = super().__new__(cls, (out, SN, convN))
+        r.out_scale, r.SN_scale = out_scale, SN_scale
+        return r
+
+
 def oracle_prefill(w, inp, out_t0=0):
-    return oracle.prefill(oracle_dims_of(w), inp["x"], inp["beta"], inp["g"], inp["cu_seqlens"],
-                          conv_w=inp["conv_w"], z=inp["z"], norm_w=inp["norm_w"], S0=inp["S0"],
-                          conv0=inp["conv0"], out_t0=out_t0)
+    r = oracle.prefill(oracle_dims_of(w), inp["x"], inp["beta"], inp["g"], inp["cu_seqlens"],
+                       conv_w=inp["conv_w"], z=inp["z"], norm_w=inp["norm_w"], S0=inp["S0"],
+                       conv0=inp["conv0"], out_t0=out_t0, with_scales=True)
+    return Ref(*r)
 
 
 def np64(t):
@@ -71,26 +95,48 @@ def max_abs_over_rms(got, ref):
     return float(np.max(np.abs(got - ref)) / max(rms, 1e-30))
 
 
-def outlier_fraction(got, ref, level=GUARD_LEVEL):
-    got, ref = np64(got), np64(ref)
-    rms = np.sqrt(np.mean(ref ** 2))
-    return float(np.mean(np.abs(got - ref) > level * rms))
-
-
 def max_abs(got, ref):
     return float(np.max(np.abs(np64(got) - np64(ref)))) if np64(ref).size else 0.0
 
 
-def assert_close(got, ref, dtype, what):
-    """Parity bar of the path; returns the error figure it was judged on."""
-    assert np.all(np.isfinite(np64(got))), f"{what}: non-finite values"
+def _log(rec):
+    path = os.environ.get("GDN_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(rec) + "\n")
+    print("parity " + json.dumps(rec))
+
+
+def assert_close(got, ref, dtype, what, scale=None, f32_scale=1.0):
+    """Parity bar of the path (element-wise); returns the figure it was judged on.
+
+    dtype is the activation dtype of the run; ``scale`` the oracle's error scale of every
+    element (None: the tensor's RMS).  ``f32_scale`` multiplies the fp32 absolute bound for
+    inputs deliberately drawn at that multiple of the workload's magnitude."""
+    g, r = np64(got), np64(ref)
+    assert g.shape == r.shape, f"{what}: shape {g.shape} != {r.shape}"
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values"
+    err = np.abs(g - r)
+    rms = float(np.sqrt(np.mean(r ** 2))) if r.size else 0.0
+    rec = {"what": what, "n": int(r.size), "rms": rms,
+           "max_abs": float(err.max()) if r.size else 0.0,
+           "rel_rms": rel_rms(got, ref) if r.size else 0.0,
+           "max_abs_over_rms": float(err.max() / max(rms, 1e-30)) if r.size else 0.0}
     if dtype == torch.float32:
-        err = max_abs(got, ref)
-        assert err <= TOL_F32_ABS, f"{what}: max-abs {err:.3g} > {TOL_F32_ABS}"
-        return err
-    err = rel_rms(got, ref)
-    frac = outlier_fraction(got, ref)
-    info = f"rel-rms {err:.3g}, max-abs/rms {max_abs_over_rms(got, ref):.3g}, outliers {frac:.2g}"
-    assert err <= TOL_BF16_REL_RMS, f"{what}: {info}"
-    assert frac <= GUARD_FRAC, f"{what}: {info}"
-    return err
+        rec["kind"], rec["bound"] = "f32 max-abs", TOL_F32_ABS * f32_scale
+        _log(rec)
+        assert rec["max_abs"] <= TOL_F32_ABS * f32_scale, f"{what}: {rec}"
+        return rec["max_abs"]
+    is_bf16_tensor = isinstance(got, torch.Tensor) and got.dtype == torch.bfloat16
+    s = rms if scale is None else np64(scale)
+    if scale is not None:
+        assert np.shape(s) == r.shape, f"{what}: scale shape {np.shape(s)} != {r.shape}"
+    bound = TOL_BF16_REL * s + (BF16_ULP_REL * np.abs(r) if is_bf16_tensor else 0.0)
+    ratio = float(np.max(err / np.maximum(bound, 1e-300))) if r.size else 0.0
+    rec["kind"] = ("bf16 " if is_bf16_tensor else "fp32 ") + ("element scale" if scale is not None
+                                                               else "tensor rms")
+    rec["worst_over_bound"] = ratio
+    _log(rec)
+    assert rec["rel_rms"] <= TOL_BF16_REL, f"{what}: {rec}"
+    assert ratio <= 1.0, f"{what}: {rec}"
+    return ratio

@@ -34,7 +34,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.gdn_abi_version() == 1
+    assert L.gdn_abi_version() == 2
     for code, text in [(0, "ok"), (-1, "invalid argument"), (-2, "unsupported shape or dtype"),
                        (-3, "CUDA error"), (-4, "device wait timed out"),
                        (-5, "workspace too small"), (7, "unknown status")]:
@@ -101,21 +101,29 @@ def test_other_entry_points_reject_bad_arguments(L):
     assert L.gdn_gated_rmsnorm(1, A, None, None, 1e-6, 4, 128, A, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_gated_rmsnorm(1, A, A, None, -1.0, 4, 128, A, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_gated_rmsnorm(3, A, A, None, 1e-6, 4, 128, A, None) == gdn.GDN_ERR_UNSUPPORTED
-    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, A, None, -1, A, None) == gdn.GDN_ERR_INVALID_ARG
-    assert L.gdn_decode_step(d, 1, A, None, A, A, None, None, A, A, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
-    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, MIS, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
+    # (dims, dtype, x, conv_w, beta, g, z, norm_w, conv_state, S, slot_idx, num_slots, batch,
+    #  out, dev_status, stream)
+    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, A, None, 0, -1, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_step(d, 1, A, None, A, A, None, None, A, A, None, 4, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, MIS, None, 4, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_decode_step(ctypes.byref(gdn.Dims(1, 16)), 1, A, A, A, A, None, None, A, A, None,
-                             4, A, None) == gdn.GDN_ERR_UNSUPPORTED
+                             4, 4, A, None, None) == gdn.GDN_ERR_UNSUPPORTED
+    # pools smaller than the batch without a slot map, and a negative pool size
+    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, A, None, 3, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_step(d, 1, A, A, A, A, None, None, A, A, A, -1, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
     bs = L.gdn_decode_step_bf16_state
-    assert bs(d, 1, A, A, A, A, None, None, A, A, None, -1, A, None) == gdn.GDN_ERR_INVALID_ARG
-    assert bs(d, 1, A, A, A, A, None, None, A, None, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
-    assert bs(d, 1, A, A, A, A, None, None, A, MIS, None, 4, A, None) == gdn.GDN_ERR_INVALID_ARG
-    assert bs(d, 3, A, A, A, A, None, None, A, A, None, 4, A, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert bs(d, 1, A, A, A, A, None, None, A, A, None, 0, -1, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert bs(d, 1, A, A, A, A, None, None, A, None, None, 4, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert bs(d, 1, A, A, A, A, None, None, A, MIS, None, 4, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert bs(d, 3, A, A, A, A, None, None, A, A, None, 4, 4, A, None, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert bs(d, 1, A, A, A, A, None, None, A, A, None, 2, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
     mt = L.gdn_decode_multi
-    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, -1, A, None, None) == gdn.GDN_ERR_INVALID_ARG
-    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, 9, A, None, None) == gdn.GDN_ERR_UNSUPPORTED
-    assert mt(d, 1, A, None, A, A, None, None, A, A, None, 4, 4, A, None, None) == gdn.GDN_ERR_INVALID_ARG
-    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, 4, A, MIS, None) == gdn.GDN_ERR_INVALID_ARG
+    # (..., slot_idx, num_slots, batch, tokens, out, snapshots, dev_status, stream)
+    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, 4, -1, A, None, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, 4, 9, A, None, None, None) == gdn.GDN_ERR_UNSUPPORTED
+    assert mt(d, 1, A, None, A, A, None, None, A, A, None, 4, 4, 4, A, None, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 4, 4, 4, A, MIS, None, None) == gdn.GDN_ERR_INVALID_ARG
+    assert mt(d, 1, A, A, A, A, None, None, A, A, None, 1, 4, 4, A, None, None, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_debug_wait_probe(None, 10, None) == gdn.GDN_ERR_INVALID_ARG
     assert L.gdn_debug_wait_probe(A, 10_000_000, None) == gdn.GDN_ERR_INVALID_ARG
 
@@ -132,8 +140,8 @@ def test_block_prefill_argument_errors(L):
     assert size(d, 0, 1, 16) == 0
     assert size(d, 256, -1, 16) == 0
     layer = L.gdn_chunk_prefill_workspace_size(d, 1, 1, 4096)
-    # layer scratch + bf16 x, z, o and fp32 b|a, beta, g per token
-    assert size(d, 2048, 1, 4096) >= layer + 4096 * (8192 * 2 + 2 * 4096 * 2 + 4 * 32 * 4)
+    # layer scratch + bf16 x, z, o and fp32 beta, g per token (the gates leave the GEMM directly)
+    assert size(d, 2048, 1, 4096) >= layer + 4096 * (8192 * 2 + 2 * 4096 * 2 + 2 * 32 * 4)
     assert _block(L, None) == gdn.GDN_ERR_INVALID_ARG
     assert _block(L, d, hidden=0) == gdn.GDN_ERR_INVALID_ARG
     assert _block(L, d, hidden=260) == gdn.GDN_ERR_INVALID_ARG      # rows of 16-byte multiples
@@ -157,9 +165,10 @@ def test_prefill_slots_argument_errors(L):
     d = ctypes.byref(gdn.Dims())
     f = L.gdn_chunk_prefill_slots
 
-    def call(dims=d, dtype=1, x=A, N=1, T=16, slot=A, pool=A, conv=A, ws=A, ws_bytes=1 << 40):
-        return f(dims, dtype, x, None, A, A, None, None, A, N, T, slot, pool, conv, A, ws, ws_bytes,
-                 None, None)
+    def call(dims=d, dtype=1, x=A, N=1, T=16, slot=A, slots=8, pool=A, conv=A, ws=A,
+             ws_bytes=1 << 40):
+        return f(dims, dtype, x, None, A, A, None, None, A, N, T, slot, slots, pool, conv, A, ws,
+                 ws_bytes, None, None)
     assert call(pool=None) == gdn.GDN_ERR_INVALID_ARG
     assert call(pool=MIS) == gdn.GDN_ERR_INVALID_ARG
     assert call(conv=MIS) == gdn.GDN_ERR_INVALID_ARG
@@ -167,7 +176,10 @@ def test_prefill_slots_argument_errors(L):
     assert call(dtype=5) == gdn.GDN_ERR_UNSUPPORTED
     assert call(ws=None) == gdn.GDN_ERR_WORKSPACE
     assert call(x=None) == gdn.GDN_ERR_INVALID_ARG
-    assert call(N=0, T=0, pool=None, slot=None, conv=None) == gdn.GDN_OK
+    assert call(slots=-1) == gdn.GDN_ERR_INVALID_ARG
+    assert call(slots=0) == gdn.GDN_ERR_INVALID_ARG                  # a slot map into no rows
+    assert call(slot=None, N=4, T=16, slots=3) == gdn.GDN_ERR_INVALID_ARG  # identity needs N rows
+    assert call(N=0, T=0, pool=None, slot=None, conv=None, slots=0) == gdn.GDN_OK
 
 
 def test_zero_size_calls_launch_nothing(L):
@@ -175,14 +187,14 @@ def test_zero_size_calls_launch_nothing(L):
     # no sequences, no tokens: valid and a no-op
     assert L.gdn_chunk_prefill(d, 1, None, None, None, None, None, None, None, 0, 0, None, None,
                                None, None, None, A, 1 << 30, None, None) == gdn.GDN_OK
-    assert L.gdn_decode_step(d, 1, None, None, None, None, None, None, None, None, None, 0, None,
-                             None) == gdn.GDN_OK
+    assert L.gdn_decode_step(d, 1, None, None, None, None, None, None, None, None, None, 0, 0,
+                             None, None, None) == gdn.GDN_OK
     assert L.gdn_decode_step_bf16_state(d, 1, None, None, None, None, None, None, None, None,
-                                        None, 0, None, None) == gdn.GDN_OK
-    assert L.gdn_decode_multi(d, 1, None, None, None, None, None, None, None, None, None, 0, 4,
-                              None, None, None) == gdn.GDN_OK
-    assert L.gdn_decode_multi(d, 1, None, None, None, None, None, None, None, None, None, 4, 0,
-                              None, None, None) == gdn.GDN_OK
+                                        None, 0, 0, None, None, None) == gdn.GDN_OK
+    assert L.gdn_decode_multi(d, 1, None, None, None, None, None, None, None, None, None, 0, 0, 4,
+                              None, None, None, None) == gdn.GDN_OK
+    assert L.gdn_decode_multi(d, 1, None, None, None, None, None, None, None, None, None, 4, 4, 0,
+                              None, None, None, None) == gdn.GDN_OK
     assert L.gdn_gated_rmsnorm(1, None, None, None, 1e-6, 0, 128, None, None) == gdn.GDN_OK
 
 
@@ -249,7 +261,7 @@ def test_plain_c_consumer(L, tmp_path):
                     "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
                     "-L", lib_dir, "-l:libgdn.so", f"-Wl,-rpath,{lib_dir}"], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
-    assert out == ["1", "2", "8192", "workspace", "too", "small", "0", "2", "256", "173"]
+    assert out == ["2", "2", "8192", "workspace", "too", "small", "0", "2", "256", "173"]
 
 
 def test_binding_refuses_undersized_buffers(L):
@@ -276,7 +288,7 @@ def test_binding_refuses_undersized_buffers(L):
     B = 3
     xs = torch.zeros(B, Cc, dtype=torch.bfloat16)
     cw = torch.zeros(Cc, 4, dtype=torch.bfloat16)
-    with pytest.raises(ValueError, match="S holds"):       # identity slots need B state rows
+    with pytest.raises(ValueError, match="pools hold 2 rows"):  # identity slots need B rows
         gdn.decode_step(xs, torch.zeros(B, Hv), torch.zeros(B, Hv),
                         torch.zeros(B, 3, Cc, dtype=torch.bfloat16),
                         torch.zeros(B - 1, Hv, 128, 128), cw, dims=d)
@@ -301,3 +313,39 @@ def test_binding_refuses_undersized_buffers(L):
                           torch.zeros(H, 2 * Hv, dtype=torch.bfloat16), torch.zeros(Hv),
                           torch.zeros(Hv), torch.zeros(Hv * 128, H - 1, dtype=torch.bfloat16),
                           cu, dims=d)
+
+
+def test_bounds_check_build_compiles_and_exports_every_symbol():
+    """The bounds-check variant (-DGDN_BOUNDS_CHECK) builds for sm_100a and exports the same
+    entry points; its status strings know GDN_ERR_BOUNDS."""
+    from gated_deltanet_layer_02_b200 import build as gdn_build
+    path = gdn_build.build(bounds_check=True)
+    assert os.path.basename(path) == "libgdn_checked.so"
+    Lc = gdn.lib_checked()
+    for name in gdn.EXPORTS:
+        assert hasattr(Lc, name), name
+    assert Lc.gdn_status_string(gdn.GDN_ERR_BOUNDS).decode().startswith("index check failed")
+    assert Lc.gdn_abi_version() == L_abi_version()
+
+
+def L_abi_version():
+    return gdn.lib().gdn_abi_version()
+
+
+def test_debug_options_are_checked(L):
+    bad = [dict(chain_split=3), dict(segment_chunks=-1), dict(fault=7),
+           dict(fault=1, fault_chunk=-1), dict(wait_limit_us=10_000_001)]
+    for kw in bad:
+        opts = gdn.DebugOptions(**{**dict(wait_limit_us=0, segment_chunks=0, chain_split=0,
+                                          fault=0, fault_chunk=0), **kw})
+        assert L.gdn_debug_set(ctypes.byref(opts)) == gdn.GDN_ERR_INVALID_ARG, kw
+    ok = gdn.DebugOptions(5000, 2, 4, gdn.GDN_FAULT_SKIP_CHAIN_LOAD, 3)
+    assert L.gdn_debug_set(ctypes.byref(ok)) == gdn.GDN_OK
+    assert L.gdn_debug_set(None) == gdn.GDN_OK
+    # the workspace size follows the segment length (one fp32 state per segment boundary)
+    d = ctypes.byref(gdn.Dims())
+    plain = L.gdn_chunk_prefill_workspace_size(d, 1, 1, 4096)
+    with gdn.debug_options(segment_chunks=8):
+        seg = L.gdn_chunk_prefill_workspace_size(d, 1, 1, 4096)
+    assert seg > plain
+    assert L.gdn_chunk_prefill_workspace_size(d, 1, 1, 4096) == plain

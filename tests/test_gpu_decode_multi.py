@@ -57,11 +57,12 @@ def test_multi_equals_single_steps_and_oracle(dtype, k):
     od = oracle_dims_of(w)
     S_ref = S_pool.double().numpy()[slot.long().numpy()].copy()
     cs_ref = cs_pool.double().numpy()[slot.long().numpy()].copy()
+    M_ref = np.abs(S_ref)
     for t in range(k):
         s = steps[t]
-        ref = oracle.decode_step(od, s["x"], s["beta"], s["g"], cs_ref, S_ref,
-                                 conv_w=st["conv_w"], z=s["z"], norm_w=st["norm_w"])
-        assert_close(out_m[:, t], ref, dtype, f"k={k} token {t}: out")
-        assert_close(snaps[:, t], S_ref, dtype, f"k={k} token {t}: state snapshot")
-    assert_close(S_m[slot.long()], S_ref, dtype, f"k={k}: final state")
+        ref, sc = oracle.decode_step(od, s["x"], s["beta"], s["g"], cs_ref, S_ref,
+                                     conv_w=st["conv_w"], z=s["z"], norm_w=st["norm_w"], M=M_ref)
+        assert_close(out_m[:, t], ref, dtype, f"k={k} token {t}: out", scale=sc)
+        assert_close(snaps[:, t], S_ref, dtype, f"k={k} token {t}: state snapshot", scale=M_ref)
+    assert_close(S_m[slot.long()], S_ref, dtype, f"k={k}: final state", scale=M_ref)
     np.testing.assert_array_equal(np64(cs_m[slot.long()]), cs_ref)

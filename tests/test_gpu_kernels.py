@@ -88,6 +88,7 @@ def test_decode_steps_with_slots(dtype, with_z):
     nw = _randn((128,), dtype, 13) if with_z else None
     S_d, cs_d = dev(S), dev(cs)
     S_ref, cs_ref = S.double().numpy().copy(), cs.double().numpy().copy()
+    M_ref = np.abs(S_ref)
     for step in range(steps):
         x = _randn((B, Cc), dtype, 100 + step)
         z = _randn((B, 4, 128), dtype, 200 + step) if with_z else None
@@ -96,9 +97,9 @@ def test_decode_steps_with_slots(dtype, with_z):
         out = gdn.decode_step(dev(x), dev(beta), dev(g), cs_d, S_d, dev(w), z=dev(z),
                               norm_w=dev(nw), slot_idx=dev(slot_idx), dims=dims)
         torch.cuda.synchronize()
-        ref = oracle.decode_step(od, x, beta, g, cs_ref, S_ref, conv_w=w, z=z, norm_w=nw,
-                                 slot_idx=slot_idx)
-        assert_close(out, ref, dtype, f"decode out step {step}")
+        ref, sc = oracle.decode_step(od, x, beta, g, cs_ref, S_ref, conv_w=w, z=z, norm_w=nw,
+                                     slot_idx=slot_idx, M=M_ref)
+        assert_close(out, ref, dtype, f"decode out step {step}", scale=sc)
     np.testing.assert_array_equal(np64(cs_d), cs_ref)
     err = np.max(np.abs(np64(S_d) - S_ref))
     assert err <= 1e-4, err

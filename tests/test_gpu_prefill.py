@@ -14,10 +14,10 @@ pytestmark = pytest.mark.gpu
 
 def _check(w, inp, what):
     out, SN, convN = gpu_prefill(w, inp)
-    ref_o, ref_S, ref_c = oracle_prefill(w, inp)
-    e1 = assert_close(out, ref_o, w.dtype, f"{what}: out")
-    e2 = assert_close(SN, ref_S, w.dtype, f"{what}: final state")
-    np.testing.assert_array_equal(np64(convN), ref_c)
+    ref = oracle_prefill(w, inp)
+    e1 = assert_close(out, ref[0], w.dtype, f"{what}: out", scale=ref.out_scale)
+    e2 = assert_close(SN, ref[1], w.dtype, f"{what}: final state", scale=ref.SN_scale)
+    np.testing.assert_array_equal(np64(convN), ref[2])
     return e1, e2
 
 
@@ -94,67 +94,62 @@ def test_split_prefill_matches_whole():
     a = gpu_prefill(w, first)
     second["S0"], second["conv0"] = a[1].cpu(), a[2].cpu()
     b = gpu_prefill(w, second)
-    ref_o, ref_S, _ = oracle_prefill(w, inp)
-    assert_close(torch.cat([a[0], b[0]]), ref_o, w.dtype, "split out")
-    assert_close(b[1], ref_S, w.dtype, "split state")
+    ref = oracle_prefill(w, inp)
+    assert_close(torch.cat([a[0], b[0]]), ref[0], w.dtype, "split out", scale=ref.out_scale)
+    assert_close(b[1], ref[1], w.dtype, "split state", scale=ref.SN_scale)
     assert torch.equal(b[2], full[2])
-
-
-@pytest.fixture
-def pipeline_env(monkeypatch):
-    """Sets the library's pipeline knobs (segment length in chunks, chain d_v split)."""
-    def set_(seg, split):
-        monkeypatch.setenv("GDN_SEGMENT_CHUNKS", str(seg))
-        monkeypatch.setenv("GDN_CHAIN_SPLIT", str(split))
-    return set_
 
 
 @pytest.mark.parametrize("seg", [1, 2, 3, 5])
 @pytest.mark.parametrize("split", [1, 2, 4])
-def test_bf16_pipelined_segments(pipeline_env, seg, split):
+def test_bf16_pipelined_segments(seg, split):
     # Segments of `seg` chunks: sequences cross segment boundaries (the state is carried in
     # fp32 between launches), short and empty sequences fall inside one segment, and the
     # chain's d_v split is forced so that every split meets every boundary case.
-    pipeline_env(seg, split)
     w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(700, 0, 5, 129, 0, 1100, 64, 260),
                       s0_std=0.1)
-    _check(w, inputs.prefill_inputs(w, 1200 + 10 * seg + split, with_conv0=True),
-           f"seg={seg} split={split}")
+    inp = inputs.prefill_inputs(w, 1200 + 10 * seg + split, with_conv0=True)
+    with gdn.debug_options(segment_chunks=seg, chain_split=split):
+        _check(w, inp, f"seg={seg} split={split}")
 
 
-def test_bf16_pipelined_matches_single_launch_bitwise(pipeline_env):
+def test_bf16_pipelined_matches_single_launch_bitwise():
     # The pipeline reorders launches only: with the same split, the segmented and the single
     # launch runs perform the same arithmetic and must agree to the bit.
     w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(900, 33, 1500), s0_std=0.1)
     inp = inputs.prefill_inputs(w, 1300, with_conv0=True)
-    pipeline_env(1 << 19, 2)
-    one = gpu_prefill(w, inp)
-    pipeline_env(2, 2)
-    seg = gpu_prefill(w, inp)
+    with gdn.debug_options(segment_chunks=1 << 19, chain_split=2):
+        one = gpu_prefill(w, inp)
+    with gdn.debug_options(segment_chunks=2, chain_split=2):
+        seg = gpu_prefill(w, inp)
     for a, b, name in zip(one, seg, ("out", "final state", "conv state")):
         assert torch.equal(a, b), name
 
 
-@pytest.mark.parametrize("lengths", [(300,), (1, 0, 700, 129), (2000,)])
-def test_bf16_fused_prep_and_chain(monkeypatch, lengths):
-    # The opt-in persistent prep + chain kernel (chains waiting on flags the prep workers set).
-    monkeypatch.setenv("GDN_FUSED", "1")
-    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=lengths, s0_std=0.1)
-    _check(w, inputs.prefill_inputs(w, 1400 + len(lengths), with_conv0=True), f"fused {lengths}")
-
-
-def test_bf16_fused_matches_separate_launches_bitwise(monkeypatch):
-    # The persistent prep + chain kernel runs the same arithmetic as the separate launches with
-    # 32-column chain blocks; only the schedule differs.
-    w = inputs.custom(16, 32, 128, torch.bfloat16, lengths=(1500,), s0_std=0.1)
-    inp = inputs.prefill_inputs(w, 1450, with_conv0=True)
-    monkeypatch.setenv("GDN_FUSED", "0")
-    monkeypatch.setenv("GDN_CHAIN_SPLIT", "4")
-    sep = gpu_prefill(w, inp)
-    monkeypatch.setenv("GDN_FUSED", "1")
-    fused = gpu_prefill(w, inp)
-    for x, y, name in zip(sep, fused, ("out", "final state", "conv state")):
-        assert torch.equal(x, y), name
+@pytest.mark.parametrize("segmented", [False, True])
+def test_chain_wait_runs_out_and_the_context_stays_usable(segmented):
+    # A load the chain waits for is left out on purpose (debug fault injection): the chain's
+    # bounded wait must run out within its limit (5 ms here), write GDN_ERR_TIMEOUT, let its
+    # other copies land, free its TMEM and end; afterwards the same stream runs a normal
+    # prefill that matches the one before the fault bit for bit.
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(700, 300), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 1350, with_conv0=True)
+    seg = 2 if segmented else 0
+    with gdn.debug_options(segment_chunks=seg):
+        good = gpu_prefill(w, inp)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    import time
+    t0 = time.perf_counter()
+    with gdn.debug_options(wait_limit_us=5000, segment_chunks=seg,
+                           fault=gdn.GDN_FAULT_SKIP_CHAIN_LOAD, fault_chunk=2):
+        gpu_prefill(w, inp, dev_status=status)
+    elapsed = time.perf_counter() - t0
+    assert int(status.item()) == gdn.GDN_ERR_TIMEOUT
+    assert elapsed < 1.0, elapsed     # gave up after its 5 ms limit, not the 2 s default
+    with gdn.debug_options(segment_chunks=seg):
+        again = gpu_prefill(w, inp)
+    for a, b, name in zip(good, again, ("out", "final state", "conv state")):
+        assert torch.equal(a, b), name
 
 
 def test_bf16_states_updated_in_place():
@@ -162,7 +157,7 @@ def test_bf16_states_updated_in_place():
     # serving loop does; the conv history then comes from its own kernel after the layer.
     w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300, 0, 2, 129), s0_std=0.1)
     inp = inputs.prefill_inputs(w, 1500, with_conv0=True)
-    ref_o, ref_S, ref_c = oracle_prefill(w, inp)
+    ref = oracle_prefill(w, inp)
     S = dev(inp["S0"]).clone()
     conv = dev(inp["conv0"]).clone()
     out, SN, convN = gdn.chunk_prefill(
@@ -171,17 +166,20 @@ def test_bf16_states_updated_in_place():
         conv0=conv, convN=conv, dims=dims_of(w))
     torch.cuda.synchronize()
     assert SN.data_ptr() == S.data_ptr() and convN.data_ptr() == conv.data_ptr()
-    assert_close(out, ref_o, w.dtype, "in place: out")
-    assert_close(S, ref_S, w.dtype, "in place: final state")
-    np.testing.assert_array_equal(np64(conv), ref_c)
+    assert_close(out, ref[0], w.dtype, "in place: out", scale=ref.out_scale)
+    assert_close(S, ref[1], w.dtype, "in place: final state", scale=ref.SN_scale)
+    np.testing.assert_array_equal(np64(conv), ref[2])
 
 
 @pytest.mark.parametrize("seg,split", [(0, 0), (1, 4), (2, 1)])
-def test_bf16_chunk_boundary_states(pipeline_env, seg, split):
+def test_bf16_chunk_boundary_states(seg, split):
     # gdn_chunk_prefill_states: entry c is the state after chunk c of the sequence-by-sequence
     # chunk numbering; the oracle gives it as the final state of the prefix ending there
-    if seg:
-        pipeline_env(seg, split)
+    with gdn.debug_options(segment_chunks=seg, chain_split=split):
+        _chunk_boundary_states(seg)
+
+
+def _chunk_boundary_states(seg):
     w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300, 0, 129, 256, 5), s0_std=0.1)
     inp = inputs.prefill_inputs(w, 1600 + seg, with_conv0=True)
     lengths = [int(v) for v in w.lengths]
@@ -202,11 +200,63 @@ def test_bf16_chunk_boundary_states(pipeline_env, seg, split):
             sub["cu_seqlens"] = torch.tensor([0, P], dtype=torch.int32)
             sub["S0"] = inp["S0"][n:n + 1].contiguous()
             sub["conv0"] = inp["conv0"][n:n + 1].contiguous()
-            _, ref_S, _ = oracle_prefill(w, sub)
-            assert_close(cs[c], ref_S[0], w.dtype, f"state after chunk {c} (sequence {n})")
+            ref = oracle_prefill(w, sub)
+            assert_close(cs[c], ref[1][0], w.dtype, f"state after chunk {c} (sequence {n})",
+                         scale=ref.SN_scale[0])
             c += 1
     assert c == C
     last = np.cumsum([(L + 127) // 128 for L in lengths]) - 1
     for n, L in enumerate(lengths):
         if L:
             assert torch.equal(cs[int(last[n])], SN[n]), f"last chunk of sequence {n}"
+
+
+@pytest.mark.parametrize("seg,split", [(0, 0), (1, 4), (2, 2), (3, 1)])
+def test_bf16_page64_states(seg, split):
+    # gdn_chunk_prefill_pages with 64-token pages: entry p is the state after page p of the
+    # sequence-by-sequence page numbering (the middle of a 128-token chunk for even pages of
+    # chunks longer than 64); the oracle gives each as the final state of the prefix ending there
+    with gdn.debug_options(segment_chunks=seg, chain_split=split):
+        w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300, 0, 129, 64, 65, 5, 200),
+                          s0_std=0.1)
+        inp = inputs.prefill_inputs(w, 1700 + 10 * seg + split, with_conv0=True)
+        lengths = [int(v) for v in w.lengths]
+        P = sum((L + 63) // 64 for L in lengths)
+        ps = torch.full((P, w.num_v_heads, 128, 128), float("nan"), dtype=torch.float32,
+                        device="cuda")
+        out, SN, convN = gpu_prefill(w, inp, page_states=ps, page_size=64)
+    ref_full = oracle_prefill(w, inp)
+    assert_close(out, ref_full[0], w.dtype, "pages: out", scale=ref_full.out_scale)
+    starts = np.cumsum([0] + lengths)
+    p = 0
+    for n, L in enumerate(lengths):
+        for j in range((L + 63) // 64):
+            E = min(64 * (j + 1), L)
+            t0 = int(starts[n])
+            sub = dict(inp)
+            for k in ("x", "beta", "g", "z"):
+                if inp[k] is not None:
+                    sub[k] = inp[k][t0:t0 + E].contiguous()
+            sub["cu_seqlens"] = torch.tensor([0, E], dtype=torch.int32)
+            sub["S0"] = inp["S0"][n:n + 1].contiguous()
+            sub["conv0"] = inp["conv0"][n:n + 1].contiguous()
+            ref = oracle_prefill(w, sub)
+            assert_close(ps[p], ref[1][0], w.dtype, f"state after page {j} of sequence {n}",
+                         scale=ref.SN_scale[0])
+            p += 1
+        if L:
+            assert torch.equal(ps[p - 1], SN[n]), f"last page of sequence {n}"
+    assert p == P
+
+
+def test_bf16_page128_states_equal_chunk_states():
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300, 129, 5), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 1750, with_conv0=True)
+    C = sum((int(L) + 127) // 128 for L in w.lengths)
+    cs = torch.empty((C, w.num_v_heads, 128, 128), dtype=torch.float32, device="cuda")
+    ps = torch.empty_like(cs)
+    a = gpu_prefill(w, inp, chunk_states=cs)
+    b = gpu_prefill(w, inp, page_states=ps, page_size=128)
+    assert torch.equal(cs, ps)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)

@@ -16,6 +16,11 @@ operand anywhere in the oracle fails at least one of them:
   P11 contraction bound |S_t|_F <= alpha_t |S_{t-1}|_F + beta_t |v_t|.
   P12 token-mixer gates: sigmoid / softplus special values and torch's softplus; with
       identity projections the token mixer reduces to the layer.
+  P13 error scales (the tolerance the GPU tests use): M >= |S| and c >= |o| element-wise
+      (triangle inequality); T = 1 closed form of M; beta = 0 gives M = exp(sum g) |S_0|;
+      the normalised-output scale is invariant, and M scales linearly, when v and S_0 are
+      scaled together; decode steps carry M exactly as the prefill does; the scales leave
+      out, SN and convN untouched.
 The chunked (WY/UT) form the CUDA path uses is checked against the oracle in
 test_chunk_algebra.py (P6).
 """
@@ -430,3 +435,118 @@ def test_p12_block_with_identity_projections_is_the_layer():
     np.testing.assert_allclose(y, o.reshape(T, -1) @ w_out, rtol=1e-12, atol=1e-12)
     np.testing.assert_array_equal(SN, SN2)
     np.testing.assert_array_equal(convN, convN2)
+
+
+# --------------------------------------------------------------------------------------- P13
+def _scaled_run(dims, x, beta, g, S0=None, **kw):
+    return _run(dims, x, beta, g, S0=S0, with_scales=True, **kw)
+
+
+def test_p13_scales_bound_values_and_leave_results_unchanged():
+    r = _rng(131)
+    T, d, hk, hv = 9, 8, 1, 2
+    q, k, v = r.standard_normal((T, hk, d)), r.standard_normal((T, hk, d)), r.standard_normal((T, hv, d))
+    beta, g = r.uniform(0, 1, (T, hv)), r.uniform(-0.5, 0, (T, hv))
+    S0 = _f32(r.standard_normal((1, hv, d, d)))
+    x = _pack_x(q, k, v)
+    out, SN, convN, osc, M = _scaled_run(_dims(hk, hv, d), x, beta, g, S0=S0)
+    out2, SN2, convN2 = _run(_dims(hk, hv, d), x, beta, g, S0=S0)
+    assert np.array_equal(out, out2) and np.array_equal(SN, SN2) and np.array_equal(convN, convN2)
+    assert np.all(M >= np.abs(SN) * (1 - 1e-12))
+    assert np.all(osc >= np.abs(out) * (1 - 1e-12))
+
+
+def test_p13_single_token_closed_form():
+    r = _rng(132)
+    d = 8
+    q, k, v = r.standard_normal((1, 1, d)), r.standard_normal((1, 1, d)), r.standard_normal((1, 1, d))
+    beta, g = np.array([[0.6]]), np.array([[-0.3]])
+    S0 = _f32(r.standard_normal((1, 1, d, d)))
+    out, SN, _, osc, M = _scaled_run(_dims(1, 1, d), _pack_x(q, k, v), beta, g, S0=S0)
+    a, b = np.exp(np.float64(_f32(g)[0, 0])), np.float64(_f32(beta)[0, 0])
+    kn, qn = np.abs(_unit(k[0, 0])), np.abs(_unit(q[0, 0]))
+    S0a = np.abs(S0[0, 0].astype(np.float64))
+    M1 = a * S0a + b * np.outer(np.abs(v[0, 0]) + a * S0a @ kn, kn)
+    np.testing.assert_allclose(M[0, 0], M1, rtol=1e-12)
+    np.testing.assert_allclose(osc[0, 0], M1 @ qn, rtol=1e-12)
+
+
+def test_p13_no_write_decays_the_magnitude():
+    r = _rng(133)
+    T, d = 6, 8
+    q, k, v = r.standard_normal((T, 1, d)), r.standard_normal((T, 1, d)), r.standard_normal((T, 1, d))
+    g = r.uniform(-0.5, 0, (T, 1))
+    S0 = _f32(r.standard_normal((1, 1, d, d)))
+    _, _, _, _, M = _scaled_run(_dims(1, 1, d), _pack_x(q, k, v), np.zeros((T, 1)), g, S0=S0)
+    G = np.sum(_f32(g).astype(np.float64))
+    np.testing.assert_allclose(M[0, 0], np.exp(G) * np.abs(S0[0, 0]), rtol=1e-12)
+
+
+def test_p13_scales_follow_the_magnitude_of_v_and_S0():
+    # conv off: scaling the v channels and S0 by 4 scales S, M and the pre-norm scales by 4 and
+    # leaves the normalised output and its scale unchanged (up to the norm's eps)
+    r = _rng(134)
+    T, d, hv = 11, 8, 2
+    q, k, v = r.standard_normal((T, 1, d)), r.standard_normal((T, 1, d)), r.standard_normal((T, hv, d))
+    beta, g = r.uniform(0, 1, (T, hv)), r.uniform(-0.5, 0, (T, hv))
+    S0 = _f32(r.standard_normal((1, hv, d, d)))
+    z = torch.from_numpy(r.standard_normal((T, hv, d)))
+    dims = _dims(1, hv, d, norm_eps=0.0)
+    one = _scaled_run(dims, _pack_x(q, k, v), beta, g, S0=S0, z=z)
+    four = _scaled_run(dims, _pack_x(q, k, 4 * v), beta, g, S0=4 * S0, z=z)
+    np.testing.assert_allclose(four[4], 4 * one[4], rtol=1e-12)
+    np.testing.assert_allclose(four[0], one[0], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(four[3], one[3], rtol=1e-10)
+    plain_one = _scaled_run(dims, _pack_x(q, k, v), beta, g, S0=S0)
+    plain_four = _scaled_run(dims, _pack_x(q, k, 4 * v), beta, g, S0=4 * S0)
+    np.testing.assert_allclose(plain_four[3], 4 * plain_one[3], rtol=1e-12)
+
+
+def test_p13_decode_carries_the_magnitude_like_prefill():
+    r = _rng(135)
+    T, d, hk, hv = 4, 8, 1, 2
+    dims = _dims(hk, hv, d)
+    q, k, v = r.standard_normal((T, hk, d)), r.standard_normal((T, hk, d)), r.standard_normal((T, hv, d))
+    beta, g = r.uniform(0, 1, (T, hv)), r.uniform(-0.5, 0, (T, hv))
+    S0 = _f32(r.standard_normal((1, hv, d, d)))
+    x = _pack_x(q, k, v)
+    cw = torch.from_numpy(r.standard_normal((x.shape[1], 4)))
+    pre = oracle.prefill(dims, torch.from_numpy(x), torch.from_numpy(_f32(beta)),
+                         torch.from_numpy(_f32(g)), inputs.cu_seqlens_of([T]), conv_w=cw,
+                         S0=torch.from_numpy(S0), nthreads=1, with_scales=True)
+    S = S0.astype(np.float64).copy()
+    M = np.abs(S)
+    cs = np.zeros((1, 3, x.shape[1]))
+    for t in range(T):
+        _, sc = oracle.decode_step(dims, torch.from_numpy(x[t:t + 1]),
+                                   torch.from_numpy(_f32(beta[t:t + 1])),
+                                   torch.from_numpy(_f32(g[t:t + 1])), cs, S, conv_w=cw, M=M)
+        np.testing.assert_allclose(sc[0], pre[3][t], rtol=1e-12)
+    np.testing.assert_allclose(M, pre[4], rtol=1e-12)
+
+
+def test_p13_conv_magnitudes_single_token():
+    # conv on, zero history, S0 = 0, T = 1: the conv output of channel c is silu(w[c,3] x[c]) with
+    # magnitude 1.1 |w[c,3] x[c]|; q and k magnitudes are divided by the norm of their conv
+    # output; M_1 = beta vm km^T and the output scale is M_1 qm
+    r = _rng(136)
+    d = 8
+    q, k, v = r.standard_normal((1, 1, d)), r.standard_normal((1, 1, d)), r.standard_normal((1, 1, d))
+    x = _pack_x(q, k, v)
+    w = r.standard_normal((x.shape[1], 4))
+    beta, g = np.array([[0.7]]), np.array([[-0.2]])
+    dims = _dims(1, 1, d)
+    out, SN, _, osc, M = oracle.prefill(
+        dims, torch.from_numpy(x), torch.from_numpy(_f32(beta)), torch.from_numpy(_f32(g)),
+        inputs.cu_seqlens_of([1]), conv_w=torch.from_numpy(w), nthreads=1, with_scales=True)
+    acc = w[:, 3] * x[0]
+    silu = acc / (1 + np.exp(-acc))
+    mag = 1.1 * np.abs(acc)
+    qm = mag[:d] / np.linalg.norm(silu[:d])
+    km = mag[d:2 * d] / np.linalg.norm(silu[d:2 * d])
+    vm = mag[2 * d:]
+    b = np.float64(_f32(beta)[0, 0])
+    M1 = b * np.outer(vm, km)
+    np.testing.assert_allclose(M[0, 0], M1, rtol=1e-12)
+    np.testing.assert_allclose(osc[0, 0], M1 @ qm, rtol=1e-12)
+    assert np.all(M[0, 0] >= np.abs(SN[0, 0]) * (1 - 1e-12))
