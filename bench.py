@@ -576,6 +576,35 @@ def job_tokens_per_s(world, tokens_per_rank, ms):
     return world * tokens_per_rank / (ms * 1e-3)
 
 
+def profile_prefill(args, idx, dev, gdn):
+    """The step graph of prefill workload `idx` replayed --warmup + --steps times (a small,
+    self-contained command for ncu captures)."""
+    w = inputs.CONFIGS[idx]
+    inp = inputs.prefill_inputs(w, inputs.config_seed(idx))
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    dims = gdn.Dims(w.num_k_heads, w.num_v_heads, w.head_dim, w.conv_kernel)
+    T, N = w.tokens, len(w.lengths)
+    out = torch.empty((T, w.num_v_heads, w.head_dim), dtype=w.dtype, device=dev)
+    SN = torch.empty((N, w.num_v_heads, w.head_dim, w.head_dim), dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(N, T, w.dtype, dims), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        gdn.chunk_prefill(d["x"], d["beta"], d["g"], d["cu_seqlens"], conv_w=d["conv_w"],
+                          z=d["z"], norm_w=d["norm_w"], S0=d["S0"], SN=SN, out=out,
+                          workspace=ws, dims=dims)
+    ms = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        b.synchronize()
+        if i >= args.warmup:
+            ms.append(a.elapsed_time(b))
+    return {"workload": w.name, "ms_per_step": statistics.mean(ms), "steps": args.steps}
+
+
 #: the headline prefill workload (the largest single-GPU configuration: one 262,144-token
 #: sequence) and the secondary prefill workloads reported beside it
 HEADLINE = 4
@@ -606,7 +635,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=64)
     ap.add_argument("--headline-only", action="store_true",
-                    help="only the headline prefill leg (for profiling runs)")
+                    help="only the headline prefill leg")
+    ap.add_argument("--prefill-only", type=int, default=None, metavar="CONFIG",
+                    help="profiling aid: only the step graph of prefill workload CONFIG (0-4), "
+                         "--warmup + --steps replays, no other leg; prints its ms per step")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -630,6 +662,9 @@ def main():
     import gated_deltanet_layer_02_b200 as gdn
     peaks, peak_src = load_peaks()
     n = world
+    if args.prefill_only is not None:
+        print(json.dumps(profile_prefill(args, args.prefill_only, dev, gdn)), flush=True)
+        return
 
     def run_prefill(idx, steps, e2e):
         r = bench_prefill(args, inputs.CONFIGS[idx], inputs.config_seed(idx), dev, gdn, peaks,

@@ -47,7 +47,7 @@ class DebugOptions(ctypes.Structure):
     """gdn_debug_options (see gdn.h): test and debug controls of the calling host thread."""
     _fields_ = [("wait_limit_us", ctypes.c_uint32), ("segment_chunks", ctypes.c_int32),
                 ("chain_split", ctypes.c_int32), ("fault", ctypes.c_int32),
-                ("fault_chunk", ctypes.c_int32)]
+                ("fault_chunk", ctypes.c_int32), ("timestamps", ctypes.c_void_p)]
 
 
 class GdnError(RuntimeError):
@@ -542,8 +542,10 @@ class debug_options:
     """
 
     def __init__(self, wait_limit_us=0, segment_chunks=0, chain_split=0, fault=GDN_FAULT_NONE,
-                 fault_chunk=0):
-        self.opts = DebugOptions(wait_limit_us, segment_chunks, chain_split, fault, fault_chunk)
+                 fault_chunk=0, timestamps=None):
+        ts = None if timestamps is None else _ptr(timestamps, "timestamps", torch.int64)
+        self.opts = DebugOptions(wait_limit_us, segment_chunks, chain_split, fault, fault_chunk,
+                                 ts)
 
     def __enter__(self):
         _check("gdn_debug_set", lib().gdn_debug_set(ctypes.byref(self.opts)))

@@ -272,6 +272,7 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
     const gdn_debug_options& dbg = gdn_host::debug_opts();
     a.wait_ns = dbg.wait_limit_us ? (uint64_t)dbg.wait_limit_us * 1000ull : gdn::kWaitLimitNs;
     a.fault_chunk = dbg.fault == GDN_FAULT_SKIP_CHAIN_LOAD ? dbg.fault_chunk : -1;
+    a.stamps = dbg.timestamps;
   }
   a.N = num_seqs;
   a.T = num_tokens;

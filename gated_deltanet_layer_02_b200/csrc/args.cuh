@@ -89,6 +89,7 @@ struct PrefillArgs {
                         // GDN_ERR_TIMEOUT
   int fault_chunk;      // debug fault injection: the first chain CTA skips the W load of this
                         // chunk (-1: none)
+  uint64_t* stamps;     // debug: %globaltimer stamps of kernel phases (first CTA), or NULL
   int num_slots;        // rows of the state pools when `slot` is set
   int N, T, Hk, Hv, nsplit;
   float q_scale, l2_eps, norm_eps;

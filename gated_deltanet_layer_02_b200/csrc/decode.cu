@@ -19,7 +19,7 @@
 
 namespace gdn {
 
-constexpr int kDecodeThreads = 256;
+constexpr int kDecodeThreads = 128;  // four warps: four CTAs per SM at 128 registers
 constexpr int kMaxR = 8;
 
 // Four consecutive state elements of a lane: fp32 (16 bytes) or bf16 (8 bytes, the serving
@@ -63,7 +63,7 @@ struct StateIO<__nv_bfloat16> {
 };
 
 template <typename T, typename TS>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a) {
   constexpr int d = kHeadDim;
   const int b = blockIdx.x / a.Hk;
   const int hk = blockIdx.x % a.Hk;

@@ -1429,6 +1429,378 @@ done:
   if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// --------------------------------------------------------------------------- out, persistent
+// The output step as a persistent, warp-specialised kernel: each CTA takes a contiguous range of
+// (chunk, value head) units and pipelines them over two shared-memory stages, so that the tiles
+// of the next unit load while the current one computes, and the epilogue of one unit overlaps
+// the products of the next.
+//   warps 0-3  (group A) per unit: P = mask(e^(G_i - G_j)) Q K^T and Q^ = diag(e^G) Q, written
+//              to TMEM as bf16 A operands (thread = token row, all 128 columns)
+//   warps 4-7  (group B) per unit: gated RMSNorm epilogue of O from one of two TMEM buffers,
+//              z and the chunk entry loaded into registers one unit ahead, bf16 rows out
+//   warp 8     TMA loads of Q, K and U into the unit's stage, as soon as the stage is free
+//   warp 9     tcgen05.mma: Q K^T; once it has completed, the TMA load of S^T into K's place;
+//              then O = Q^ S^T + P U into TMEM buffer (unit % 2)
+// Stage s (96 KB): Q | K, then S^T | U.  It is free again when the unit's O products complete
+// (group A has read Q before it released P and Q^).  Every hand-over is an mbarrier (TMA
+// transactions, tcgen05.commit, or 128 thread arrivals), and every wait is bounded; a wait that
+// runs out sets the abort flag, which the other roles' waits also observe.
+constexpr int kOutPThreads = 320;
+constexpr uint32_t kOpStage = 98304;                        // Q | K-then-S^T | U
+constexpr uint32_t kOpQ = 0, kOpKS = 32768, kOpU = 65536;   // offsets inside a stage
+constexpr uint32_t kOpEnd = 2 * kOpStage;                   // 196608
+constexpr uint32_t kOutPSmem = kOpEnd + 1024 + 2048;
+constexpr uint32_t kColPQ = 0, kColO0 = 128;                // O buffer b at 128 + 128 b
+
+struct OutPCtl {
+  uint64_t* qk_full;      // [2]
+  uint64_t* u_full;       // [2]
+  uint64_t* s_full;       // [2]
+  uint64_t* stage_empty;  // [2]
+  uint64_t* gram_done;
+  uint64_t* pq_ready;
+  uint64_t* o_full;       // [2]
+  uint64_t* o_empty;      // [2]
+  uint64_t* drain;        // products in flight after an abort
+  uint32_t* tslot;
+  int* abort;
+  float* G_s;             // [128] gates of the unit group A works on
+  float* F_s;             // [128] column factors
+  float* w_s;             // [128] norm weight
+  __device__ explicit OutPCtl(uint8_t* sm) {
+    uint64_t* b = reinterpret_cast<uint64_t*>(sm + kOpEnd);
+    qk_full = b;
+    u_full = b + 2;
+    s_full = b + 4;
+    stage_empty = b + 6;
+    gram_done = b + 8;
+    pq_ready = b + 9;
+    o_full = b + 10;
+    o_empty = b + 12;
+    drain = b + 14;
+    tslot = reinterpret_cast<uint32_t*>(b + 15);
+    abort = reinterpret_cast<int*>(tslot + 1);
+    G_s = reinterpret_cast<float*>(sm + kOpEnd + 256);
+    F_s = G_s + kC;
+    w_s = F_s + kC;
+  }
+};
+
+// Bounded wait that also gives up once another role has set the abort flag.
+__device__ __forceinline__ bool wait_role(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
+    __nanosleep(32);
+  }
+}
+
+__global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
+    PrefillArgs a, const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+    const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapU) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const OutPCtl ctl(sm);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Hv = a.Hv;
+  if (tid == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(ctl.qk_full + b, 1);
+      mbar_init(ctl.u_full + b, 1);
+      mbar_init(ctl.s_full + b, 1);
+      mbar_init(ctl.stage_empty + b, 1);
+      mbar_init(ctl.o_full + b, 1);
+      mbar_init(ctl.o_empty + b, 128);
+    }
+    mbar_init(ctl.gram_done, 1);
+    mbar_init(ctl.pq_ready, 128);
+    mbar_init(ctl.drain, 1);
+    *ctl.abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8) tmem_alloc(ctl.tslot, 512);
+  if (tid >= 128 && tid < 256)
+    ctl.w_s[tid - 128] = a.norm_w ? __bfloat162float(a.norm_w[tid - 128]) : 1.f;
+  pdl_wait();  // the chain's S^T and U (and, before it, every earlier kernel of the call)
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *ctl.tslot;
+  volatile int* abort = ctl.abort;
+  // this CTA's units: a contiguous range of the (chunk, value head) units of the launch, so
+  // that the two value heads of a key head (same Q and K tiles) follow each other
+  const int nchunks = min(a.c1, a.ws.seq_first[a.N]) - a.c0;
+  const int nunits = max(nchunks, 0) * Hv;
+  const int per = (nunits + gridDim.x - 1) / gridDim.x;
+  const int u0 = blockIdx.x * per, u1 = min(nunits, u0 + per);
+  const int count = max(u1 - u0, 0);
+  bool ok = true;
+  // debug stamps (first CTA, first 32 units): [role * 64 + 2 i (+1)] = start / end of unit i
+  uint64_t* stamps = (a.stamps && blockIdx.x == 0) ? a.stamps : nullptr;
+  auto stamp = [&](int role, int i, int end) {
+    if (stamps && i < 32) stamps[role * 64 + 2 * i + end] = global_timer_ns();
+  };
+  int last_qk[2] = {-1, -1};  // producer: last unit loaded into each stage
+  int last_s = -1;            // MMA role: last unit whose S^T load it issued
+
+  if (warp == 8) {
+    // ------------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      for (int i = 0; i < count && ok; ++i) {
+        const int u = u0 + i, c = a.c0 + u / Hv, h = u % Hv, hk = h / (Hv / a.Hk);
+        const int st = i & 1;
+        if (i >= 2) ok = wait_role(ctl.stage_empty + st, ((i >> 1) - 1) & 1, abort, a.wait_ns);
+        if (!ok) break;
+        uint8_t* stage = sm + st * kOpStage;
+        stamp(0, i, 0);
+        const int rowQK = (c * a.Hk + hk) * kC, rowV = (c * Hv + h) * kC;
+        mbar_arrive_expect_tx(ctl.qk_full + st, 4 * kTile);
+        tma_load_2d(stage + kOpQ, &mapQ, ctl.qk_full + st, 0, rowQK);
+        tma_load_2d(stage + kOpQ + kTile, &mapQ, ctl.qk_full + st, 64, rowQK);
+        tma_load_2d(stage + kOpKS, &mapK, ctl.qk_full + st, 0, rowQK);
+        tma_load_2d(stage + kOpKS + kTile, &mapK, ctl.qk_full + st, 64, rowQK);
+        mbar_arrive_expect_tx(ctl.u_full + st, 2 * kTile);
+        tma_load_2d(stage + kOpU, &mapU, ctl.u_full + st, 0, rowV);
+        tma_load_2d(stage + kOpU + kTile, &mapU, ctl.u_full + st, 64, rowV);
+        last_qk[st] = i;
+      }
+      if (!ok) *abort = 1;
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      for (int i = 0; i < count && ok; ++i) {
+        const int u = u0 + i, c = a.c0 + u / Hv, h = u % Hv;
+        const int st = i & 1;
+        const uint32_t sQ = smem_u32(sm + st * kOpStage + kOpQ);
+        const uint32_t sKS = smem_u32(sm + st * kOpStage + kOpKS);
+        const uint32_t sU = smem_u32(sm + st * kOpStage + kOpU);
+        ok = wait_role(ctl.qk_full + st, (i >> 1) & 1, abort, a.wait_ns);
+        if (!ok) break;
+        stamp(1, i, 0);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + kColPQ, desc_kmajor(sQ, kk, kTile), desc_kmajor(sKS, kk, kTile),
+                   idesc_bf16(128, 128, false, false), kk > 0);
+        mma_commit(ctl.gram_done);
+        // K is consumed once the product completes: S^T of the unit into its place
+        ok = wait_role(ctl.gram_done, i & 1, abort, a.wait_ns);
+        if (!ok) break;
+        const int rowV = (c * Hv + h) * kC;
+        uint8_t* ks = sm + st * kOpStage + kOpKS;
+        mbar_arrive_expect_tx(ctl.s_full + st, 2 * kTile);
+        tma_load_2d(ks, &mapS, ctl.s_full + st, 0, rowV);
+        tma_load_2d(ks + kTile, &mapS, ctl.s_full + st, 64, rowV);
+        last_s = i;
+        ok = wait_role(ctl.pq_ready, i & 1, abort, a.wait_ns) &&
+             wait_role(ctl.s_full + st, (i >> 1) & 1, abort, a.wait_ns) &&
+             wait_role(ctl.u_full + st, (i >> 1) & 1, abort, a.wait_ns) &&
+             (i < 2 || wait_role(ctl.o_empty + st, ((i >> 1) - 1) & 1, abort, a.wait_ns));
+        if (!ok) break;
+        stamp(1, i, 1);
+        tc_fence_after();
+        const uint32_t colO = kColO0 + st * 128;
+        constexpr uint32_t id = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + colO, tmem + kColPQ + 64 + kk * 8, desc_mnmajor(sKS, kk, kTile), id,
+                      kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + colO, tmem + kColPQ + kk * 8, desc_mnmajor(sU, kk, kTile), id, 1);
+        mma_commit(ctl.o_full + st);
+        mma_commit(ctl.stage_empty + st);
+      }
+      if (!ok) *abort = 1;
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------ group A: P and Q^ into TMEM, row tid
+    const int i_row = tid;
+    const uint32_t lane_addr = tmem_at(tmem, warp * 32, 0);
+    float g_next = 0.f;
+    if (count > 0) {
+      const int c = a.c0 + u0 / Hv, h = u0 % Hv;
+      g_next = a.ws.Gw[((size_t)c * Hv + h) * kC + i_row];
+    }
+    for (int i = 0; i < count; ++i) {
+      const int st = i & 1;
+      // gates of this unit into shared memory (loaded one unit ahead), column factors
+      bar_sync_n(1, 128);  // the previous unit's readers of G_s / F_s are done
+      ctl.G_s[i_row] = g_next;
+      if (i + 1 < count) {
+        const int u = u0 + i + 1, c = a.c0 + u / Hv, h = u % Hv;
+        g_next = a.ws.Gw[((size_t)c * Hv + h) * kC + i_row];
+      }
+      bar_sync_n(1, 128);
+      ctl.F_s[i_row] = __expf(ctl.G_s[i_row | 31] - ctl.G_s[i_row]);
+      // one decision for the whole group (its named barriers need all 128 threads)
+      const bool got = wait_role(ctl.gram_done, i & 1, abort, a.wait_ns);
+      if (bar_or_n(1, 128, !got)) {
+        ok = false;
+        break;
+      }
+      if (i_row == 0) stamp(2, i, 0);
+      tc_fence_after();
+      const float Gi = ctl.G_s[i_row];
+      uint32_t pp[64], qq[64];
+      const int rq = i_row >> 5;  // row block of this thread (warp-uniform)
+#pragma unroll
+      for (int jb = 0; jb < 4; ++jb) {
+        const int j0 = jb * 32;
+        if (jb > rq) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pp[jb * 16 + e] = 0u;
+          continue;
+        }
+        float v[32];
+        tmem_ld32(lane_addr + kColPQ + j0, v);
+        tmem_ld_wait();
+        if (jb < rq) {
+          // every j < every i: exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31
+          const float rf = __expf(Gi - ctl.G_s[j0 + 31]);
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            pp[jb * 16 + e / 2] = pack_bf16x2(rf * ctl.F_s[j0 + e] * v[e],
+                                              rf * ctl.F_s[j0 + e + 1] * v[e + 1]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int j = j0 + e;
+            const float p0 = j <= i_row ? __expf(Gi - ctl.G_s[j]) * v[e] : 0.f;
+            const float p1 = j + 1 <= i_row ? __expf(Gi - ctl.G_s[j + 1]) * v[e + 1] : 0.f;
+            pp[jb * 16 + e / 2] = pack_bf16x2(p0, p1);
+          }
+        }
+      }
+      const float eg = __expf(Gi);
+      const uint8_t* Qs = sm + st * kOpStage + kOpQ;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const uint4 u4 =
+            *reinterpret_cast<const uint4*>(Qs + (q >> 3) * kTile + sw128_off(i_row, q & 7));
+        const __nv_bfloat162* hq = reinterpret_cast<const __nv_bfloat162*>(&u4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(hq[e]);
+          qq[q * 4 + e] = pack_bf16x2(f.x * eg, f.y * eg);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        tmem_st32(lane_addr + kColPQ + q * 32, *reinterpret_cast<float(*)[32]>(pp + q * 32));
+        tmem_st32(lane_addr + kColPQ + 64 + q * 32, *reinterpret_cast<float(*)[32]>(qq + q * 32));
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ctl.pq_ready);  // Q of the stage is read, P and Q^ are in TMEM
+      if (i_row == 0) stamp(2, i, 1);
+    }
+    if (!ok) *abort = 1;
+  } else {
+    // ----------------------------------------------- group B: gated RMSNorm epilogue, row
+    const int i_row = tid - 128;
+    const uint32_t lane_addr = tmem_at(tmem, (warp & 3) * 32, 0);
+    uint4 zreg[16];
+    ChunkInfo ci_next{};
+    auto prefetch = [&](int i) {  // chunk entry and z row of unit i
+      const int u = u0 + i, c = a.c0 + u / Hv, h = u % Hv;
+      ci_next = a.ws.chunks[c];
+      if (a.z && i_row < ci_next.L) {
+        const uint4* zp =
+            reinterpret_cast<const uint4*>(a.z + ((size_t)(ci_next.t0 + i_row) * Hv + h) * kD);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) zreg[q] = __ldg(zp + q);
+      }
+    };
+    if (count > 0) prefetch(0);
+    for (int i = 0; i < count; ++i) {
+      const int u = u0 + i, h = u % Hv;
+      const ChunkInfo ci = ci_next;
+      const int st = i & 1;
+      ok = wait_role(ctl.o_full + st, (i >> 1) & 1, abort, a.wait_ns);
+      if (!ok) break;
+      if (i_row == 0) stamp(3, i, 0);
+      tc_fence_after();
+      const uint32_t colO = kColO0 + st * 128;
+      float inv = 1.f;
+      if (a.z) {
+        float ss = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float v[32];
+          tmem_ld32(lane_addr + colO + q * 32, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
+        }
+        inv = rsqrtf(ss / kD + a.norm_eps);
+      }
+      __nv_bfloat16* dst = a.out + ((size_t)(ci.t0 + i_row) * Hv + h) * kD;
+      const bool valid = i_row < ci.L;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float v[32];
+        tmem_ld32(lane_addr + colO + q * 32, v);
+        tmem_ld_wait();
+        if (a.z) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const __nv_bfloat162* zh = reinterpret_cast<const __nv_bfloat162*>(&zreg[q * 4 + r]);
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              const float2 zf = __bfloat1622float2(zh[e2]);
+              const int e = r * 8 + e2 * 2;
+              v[e] = v[e] * inv * ctl.w_s[q * 32 + e] * silu_fast(zf.x);
+              v[e + 1] = v[e + 1] * inv * ctl.w_s[q * 32 + e + 1] * silu_fast(zf.y);
+            }
+          }
+        }
+        if (valid) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            float o8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o8[e] = v[r * 8 + e];
+            store8(dst + q * 32 + r * 8, o8);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(ctl.o_empty + st);
+      if (i_row == 0) stamp(3, i, 1);
+      if (i + 1 < count) prefetch(i + 1);
+    }
+    if (!ok) *abort = 1;
+  }
+  // every role has left its loop; without an abort, group B has seen the last products
+  // complete and every load was consumed
+  __syncthreads();
+  if (*abort) {
+    if (tid == 0) report_status(a.status, GDN_ERR_TIMEOUT);
+    if (tid == 32 * 9) {  // every product and S^T load issued so far lands first
+      mma_commit(ctl.drain);
+      mbar_wait(ctl.drain, 0, a.wait_ns);
+      if (last_s >= 0) mbar_wait(ctl.s_full + (last_s & 1), (last_s >> 1) & 1, a.wait_ns);
+    }
+    if (tid == 32 * 8) {  // and every load of the producer
+      for (int b = 0; b < 2; ++b)
+        if (last_qk[b] >= 0) {
+          mbar_wait(ctl.qk_full + b, (last_qk[b] >> 1) & 1, a.wait_ns);
+          mbar_wait(ctl.u_full + b, (last_qk[b] >> 1) & 1, a.wait_ns);
+        }
+    }
+    __syncthreads();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) tmem_dealloc(tmem, 512);
+}
+
 }  // namespace gdn
 
 // =================================================================================== host
@@ -1652,8 +2024,18 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gdn::gdn_qkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                gdn::kQkvSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(gdn::gdn_out_persistent_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, gdn::kOutPSmem);
     if (e != cudaSuccess) return e;
     attr = true;
+  }
+  int num_sms = 0;
+  {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
   }
   cudaError_t e;
   trace_begin("chunk_schedule", s);
@@ -1696,9 +2078,12 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     }
   };
   auto launch_out = [&](const gdn::PrefillArgs& sa, cudaStream_t st, bool pdl) -> cudaError_t {
+    // persistent: one CTA per SM at most, each taking a contiguous range of units
+    const int units = (sa.c1 - sa.c0) * sa.Hv;
+    const int grid = std::max(1, std::min(units, num_sms));
     trace_begin("gdn_out", st);
-    cudaError_t e2 = launch_k(pdl, gdn::gdn_out_kernel, dim3((unsigned)(sa.c1 - sa.c0), sa.Hv),
-                              dim3(gdn::kOutThreads), gdn::kOutSmem, st, sa, mQ, mK, mS, mU);
+    cudaError_t e2 = launch_k(pdl, gdn::gdn_out_persistent_kernel, dim3(grid),
+                              dim3(gdn::kOutPThreads), gdn::kOutPSmem, st, sa, mQ, mK, mS, mU);
     trace_end(st);
     return e2;
   };

@@ -395,6 +395,9 @@ int gdn_trace_span(gdn_trace* trace, int32_t i, float* start_ms, float* end_ms);
  *                  runs out.  Used to test the timeout path with no GPU fault: the call then
  *                  reports GDN_ERR_TIMEOUT in dev_status and its outputs are undefined.
  *   fault_chunk    see fault.
+ *   timestamps     device pointer (uint64, 1024 entries) or NULL: the kernels of the bf16
+ *                  prefill that support it record %globaltimer stamps of their phases there
+ *                  (first CTA only), for profiling the pipeline of a persistent kernel.
  * Returns GDN_OK, or GDN_ERR_INVALID_ARG for an out-of-range field (settings unchanged).
  */
 #define GDN_FAULT_NONE 0
@@ -405,6 +408,7 @@ typedef struct gdn_debug_options {
   int32_t chain_split;
   int32_t fault;
   int32_t fault_chunk;
+  uint64_t* timestamps;
 } gdn_debug_options;
 int gdn_debug_set(const gdn_debug_options* opts);
 
