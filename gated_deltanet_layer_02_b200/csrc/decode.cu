@@ -11,9 +11,10 @@
 //   o_r = alpha * (S_r . q) + u * kq        (= S'_r . q)
 //   S'_r = alpha * S_r + u * k
 // so each state element is read once and written once.  One CTA per (sequence, key head)
-// handles that key head's R = Hv/Hk value heads; each warp streams whole rows (a lane owns 4
-// consecutive columns, 512 contiguous bytes per warp load) with kRowBatch rows in flight, and
-// reduces the two dot products with warp shuffles.
+// handles that key head's R = Hv/Hk value heads.  A warp streams four rows at a time (a row
+// quad), eight lanes per row: a lane holds 16 elements of its row, and the two dot products
+// reduce in three shuffle steps inside each group of eight lanes.  Every aligned 128-byte line
+// of a row is read by one group of eight lanes with one 16-byte load each.
 #include "args.cuh"
 #include "common.cuh"
 
@@ -22,45 +23,109 @@ namespace gdn {
 constexpr int kDecodeThreads = 128;  // four warps: four CTAs per SM at 128 registers
 constexpr int kMaxR = 8;
 
-// Four consecutive state elements of a lane: fp32 (16 bytes) or bf16 (8 bytes, the serving
-// option of a bf16 recurrent state: arithmetic stays fp32, the new state is rounded to nearest
-// even once per step).  Loads stay raw until used, so that the bf16 state keeps as many bytes
-// in flight (twice the rows) in the same registers.  Streaming loads and stores: the state is
-// touched once per step.
+// Sixteen elements of a row held by one lane (s = lane & 7, its place in the row's group):
+// fp32 columns 4 s + 32 m + e (m = 0..3, e = 0..3), or bf16 columns 8 s + 64 m + e (m = 0, 1,
+// e = 0..7) for the serving option of a bf16 recurrent state (arithmetic stays fp32, the new
+// state is rounded to nearest even once per step).  Loads stay raw until used, so that the
+// bf16 state keeps as many bytes in flight (twice the rows) in the same registers.  Streaming
+// loads and stores: the state is touched once per step.
 template <typename TS>
-struct StateIO;
+struct RowPart;
 template <>
-struct StateIO<float> {
-  using Raw = float4;
-  static constexpr int kRows = 8;  // rows per batch and warp
-  static __device__ __forceinline__ Raw load(const float* p) {
-    return __ldcs(reinterpret_cast<const float4*>(p));
+struct RowPart<float> {
+  static constexpr int kQuads = 2;  // row quads per batch and warp (8 rows)
+  struct Raw {
+    float4 v[4];
+  };
+  static __device__ __forceinline__ int col(int s, int j) { return 4 * s + 32 * (j >> 2) + (j & 3); }
+  static __device__ __forceinline__ void load(Raw& r, const float* row, int s) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) r.v[m] = __ldcs(reinterpret_cast<const float4*>(row + 4 * s + 32 * m));
   }
-  static __device__ __forceinline__ float4 f4(Raw r) { return r; }
-  static __device__ __forceinline__ void store(float* p, float4 v) {
-    __stcs(reinterpret_cast<float4*>(p), v);
+  static __device__ __forceinline__ void unpack(const Raw& r, float (&f)[16]) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      f[4 * m] = r.v[m].x;
+      f[4 * m + 1] = r.v[m].y;
+      f[4 * m + 2] = r.v[m].z;
+      f[4 * m + 3] = r.v[m].w;
+    }
+  }
+  static __device__ __forceinline__ void store(float* row, int s, const float (&f)[16]) {
+#pragma unroll
+    for (int m = 0; m < 4; ++m)
+      __stcs(reinterpret_cast<float4*>(row + 4 * s + 32 * m),
+             make_float4(f[4 * m], f[4 * m + 1], f[4 * m + 2], f[4 * m + 3]));
   }
 };
 template <>
-struct StateIO<__nv_bfloat16> {
-  using Raw = uint2;
-  static constexpr int kRows = 16;
-  static __device__ __forceinline__ Raw load(const __nv_bfloat16* p) {
-    return __ldcs(reinterpret_cast<const uint2*>(p));
+struct RowPart<__nv_bfloat16> {
+  static constexpr int kQuads = 4;  // 16 rows
+  struct Raw {
+    uint4 v[2];
+  };
+  static __device__ __forceinline__ int col(int s, int j) { return 8 * s + 64 * (j >> 3) + (j & 7); }
+  static __device__ __forceinline__ void load(Raw& r, const __nv_bfloat16* row, int s) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) r.v[m] = __ldcs(reinterpret_cast<const uint4*>(row + 8 * s + 64 * m));
   }
-  static __device__ __forceinline__ float4 f4(Raw u) {
-    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-    return make_float4(lo.x, lo.y, hi.x, hi.y);
+  static __device__ __forceinline__ void unpack(const Raw& r, float (&f)[16]) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t w[4] = {r.v[m].x, r.v[m].y, r.v[m].z, r.v[m].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+        f[8 * m + 2 * e] = p.x;
+        f[8 * m + 2 * e + 1] = p.y;
+      }
+    }
   }
-  static __device__ __forceinline__ void store(__nv_bfloat16* p, float4 v) {
-    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
-    uint2 u;
-    u.x = *reinterpret_cast<const uint32_t*>(&lo);
-    u.y = *reinterpret_cast<const uint32_t*>(&hi);
-    __stcs(reinterpret_cast<uint2*>(p), u);
+  static __device__ __forceinline__ void store(__nv_bfloat16* row, int s, const float (&f)[16]) {
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(f[8 * m + 2 * e], f[8 * m + 2 * e + 1]);
+        w[e] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+      __stcs(reinterpret_cast<uint4*>(row + 8 * s + 64 * m), make_uint4(w[0], w[1], w[2], w[3]));
+    }
   }
 };
+
+// One token's update of one row (the lane's 16 elements f, in place); returns o_r (in every
+// lane of the row's group).  kn, qn: the lane's elements of the normalised k and q.  The one-
+// and k-token kernels both call this, so that their results agree bit for bit.
+__device__ __forceinline__ float row_update(float (&f)[16], const float (&kn)[16],
+                                            const float (&qn)[16], float alpha, float beta,
+                                            float vv, float kq) {
+  float dk4[4] = {0.f, 0.f, 0.f, 0.f}, dq4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    dk4[j & 3] = fmaf(f[j], kn[j], dk4[j & 3]);
+    dq4[j & 3] = fmaf(f[j], qn[j], dq4[j & 3]);
+  }
+  float dk = (dk4[0] + dk4[1]) + (dk4[2] + dk4[3]), dq = (dq4[0] + dq4[1]) + (dq4[2] + dq4[3]);
+#pragma unroll
+  for (int o = 4; o > 0; o >>= 1) {
+    dk += __shfl_xor_sync(0xffffffffu, dk, o);
+    dq += __shfl_xor_sync(0xffffffffu, dq, o);
+  }
+  const float u = beta * (vv - alpha * dk);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) f[j] = fmaf(alpha, f[j], u * kn[j]);
+  return fmaf(alpha, dq, u * kq);
+}
+
+// Input channel of position gch of the conv outputs of key head hk (q | k | v_0..v_{R-1}).
+__device__ __forceinline__ int channel_of(int gch, int hk, int R, int Hk) {
+  const int grp = gch / kHeadDim, off = gch % kHeadDim;
+  if (grp == 0) return hk * kHeadDim + off;
+  if (grp == 1) return Hk * kHeadDim + hk * kHeadDim + off;
+  return 2 * Hk * kHeadDim + (hk * R + grp - 2) * kHeadDim + off;
+}
 
 template <typename T, typename TS>
 __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a) {
@@ -71,6 +136,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
   const int Cc = (2 * a.Hk + a.Hv) * d;
   const int slot = state_row(a.slot_idx, b, a.num_slots);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = lane >> 3, sub = lane & 7;
   if (slot < 0) {  // slot out of range: the sequence is skipped, its outputs are not written
     if (tid == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
     return;
@@ -79,34 +145,35 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
   __shared__ float y_s[(2 + kMaxR) * d];  // q | k | v_0..v_{R-1} after conv
   __shared__ float o_s[kMaxR * d];
   __shared__ float red_s[4];
+  __shared__ float2 ab_s[kMaxR];          // (alpha, beta) per value head
 
   const T* x = static_cast<const T*>(a.x) + (size_t)b * Cc;
   const T* w = static_cast<const T*>(a.conv_w);
   T* cs = static_cast<T*>(a.conv_state) + (size_t)slot * 3 * Cc;
 
   // the first batch of state rows does not depend on q and k: its loads go out before the conv
-  using IO = StateIO<TS>;
-  constexpr int kRowBatch = IO::kRows;
+  using RP = RowPart<TS>;
+  constexpr int kQ = RP::kQuads;
+  constexpr int kBatch = 4 * kQ;
   const int rows_per_warp = R * d / (kDecodeThreads / 32);
-  const int nbatch = rows_per_warp / kRowBatch;
+  const int nbatch = rows_per_warp / kBatch;
   TS* S = static_cast<TS*>(a.S);
-  auto row_ptr = [&](int gr) {
-    const int hr = gr / d, v = gr % d;
-    return S + (((size_t)slot * a.Hv + hk * R + hr) * d + v) * d + 4 * lane;
+  auto row_ptr = [&](int gr) {  // gr: row of the CTA's R d rows
+    return S + ((size_t)slot * a.Hv + hk * R) * d * d + (size_t)gr * d;
   };
-  typename IO::Raw sv[kRowBatch], sn[kRowBatch];
+  typename RP::Raw cur[kQ], nxt[kQ];
 #pragma unroll
-  for (int i = 0; i < kRowBatch; ++i) sv[i] = IO::load(row_ptr(warp * rows_per_warp + i));
+  for (int q = 0; q < kQ; ++q) RP::load(cur[q], row_ptr(warp * rows_per_warp + 4 * q + grp), sub);
 
+  if (tid < R) {
+    const int h = hk * R + tid;
+    ab_s[tid] = make_float2(expf(a.g[(size_t)b * a.Hv + h]), a.beta[(size_t)b * a.Hv + h]);
+  }
   // ---- conv + SiLU with in-place history shift: 2 channels per item
   const int items = (2 + R) * d / 2;
   for (int it = tid; it < items; it += kDecodeThreads) {
-    const int gch = it * 2;              // position inside y_s
-    const int grp = gch / d, off = gch % d;
-    int c;
-    if (grp == 0) c = hk * d + off;
-    else if (grp == 1) c = a.Hk * d + hk * d + off;
-    else c = 2 * a.Hk * d + (hk * R + grp - 2) * d + off;
+    const int gch = it * 2;  // position inside y_s
+    const int c = channel_of(gch, hk, R, a.Hk);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const float s0 = to_f(cs[c + e]), s1 = to_f(cs[Cc + c + e]), s2 = to_f(cs[2 * Cc + c + e]);
@@ -134,54 +201,32 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
   const float rq = a.q_scale * rsqrtf(red_s[0] + a.l2_eps);
   const float rk = rsqrtf(red_s[1] + a.l2_eps);
   const float kq = red_s[2] * rq * rk;
-  float kreg[4], qreg[4];
+  float kn[16], qn[16];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    kreg[j] = y_s[d + 4 * lane + j] * rk;
-    qreg[j] = y_s[4 * lane + j] * rq;
+  for (int j = 0; j < 16; ++j) {
+    kn[j] = y_s[d + RP::col(sub, j)] * rk;
+    qn[j] = y_s[RP::col(sub, j)] * rq;
   }
 
-  // ---- state pass: R*d rows split over the warps, two batches of rows in flight
+  // ---- state pass: the warp's rows in batches of kQ row quads, the next batch in flight
   for (int bt = 0; bt < nbatch; ++bt) {
-    const int r0 = warp * rows_per_warp + bt * kRowBatch;
+    const int r0 = warp * rows_per_warp + bt * kBatch;
     if (bt + 1 < nbatch) {
 #pragma unroll
-      for (int i = 0; i < kRowBatch; ++i) sn[i] = IO::load(row_ptr(r0 + kRowBatch + i));
-    }
-    float dk[kRowBatch], dq[kRowBatch];
-#pragma unroll
-    for (int i = 0; i < kRowBatch; ++i) {
-      const float4 f = IO::f4(sv[i]);
-      dk[i] = f.x * kreg[0] + f.y * kreg[1] + f.z * kreg[2] + f.w * kreg[3];
-      dq[i] = f.x * qreg[0] + f.y * qreg[1] + f.z * qreg[2] + f.w * qreg[3];
+      for (int q = 0; q < kQ; ++q) RP::load(nxt[q], row_ptr(r0 + kBatch + 4 * q + grp), sub);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-      for (int i = 0; i < kRowBatch; ++i) {
-        dk[i] += __shfl_xor_sync(0xffffffffu, dk[i], o);
-        dq[i] += __shfl_xor_sync(0xffffffffu, dq[i], o);
-      }
+    for (int q = 0; q < kQ; ++q) {
+      const int gr = r0 + 4 * q + grp, hr = gr / d;
+      const float2 ab = ab_s[hr];
+      float f[16];
+      RP::unpack(cur[q], f);
+      const float o = row_update(f, kn, qn, ab.x, ab.y, y_s[(2 + hr) * d + gr % d], kq);
+      if (sub == 0) o_s[gr] = o;
+      RP::store(row_ptr(gr), sub, f);
     }
 #pragma unroll
-    for (int i = 0; i < kRowBatch; ++i) {
-      const int gr = r0 + i, hr = gr / d, v = gr % d;
-      const int h = hk * R + hr;
-      const float alpha = expf(__ldg(a.g + (size_t)b * a.Hv + h));
-      const float beta = __ldg(a.beta + (size_t)b * a.Hv + h);
-      const float vv = y_s[(2 + hr) * d + v];
-      const float u = beta * (vv - alpha * dk[i]);
-      if (lane == 0) o_s[hr * d + v] = alpha * dq[i] + u * kq;
-      const float4 f = IO::f4(sv[i]);
-      float4 nv;
-      nv.x = alpha * f.x + u * kreg[0];
-      nv.y = alpha * f.y + u * kreg[1];
-      nv.z = alpha * f.z + u * kreg[2];
-      nv.w = alpha * f.w + u * kreg[3];
-      IO::store(row_ptr(gr), nv);
-    }
-#pragma unroll
-    for (int i = 0; i < kRowBatch; ++i) sv[i] = sn[i];
+    for (int q = 0; q < kQ; ++q) cur[q] = nxt[q];
   }
   __syncthreads();
   // ---- gated RMSNorm (or plain output), one warp per value head
@@ -213,15 +258,22 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
 // ---------------------------------------------------------------------------- multi-token
 // k tokens per sequence in one launch (verification of k speculative draft tokens): the state
 // rows are read once, take the k updates in registers and are written once; every token uses
-// exactly the arithmetic of decode_kernel, so the results equal k calls of the one-token step.
+// exactly the arithmetic of decode_kernel (the same row_update, the same normalised q and k
+// products), so the results equal k calls of the one-token step.  Per-token constants (the
+// normalised q and k, alpha, beta) are set up once in shared memory before the state pass.
 // With `snaps` set, the state after every token is stored as well ([B, k, Hv, d, d] fp32), so
 // that a caller that accepts only the first m tokens can take snapshot m - 1.  Dynamic shared
-// memory: per token (2 + R) d conv outputs, R d outputs and three norms.
+// memory: per token (2 + R) d conv outputs (q and k normalised in place), R d outputs, three
+// norms and R (alpha, beta) pairs.
 constexpr int kMaxTokens = 8;
 
+__host__ __device__ constexpr size_t multi_smem_floats(int k, int R) {
+  return (size_t)k * (2 + 2 * R) * kHeadDim + 3 * k + 2 * k * R;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kDecodeThreads) decode_multi_kernel(DecodeArgs a, int k,
-                                                                      float* snaps) {
+__global__ void __launch_bounds__(kDecodeThreads, 4) decode_multi_kernel(DecodeArgs a, int k,
+                                                                         float* snaps) {
   constexpr int d = kHeadDim;
   const int b = blockIdx.x / a.Hk;
   const int hk = blockIdx.x % a.Hk;
@@ -229,6 +281,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_multi_kernel(DecodeArgs
   const int Cc = (2 * a.Hk + a.Hv) * d;
   const int slot = state_row(a.slot_idx, b, a.num_slots);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = lane >> 3, sub = lane & 7;
   if (slot < 0) {  // slot out of range: the sequence is skipped, its outputs are not written
     if (tid == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
     return;
@@ -237,31 +290,31 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_multi_kernel(DecodeArgs
   float* y_s = dsm;                          // [k][(2 + R) d]: q | k | v_0..v_{R-1}
   float* o_s = y_s + k * (2 + R) * d;        // [k][R d]
   float* red_s = o_s + k * R * d;            // [k][3]: |q|^2, |k|^2, q.k
+  float2* ab_s = reinterpret_cast<float2*>(red_s + 3 * k + (k & 1));  // [k][R]
 
   const T* w = static_cast<const T*>(a.conv_w);
   T* cs = static_cast<T*>(a.conv_state) + (size_t)slot * 3 * Cc;
-  using IO = StateIO<float>;
-  constexpr int kRowBatch = IO::kRows;
+  using RP = RowPart<float>;
+  constexpr int kQ = RP::kQuads;
+  constexpr int kBatch = 4 * kQ;
   const int rows_per_warp = R * d / (kDecodeThreads / 32);
-  const int nbatch = rows_per_warp / kRowBatch;
+  const int nbatch = rows_per_warp / kBatch;
   float* S = static_cast<float*>(a.S);
-  auto row_off = [&](int gr) {
-    const int hr = gr / d, v = gr % d;
-    return (((size_t)slot * a.Hv + hk * R + hr) * d + v) * d + 4 * lane;
-  };
-  float4 sv[kRowBatch];
+  auto row_off = [&](int gr) { return ((size_t)slot * a.Hv + hk * R) * d * d + (size_t)gr * d; };
+  RP::Raw cur[kQ], nxt[kQ];
 #pragma unroll
-  for (int i = 0; i < kRowBatch; ++i) sv[i] = IO::load(S + row_off(warp * rows_per_warp + i));
+  for (int q = 0; q < kQ; ++q) RP::load(cur[q], S + row_off(warp * rows_per_warp + 4 * q + grp), sub);
 
+  for (int i = tid; i < k * R; i += kDecodeThreads) {
+    const int t = i / R, h = hk * R + i % R;
+    const size_t gi = ((size_t)b * k + t) * a.Hv + h;
+    ab_s[i] = make_float2(expf(a.g[gi]), a.beta[gi]);
+  }
   // ---- conv + SiLU over the k tokens, history in registers, final history written back
   const int items = (2 + R) * d / 2;
   for (int it = tid; it < items; it += kDecodeThreads) {
     const int gch = it * 2;
-    const int grp = gch / d, off = gch % d;
-    int c;
-    if (grp == 0) c = hk * d + off;
-    else if (grp == 1) c = a.Hk * d + hk * d + off;
-    else c = 2 * a.Hk * d + (hk * R + grp - 2) * d + off;
+    const int c = channel_of(gch, hk, R, a.Hk);
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       float s0 = to_f(cs[c + e]), s1 = to_f(cs[Cc + c + e]), s2 = to_f(cs[2 * Cc + c + e]);
@@ -294,62 +347,53 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_multi_kernel(DecodeArgs
     if (lane == 0) red_s[t * 3 + kind] = acc;
   }
   __syncthreads();
+  // ---- q and k normalised in place (the products the one-token kernel forms in registers)
+  for (int i = tid; i < k * 2 * d; i += kDecodeThreads) {
+    const int t = i / (2 * d), c = i % (2 * d);
+    const float r = c < d ? a.q_scale * rsqrtf(red_s[t * 3] + a.l2_eps)
+                          : rsqrtf(red_s[t * 3 + 1] + a.l2_eps);
+    y_s[t * (2 + R) * d + c] *= r;
+  }
+  __syncthreads();
 
-  // ---- state pass: each batch of rows takes the k updates in registers
+  // ---- state pass: each batch of row quads takes the k updates in registers, next in flight
   for (int bt = 0; bt < nbatch; ++bt) {
-    const int r0 = warp * rows_per_warp + bt * kRowBatch;
+    const int r0 = warp * rows_per_warp + bt * kBatch;
+    if (bt + 1 < nbatch) {
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) RP::load(nxt[q], S + row_off(r0 + kBatch + 4 * q + grp), sub);
+    }
+    float f[kQ][16];
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) RP::unpack(cur[q], f[q]);
     for (int t = 0; t < k; ++t) {
       const float* yt = y_s + t * (2 + R) * d;
       const float rq = a.q_scale * rsqrtf(red_s[t * 3] + a.l2_eps);
       const float rk = rsqrtf(red_s[t * 3 + 1] + a.l2_eps);
       const float kq = red_s[t * 3 + 2] * rq * rk;
-      float kreg[4], qreg[4];
+      float kn[16], qn[16];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        kreg[j] = yt[d + 4 * lane + j] * rk;
-        qreg[j] = yt[4 * lane + j] * rq;
-      }
-      float dk[kRowBatch], dq[kRowBatch];
-#pragma unroll
-      for (int i = 0; i < kRowBatch; ++i) {
-        const float4 f = sv[i];
-        dk[i] = f.x * kreg[0] + f.y * kreg[1] + f.z * kreg[2] + f.w * kreg[3];
-        dq[i] = f.x * qreg[0] + f.y * qreg[1] + f.z * qreg[2] + f.w * qreg[3];
+      for (int m = 0; m < 4; ++m) {
+        const float4 kv = *reinterpret_cast<const float4*>(yt + d + 4 * sub + 32 * m);
+        const float4 qv = *reinterpret_cast<const float4*>(yt + 4 * sub + 32 * m);
+        kn[4 * m] = kv.x, kn[4 * m + 1] = kv.y, kn[4 * m + 2] = kv.z, kn[4 * m + 3] = kv.w;
+        qn[4 * m] = qv.x, qn[4 * m + 1] = qv.y, qn[4 * m + 2] = qv.z, qn[4 * m + 3] = qv.w;
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-        for (int i = 0; i < kRowBatch; ++i) {
-          dk[i] += __shfl_xor_sync(0xffffffffu, dk[i], o);
-          dq[i] += __shfl_xor_sync(0xffffffffu, dq[i], o);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < kRowBatch; ++i) {
-        const int gr = r0 + i, hr = gr / d, v = gr % d;
-        const int h = hk * R + hr;
-        const float alpha = expf(__ldg(a.g + ((size_t)b * k + t) * a.Hv + h));
-        const float beta = __ldg(a.beta + ((size_t)b * k + t) * a.Hv + h);
-        const float vv = yt[(2 + hr) * d + v];
-        const float u = beta * (vv - alpha * dk[i]);
-        if (lane == 0) o_s[(t * R + hr) * d + v] = alpha * dq[i] + u * kq;
-        const float4 f = sv[i];
-        float4 nv;
-        nv.x = alpha * f.x + u * kreg[0];
-        nv.y = alpha * f.y + u * kreg[1];
-        nv.z = alpha * f.z + u * kreg[2];
-        nv.w = alpha * f.w + u * kreg[3];
-        sv[i] = nv;
+      for (int q = 0; q < kQ; ++q) {
+        const int gr = r0 + 4 * q + grp, hr = gr / d;
+        const float2 ab = ab_s[t * R + hr];
+        const float o = row_update(f[q], kn, qn, ab.x, ab.y, yt[(2 + hr) * d + gr % d], kq);
+        if (sub == 0) o_s[t * R * d + gr] = o;
         if (snaps)
-          IO::store(snaps + ((((size_t)b * k + t) * a.Hv + h) * d + v) * d + 4 * lane, nv);
+          RP::store(snaps + (((size_t)b * k + t) * a.Hv + hk * R) * d * d + (size_t)gr * d, sub,
+                    f[q]);
       }
     }
 #pragma unroll
-    for (int i = 0; i < kRowBatch; ++i) IO::store(S + row_off(r0 + i), sv[i]);
-    if (bt + 1 < nbatch) {
+    for (int q = 0; q < kQ; ++q) RP::store(S + row_off(r0 + 4 * q + grp), sub, f[q]);
 #pragma unroll
-      for (int i = 0; i < kRowBatch; ++i) sv[i] = IO::load(S + row_off(r0 + kRowBatch + i));
-    }
+    for (int q = 0; q < kQ; ++q) cur[q] = nxt[q];
   }
   __syncthreads();
   // ---- gated RMSNorm (or plain output) per token, one warp per (token, value head)
@@ -405,11 +449,11 @@ cudaError_t launch_decode_multi(bool bf16, const gdn::DecodeArgs& a, int k, floa
                                 cudaStream_t s) {
   if (a.B == 0 || k == 0) return cudaSuccess;
   const int R = a.Hv / a.Hk;
-  const size_t smem = ((size_t)k * (2 + 2 * R) * gdn::kHeadDim + 3 * k) * sizeof(float);
+  const size_t smem = (gdn::multi_smem_floats(k, R) + 1) * sizeof(float);
   static bool attr = false;
   if (!attr) {  // the largest request: kMaxTokens tokens, kMaxR value heads per key head
-    const int most = (gdn::kMaxTokens * (2 + 2 * gdn::kMaxR) * gdn::kHeadDim + 3 * gdn::kMaxTokens) *
-                     (int)sizeof(float);
+    const int most =
+        (int)((gdn::multi_smem_floats(gdn::kMaxTokens, gdn::kMaxR) + 1) * sizeof(float));
     cudaError_t e = cudaFuncSetAttribute(gdn::decode_multi_kernel<__nv_bfloat16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     if (e == cudaSuccess)

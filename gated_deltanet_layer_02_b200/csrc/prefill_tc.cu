@@ -483,7 +483,7 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int j = j0 + e;
-          adiag[e] = (j < i) ? bi * __expf(Gi - G_s[j]) * v[e] : 0.f;
+          adiag[e] = lower_decay(j < i, Gi, G_s[j], bi * v[e]);
         }
       }
     }
@@ -1332,8 +1332,8 @@ __global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int j = j0 + e;
-          const float p0 = (any_lower && j <= i) ? __expf(Gi - G_s[j]) * v[e] : 0.f;
-          const float p1 = (any_lower && j + 1 <= i) ? __expf(Gi - G_s[j + 1]) * v[e + 1] : 0.f;
+          const float p0 = lower_decay(any_lower && j <= i, Gi, G_s[j], v[e]);
+          const float p1 = lower_decay(any_lower && j + 1 <= i, Gi, G_s[j + 1], v[e + 1]);
           pp[cc * 16 + e / 2] = pack_bf16x2(p0, p1);
         }
       }
@@ -1450,15 +1450,15 @@ constexpr uint32_t kOpStage = 98304;                        // Q | K-then-S^T | 
 constexpr uint32_t kOpQ = 0, kOpKS = 32768, kOpU = 65536;   // offsets inside a stage
 constexpr uint32_t kOpEnd = 2 * kOpStage;                   // 196608
 constexpr uint32_t kOutPSmem = kOpEnd + 1024 + 2048;
-constexpr uint32_t kColPQ = 0, kColO0 = 128;                // O buffer b at 128 + 128 b
+constexpr uint32_t kColPQ0 = 0, kColO0 = 256;  // P|Q^ buffer b at 128 b, O buffer b at 256 + 128 b
 
 struct OutPCtl {
   uint64_t* qk_full;      // [2]
   uint64_t* u_full;       // [2]
   uint64_t* s_full;       // [2]
   uint64_t* stage_empty;  // [2]
-  uint64_t* gram_done;
-  uint64_t* pq_ready;
+  uint64_t* gram_done;    // [2]
+  uint64_t* pq_ready;     // [2]
   uint64_t* o_full;       // [2]
   uint64_t* o_empty;      // [2]
   uint64_t* drain;        // products in flight after an abort
@@ -1474,11 +1474,11 @@ struct OutPCtl {
     s_full = b + 4;
     stage_empty = b + 6;
     gram_done = b + 8;
-    pq_ready = b + 9;
-    o_full = b + 10;
-    o_empty = b + 12;
-    drain = b + 14;
-    tslot = reinterpret_cast<uint32_t*>(b + 15);
+    pq_ready = b + 10;
+    o_full = b + 12;
+    o_empty = b + 14;
+    drain = b + 16;
+    tslot = reinterpret_cast<uint32_t*>(b + 17);
     abort = reinterpret_cast<int*>(tslot + 1);
     G_s = reinterpret_cast<float*>(sm + kOpEnd + 256);
     F_s = G_s + kC;
@@ -1516,9 +1516,9 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
       mbar_init(ctl.stage_empty + b, 1);
       mbar_init(ctl.o_full + b, 1);
       mbar_init(ctl.o_empty + b, 128);
+      mbar_init(ctl.gram_done + b, 1);
+      mbar_init(ctl.pq_ready + b, 128);
     }
-    mbar_init(ctl.gram_done, 1);
-    mbar_init(ctl.pq_ready, 128);
     mbar_init(ctl.drain, 1);
     *ctl.abort = 0;
     fence_barrier_init();
@@ -1572,24 +1572,29 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------------------- MMA issue
+    // Q K^T of unit i + 1 goes out before O of unit i (two P|Q^ buffers), so that group A works
+    // on the next unit while the current one's products run
     if (lane == 0) {
+      auto gram = [&](int i) -> bool {
+        const int st = i & 1;
+        if (!wait_role(ctl.qk_full + st, (i >> 1) & 1, abort, a.wait_ns)) return false;
+        stamp(1, i, 0);
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(sm + st * kOpStage + kOpQ);
+        const uint32_t sK = smem_u32(sm + st * kOpStage + kOpKS);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tmem + kColPQ0 + st * 128, desc_kmajor(sQ, kk, kTile),
+                   desc_kmajor(sK, kk, kTile), idesc_bf16(128, 128, false, false), kk > 0);
+        mma_commit(ctl.gram_done + st);
+        return true;
+      };
+      if (count > 0) ok = gram(0);
       for (int i = 0; i < count && ok; ++i) {
         const int u = u0 + i, c = a.c0 + u / Hv, h = u % Hv;
         const int st = i & 1;
-        const uint32_t sQ = smem_u32(sm + st * kOpStage + kOpQ);
-        const uint32_t sKS = smem_u32(sm + st * kOpStage + kOpKS);
-        const uint32_t sU = smem_u32(sm + st * kOpStage + kOpU);
-        ok = wait_role(ctl.qk_full + st, (i >> 1) & 1, abort, a.wait_ns);
-        if (!ok) break;
-        stamp(1, i, 0);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tmem + kColPQ, desc_kmajor(sQ, kk, kTile), desc_kmajor(sKS, kk, kTile),
-                   idesc_bf16(128, 128, false, false), kk > 0);
-        mma_commit(ctl.gram_done);
-        // K is consumed once the product completes: S^T of the unit into its place
-        ok = wait_role(ctl.gram_done, i & 1, abort, a.wait_ns);
+        // K of unit i is consumed once its product completes: S^T into its place at once
+        ok = wait_role(ctl.gram_done + st, (i >> 1) & 1, abort, a.wait_ns);
         if (!ok) break;
         const int rowV = (c * Hv + h) * kC;
         uint8_t* ks = sm + st * kOpStage + kOpKS;
@@ -1597,22 +1602,25 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
         tma_load_2d(ks, &mapS, ctl.s_full + st, 0, rowV);
         tma_load_2d(ks + kTile, &mapS, ctl.s_full + st, 64, rowV);
         last_s = i;
-        ok = wait_role(ctl.pq_ready, i & 1, abort, a.wait_ns) &&
+        // the next unit's product, so that group A can start on it
+        if (i + 1 < count && !(ok = gram(i + 1))) break;
+        ok = wait_role(ctl.pq_ready + st, (i >> 1) & 1, abort, a.wait_ns) &&
              wait_role(ctl.s_full + st, (i >> 1) & 1, abort, a.wait_ns) &&
              wait_role(ctl.u_full + st, (i >> 1) & 1, abort, a.wait_ns) &&
              (i < 2 || wait_role(ctl.o_empty + st, ((i >> 1) - 1) & 1, abort, a.wait_ns));
         if (!ok) break;
         stamp(1, i, 1);
         tc_fence_after();
-        const uint32_t colO = kColO0 + st * 128;
+        const uint32_t sKS = smem_u32(ks), sU = smem_u32(sm + st * kOpStage + kOpU);
+        const uint32_t colO = kColO0 + st * 128, colPQ = kColPQ0 + st * 128;
         constexpr uint32_t id = idesc_bf16(128, 128, false, true);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + colO, tmem + kColPQ + 64 + kk * 8, desc_mnmajor(sKS, kk, kTile), id,
+          mma_bf16_ts(tmem + colO, tmem + colPQ + 64 + kk * 8, desc_mnmajor(sKS, kk, kTile), id,
                       kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + colO, tmem + kColPQ + kk * 8, desc_mnmajor(sU, kk, kTile), id, 1);
+          mma_bf16_ts(tmem + colO, tmem + colPQ + kk * 8, desc_mnmajor(sU, kk, kTile), id, 1);
         mma_commit(ctl.o_full + st);
         mma_commit(ctl.stage_empty + st);
       }
@@ -1639,7 +1647,7 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
       bar_sync_n(1, 128);
       ctl.F_s[i_row] = __expf(ctl.G_s[i_row | 31] - ctl.G_s[i_row]);
       // one decision for the whole group (its named barriers need all 128 threads)
-      const bool got = wait_role(ctl.gram_done, i & 1, abort, a.wait_ns);
+      const bool got = wait_role(ctl.gram_done + st, (i >> 1) & 1, abort, a.wait_ns);
       if (bar_or_n(1, 128, !got)) {
         ok = false;
         break;
@@ -1647,57 +1655,77 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
       if (i_row == 0) stamp(2, i, 0);
       tc_fence_after();
       const float Gi = ctl.G_s[i_row];
-      uint32_t pp[64], qq[64];
       const int rq = i_row >> 5;  // row block of this thread (warp-uniform)
-#pragma unroll
+      const uint32_t colPQ = kColPQ0 + st * 128;
+      // P block jb (bf16 pairs) goes to columns 16 jb.., over fp32 gram columns this thread has
+      // already read (the gram block jb starts at column 32 jb); loops kept rolled so that the
+      // code stays small (four roles share each SM sub-partition's instruction cache)
+#pragma unroll 1
       for (int jb = 0; jb < 4; ++jb) {
         const int j0 = jb * 32;
+        uint32_t p16[16];
         if (jb > rq) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pp[jb * 16 + e] = 0u;
-          continue;
-        }
-        float v[32];
-        tmem_ld32(lane_addr + kColPQ + j0, v);
-        tmem_ld_wait();
-        if (jb < rq) {
-          // every j < every i: exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31
-          const float rf = __expf(Gi - ctl.G_s[j0 + 31]);
-#pragma unroll
-          for (int e = 0; e < 32; e += 2)
-            pp[jb * 16 + e / 2] = pack_bf16x2(rf * ctl.F_s[j0 + e] * v[e],
-                                              rf * ctl.F_s[j0 + e + 1] * v[e + 1]);
+          for (int e = 0; e < 16; ++e) p16[e] = 0u;
         } else {
+          float v[32];
+          if (jb == 0 && i_row == 96) stamp(6, i, 0);
+          tmem_ld32(lane_addr + colPQ + j0, v);
+          tmem_ld_wait();
+          if (jb == 0 && i_row == 96) stamp(6, i, 1);
+          if (jb < rq) {
+            // every j < every i: exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31
+            const float rf = __expf(Gi - ctl.G_s[j0 + 31]);
+            const float4* F4 = reinterpret_cast<const float4*>(ctl.F_s + j0);
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int j = j0 + e;
-            const float p0 = j <= i_row ? __expf(Gi - ctl.G_s[j]) * v[e] : 0.f;
-            const float p1 = j + 1 <= i_row ? __expf(Gi - ctl.G_s[j + 1]) * v[e + 1] : 0.f;
-            pp[jb * 16 + e / 2] = pack_bf16x2(p0, p1);
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 f = F4[e4];
+              p16[2 * e4] = pack_bf16x2(rf * f.x * v[4 * e4], rf * f.y * v[4 * e4 + 1]);
+              p16[2 * e4 + 1] = pack_bf16x2(rf * f.z * v[4 * e4 + 2], rf * f.w * v[4 * e4 + 3]);
+            }
+          } else {
+            const float4* G4 = reinterpret_cast<const float4*>(ctl.G_s + j0);
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 gj = G4[e4];
+              const int j = j0 + 4 * e4;
+              p16[2 * e4] = pack_bf16x2(lower_decay(j <= i_row, Gi, gj.x, v[4 * e4]),
+                                        lower_decay(j + 1 <= i_row, Gi, gj.y, v[4 * e4 + 1]));
+              p16[2 * e4 + 1] = pack_bf16x2(lower_decay(j + 2 <= i_row, Gi, gj.z, v[4 * e4 + 2]),
+                                            lower_decay(j + 3 <= i_row, Gi, gj.w, v[4 * e4 + 3]));
+            }
           }
         }
+        if (stamps && i_row == 96 && i < 8) stamps[512 + i * 16 + 2 * jb] = global_timer_ns();
+        tmem_st16(lane_addr + colPQ + jb * 16, p16);
+        if (stamps && i_row == 96 && i < 8) stamps[512 + i * 16 + 2 * jb + 1] = global_timer_ns();
       }
+      if (i_row == 96) stamp(4, i, 0);
+      // Q^ = e^(G_i) Q row into columns 64.. (the gram columns there are read by now)
       const float eg = __expf(Gi);
       const uint8_t* Qs = sm + st * kOpStage + kOpQ;
+#pragma unroll 1
+      for (int qb = 0; qb < 4; ++qb) {
+        uint32_t q16[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const uint4 u4 =
-            *reinterpret_cast<const uint4*>(Qs + (q >> 3) * kTile + sw128_off(i_row, q & 7));
-        const __nv_bfloat162* hq = reinterpret_cast<const __nv_bfloat162*>(&u4);
+        for (int q = 0; q < 4; ++q) {
+          const int c16 = qb * 4 + q;  // 16-byte chunk of the row (8 elements)
+          const uint4 u4 =
+              *reinterpret_cast<const uint4*>(Qs + (c16 >> 3) * kTile + sw128_off(i_row, c16 & 7));
+          const __nv_bfloat162* hq = reinterpret_cast<const __nv_bfloat162*>(&u4);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(hq[e]);
-          qq[q * 4 + e] = pack_bf16x2(f.x * eg, f.y * eg);
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hq[e]);
+            q16[q * 4 + e] = pack_bf16x2(f.x * eg, f.y * eg);
+          }
         }
+        tmem_st16(lane_addr + colPQ + 64 + qb * 16, q16);
+        if (stamps && i_row == 96 && i < 8) stamps[640 + i * 8 + qb] = global_timer_ns();
       }
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        tmem_st32(lane_addr + kColPQ + q * 32, *reinterpret_cast<float(*)[32]>(pp + q * 32));
-        tmem_st32(lane_addr + kColPQ + 64 + q * 32, *reinterpret_cast<float(*)[32]>(qq + q * 32));
-      }
+      if (i_row == 96) stamp(4, i, 1);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ctl.pq_ready);  // Q of the stage is read, P and Q^ are in TMEM
+      mbar_arrive(ctl.pq_ready + st);  // Q of the stage is read, P and Q^ are in TMEM
       if (i_row == 0) stamp(2, i, 1);
     }
     if (!ok) *abort = 1;
@@ -1706,10 +1734,15 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
     const int i_row = tid - 128;
     const uint32_t lane_addr = tmem_at(tmem, (warp & 3) * 32, 0);
     uint4 zreg[16];
-    ChunkInfo ci_next{};
-    auto prefetch = [&](int i) {  // chunk entry and z row of unit i
-      const int u = u0 + i, c = a.c0 + u / Hv, h = u % Hv;
-      ci_next = a.ws.chunks[c];
+    // chunk entries two units ahead, z rows one unit ahead (two dependent loads otherwise)
+    auto entry = [&](int i) {
+      ChunkInfo e{};
+      if (i < count) e = a.ws.chunks[a.c0 + (u0 + i) / Hv];
+      return e;
+    };
+    ChunkInfo ci_next = entry(0), ci_next2 = entry(1);
+    auto prefetch = [&](int i) {  // z row of unit i (its chunk entry is ci_next)
+      const int h = (u0 + i) % Hv;
       if (a.z && i_row < ci_next.L) {
         const uint4* zp =
             reinterpret_cast<const uint4*>(a.z + ((size_t)(ci_next.t0 + i_row) * Hv + h) * kD);
@@ -1721,6 +1754,8 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
     for (int i = 0; i < count; ++i) {
       const int u = u0 + i, h = u % Hv;
       const ChunkInfo ci = ci_next;
+      ci_next = ci_next2;
+      ci_next2 = entry(i + 2);
       const int st = i & 1;
       ok = wait_role(ctl.o_full + st, (i >> 1) & 1, abort, a.wait_ns);
       if (!ok) break;
@@ -1733,8 +1768,10 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float v[32];
+          if (q == 0 && i_row == 0) stamp(5, i, 0);
           tmem_ld32(lane_addr + colO + q * 32, v);
           tmem_ld_wait();
+          if (q == 0 && i_row == 0) stamp(5, i, 1);
 #pragma unroll
           for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
         }

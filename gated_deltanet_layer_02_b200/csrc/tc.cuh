@@ -191,6 +191,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -251,6 +260,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128-B-swizzled row tile.
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
   return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+// x exp(G_i - G_j) where keep (the lower triangle of a chunk), else 0, as a select rather than
+// a branch (every lane holds its own row i, so the condition differs across the warp).  The
+// exponent is clamped at 0: on the kept side it is <= 0 already (G is a running sum of
+// log-gates <= 0), on the other side the clamp keeps the discarded value finite.
+__device__ __forceinline__ float lower_decay(bool keep, float Gi, float Gj, float x) {
+  const float e = __expf(fminf(Gi - Gj, 0.f)) * x;
+  float r;
+  asm("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\tselp.f32 %0, %1, 0f00000000, p;\n\t}"
+      : "=f"(r)
+      : "f"(e), "r"((uint32_t)keep));
+  return r;
 }
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
