@@ -101,21 +101,32 @@ struct RowPart<__nv_bfloat16> {
 __device__ __forceinline__ float row_update(float (&f)[16], const float (&kn)[16],
                                             const float (&qn)[16], float alpha, float beta,
                                             float vv, float kq) {
-  float dk4[4] = {0.f, 0.f, 0.f, 0.f}, dq4[4] = {0.f, 0.f, 0.f, 0.f};
+  // packed fp32 pairs (FFMA2): two element pairs per accumulator
+  float2 dk2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 dq2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    dk4[j & 3] = fmaf(f[j], kn[j], dk4[j & 3]);
-    dq4[j & 3] = fmaf(f[j], qn[j], dq4[j & 3]);
+  for (int j = 0; j < 16; j += 2) {
+    const float2 fj = make_float2(f[j], f[j + 1]);
+    const int p = (j >> 1) & 1;
+    dk2[p] = __ffma2_rn(fj, make_float2(kn[j], kn[j + 1]), dk2[p]);
+    dq2[p] = __ffma2_rn(fj, make_float2(qn[j], qn[j + 1]), dq2[p]);
   }
-  float dk = (dk4[0] + dk4[1]) + (dk4[2] + dk4[3]), dq = (dq4[0] + dq4[1]) + (dq4[2] + dq4[3]);
+  float dk = (dk2[0].x + dk2[0].y) + (dk2[1].x + dk2[1].y);
+  float dq = (dq2[0].x + dq2[0].y) + (dq2[1].x + dq2[1].y);
 #pragma unroll
   for (int o = 4; o > 0; o >>= 1) {
     dk += __shfl_xor_sync(0xffffffffu, dk, o);
     dq += __shfl_xor_sync(0xffffffffu, dq, o);
   }
   const float u = beta * (vv - alpha * dk);
+  const float2 a2 = make_float2(alpha, alpha), u2 = make_float2(u, u);
 #pragma unroll
-  for (int j = 0; j < 16; ++j) f[j] = fmaf(alpha, f[j], u * kn[j]);
+  for (int j = 0; j < 16; j += 2) {
+    const float2 r = __ffma2_rn(u2, make_float2(kn[j], kn[j + 1]),
+                                __fmul2_rn(a2, make_float2(f[j], f[j + 1])));
+    f[j] = r.x;
+    f[j + 1] = r.y;
+  }
   return fmaf(alpha, dq, u * kq);
 }
 
@@ -347,12 +358,14 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_multi_kernel(DecodeA
     if (lane == 0) red_s[t * 3 + kind] = acc;
   }
   __syncthreads();
-  // ---- q and k normalised in place (the products the one-token kernel forms in registers)
+  // ---- q and k normalised in place, and k.q of the normalised vectors (the values the
+  // one-token kernel forms in registers, by the same expressions)
   for (int i = tid; i < k * 2 * d; i += kDecodeThreads) {
     const int t = i / (2 * d), c = i % (2 * d);
-    const float r = c < d ? a.q_scale * rsqrtf(red_s[t * 3] + a.l2_eps)
-                          : rsqrtf(red_s[t * 3 + 1] + a.l2_eps);
-    y_s[t * (2 + R) * d + c] *= r;
+    const float rq = a.q_scale * rsqrtf(red_s[t * 3] + a.l2_eps);
+    const float rk = rsqrtf(red_s[t * 3 + 1] + a.l2_eps);
+    y_s[t * (2 + R) * d + c] *= c < d ? rq : rk;
+    if (c == 0) red_s[t * 3 + 2] = red_s[t * 3 + 2] * rq * rk;  // read by no other thread here
   }
   __syncthreads();
 
@@ -368,9 +381,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_multi_kernel(DecodeA
     for (int q = 0; q < kQ; ++q) RP::unpack(cur[q], f[q]);
     for (int t = 0; t < k; ++t) {
       const float* yt = y_s + t * (2 + R) * d;
-      const float rq = a.q_scale * rsqrtf(red_s[t * 3] + a.l2_eps);
-      const float rk = rsqrtf(red_s[t * 3 + 1] + a.l2_eps);
-      const float kq = red_s[t * 3 + 2] * rq * rk;
+      const float kq = red_s[t * 3 + 2];
       float kn[16], qn[16];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
