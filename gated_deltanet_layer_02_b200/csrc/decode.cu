@@ -17,6 +17,7 @@
 // of a row is read by one group of eight lanes with one 16-byte load each.
 #include "args.cuh"
 #include "common.cuh"
+#include "tc.cuh"
 
 namespace gdn {
 
@@ -130,6 +131,13 @@ __device__ __forceinline__ float row_update(float (&f)[16], const float (&kn)[16
   return fmaf(alpha, dq, u * kq);
 }
 
+// One step of the causal conv (width 4, history s0 oldest .. s2 newest, input xv) and the SiLU;
+// the one- and k-token kernels both call it, with the products in this fixed order.
+__device__ __forceinline__ float conv_silu(const float (&w)[4], float s0, float s1, float s2,
+                                           float xv) {
+  return silu_f(fmaf(w[3], xv, fmaf(w[2], s2, fmaf(w[1], s1, w[0] * s0))));
+}
+
 // Input channel of position gch of the conv outputs of key head hk (q | k | v_0..v_{R-1}).
 __device__ __forceinline__ int channel_of(int gch, int hk, int R, int Hk) {
   const int grp = gch / kHeadDim, off = gch % kHeadDim;
@@ -190,8 +198,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
       const float s0 = to_f(cs[c + e]), s1 = to_f(cs[Cc + c + e]), s2 = to_f(cs[2 * Cc + c + e]);
       const T xt = x[c + e];
       const T* wr = w + (size_t)(c + e) * 4;
-      const float acc = to_f(wr[0]) * s0 + to_f(wr[1]) * s1 + to_f(wr[2]) * s2 + to_f(wr[3]) * to_f(xt);
-      y_s[gch + e] = silu_f(acc);
+      const float wf[4] = {to_f(wr[0]), to_f(wr[1]), to_f(wr[2]), to_f(wr[3])};
+      y_s[gch + e] = conv_silu(wf, s0, s1, s2, to_f(xt));
       cs[c + e] = from_f<T>(s1);
       cs[Cc + c + e] = from_f<T>(s2);
       cs[2 * Cc + c + e] = xt;
@@ -273,13 +281,24 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_kernel(DecodeArgs a)
 // products), so the results equal k calls of the one-token step.  Per-token constants (the
 // normalised q and k, alpha, beta) are set up once in shared memory before the state pass.
 // With `snaps` set, the state after every token is stored as well ([B, k, Hv, d, d] fp32), so
-// that a caller that accepts only the first m tokens can take snapshot m - 1.  Dynamic shared
-// memory: per token (2 + R) d conv outputs (q and k normalised in place), R d outputs, three
-// norms and R (alpha, beta) pairs.
+// that a caller that accepts only the first m tokens can take snapshot m - 1.
+// The rows stream through shared memory: each warp keeps kMultiStages batches of 8 rows (4 KB,
+// contiguous in the state) in flight as bulk copies (cp.async.bulk, no registers held while
+// they are in flight), so that the k token updates of one batch overlap the loads of the next
+// ones; the new rows go back to HBM from registers.  Dynamic shared memory: the warps' stages
+// and their mbarriers, then per token (2 + R) d conv outputs (q and k normalised in place),
+// R d outputs, three norms and R (alpha, beta) pairs.
 constexpr int kMaxTokens = 8;
+constexpr int kMultiStages = 2;
+constexpr int kMultiBatchBytes = 8 * kHeadDim * 4;  // 8 rows of fp32
+constexpr size_t kMultiRingBytes =
+    (size_t)(kDecodeThreads / 32) * kMultiStages * kMultiBatchBytes + 128;  // + mbarriers
 
 __host__ __device__ constexpr size_t multi_smem_floats(int k, int R) {
   return (size_t)k * (2 + 2 * R) * kHeadDim + 3 * k + 2 * k * R;
+}
+__host__ __device__ constexpr size_t multi_smem_bytes(int k, int R) {
+  return kMultiRingBytes + (multi_smem_floats(k, R) + 1) * sizeof(float);
 }
 
 template <typename T>
@@ -297,7 +316,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_multi_kernel(DecodeA
     if (tid == 0) report_status(a.status, GDN_ERR_INVALID_ARG);
     return;
   }
-  extern __shared__ float dsm[];
+  extern __shared__ __align__(128) uint8_t dsm_raw[];
+  uint8_t* ring = dsm_raw + (size_t)warp * kMultiStages * kMultiBatchBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dsm_raw + kMultiRingBytes - 128) + warp * kMultiStages;
+  float* dsm = reinterpret_cast<float*>(dsm_raw + kMultiRingBytes);
   float* y_s = dsm;                          // [k][(2 + R) d]: q | k | v_0..v_{R-1}
   float* o_s = y_s + k * (2 + R) * d;        // [k][R d]
   float* red_s = o_s + k * R * d;            // [k][3]: |q|^2, |k|^2, q.k
@@ -312,32 +334,53 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_multi_kernel(DecodeA
   const int nbatch = rows_per_warp / kBatch;
   float* S = static_cast<float*>(a.S);
   auto row_off = [&](int gr) { return ((size_t)slot * a.Hv + hk * R) * d * d + (size_t)gr * d; };
-  RP::Raw cur[kQ], nxt[kQ];
-#pragma unroll
-  for (int q = 0; q < kQ; ++q) RP::load(cur[q], S + row_off(warp * rows_per_warp + 4 * q + grp), sub);
+  // the first stages of this warp's rows go out before the conv (they do not depend on it)
+  auto issue = [&](int bt) {  // lane 0: batch bt of the warp into its stage
+    const int st = bt % kMultiStages;
+    mbar_arrive_expect_tx(bars + st, kMultiBatchBytes);
+    bulk_load(ring + st * kMultiBatchBytes, S + row_off(warp * rows_per_warp + bt * kBatch),
+              kMultiBatchBytes, bars + st);
+  };
+  if (lane == 0) {
+    for (int st = 0; st < kMultiStages; ++st) mbar_init(bars + st, 1);
+    fence_barrier_init();
+    for (int bt = 0; bt < kMultiStages && bt < nbatch; ++bt) issue(bt);
+  }
+  __syncwarp();
 
   for (int i = tid; i < k * R; i += kDecodeThreads) {
     const int t = i / R, h = hk * R + i % R;
     const size_t gi = ((size_t)b * k + t) * a.Hv + h;
     ab_s[i] = make_float2(expf(a.g[gi]), a.beta[gi]);
   }
-  // ---- conv + SiLU over the k tokens, history in registers, final history written back
+  // ---- conv + SiLU over the k tokens, history in registers, final history written back.
+  // Every load of an item goes out before its first step (one memory latency per item).
   const int items = (2 + R) * d / 2;
+  const T* xb = static_cast<const T*>(a.x) + (size_t)b * k * Cc;
   for (int it = tid; it < items; it += kDecodeThreads) {
     const int gch = it * 2;
     const int c = channel_of(gch, hk, R, a.Hk);
+    T xs[kMaxTokens][2];
+#pragma unroll
+    for (int t = 0; t < kMaxTokens; ++t) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) xs[t][e] = t < k ? xb[(size_t)t * Cc + c + e] : T();
+    }
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       float s0 = to_f(cs[c + e]), s1 = to_f(cs[Cc + c + e]), s2 = to_f(cs[2 * Cc + c + e]);
       const T* wr = w + (size_t)(c + e) * 4;
+      const float wf[4] = {to_f(wr[0]), to_f(wr[1]), to_f(wr[2]), to_f(wr[3])};
       T xt = T();
-      for (int t = 0; t < k; ++t) {
-        xt = static_cast<const T*>(a.x)[((size_t)b * k + t) * Cc + c + e];
-        const float acc = to_f(wr[0]) * s0 + to_f(wr[1]) * s1 + to_f(wr[2]) * s2 + to_f(wr[3]) * to_f(xt);
-        y_s[t * (2 + R) * d + gch + e] = silu_f(acc);
-        s0 = s1;
-        s1 = s2;
-        s2 = to_f(xt);
+#pragma unroll
+      for (int t = 0; t < kMaxTokens; ++t) {
+        if (t < k) {
+          xt = xs[t][e];
+          y_s[t * (2 + R) * d + gch + e] = conv_silu(wf, s0, s1, s2, to_f(xt));
+          s0 = s1;
+          s1 = s2;
+          s2 = to_f(xt);
+        }
       }
       cs[c + e] = from_f<T>(s0);
       cs[Cc + c + e] = from_f<T>(s1);
@@ -369,16 +412,30 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_multi_kernel(DecodeA
   }
   __syncthreads();
 
-  // ---- state pass: each batch of row quads takes the k updates in registers, next in flight
-  for (int bt = 0; bt < nbatch; ++bt) {
+  // ---- state pass: each batch of row quads takes the k updates in registers
+  int issued = min(kMultiStages, nbatch), bt = 0;
+  bool ok = true;
+  for (; bt < nbatch; ++bt) {
     const int r0 = warp * rows_per_warp + bt * kBatch;
-    if (bt + 1 < nbatch) {
-#pragma unroll
-      for (int q = 0; q < kQ; ++q) RP::load(nxt[q], S + row_off(r0 + kBatch + 4 * q + grp), sub);
-    }
+    const int st = bt % kMultiStages;
+    ok = mbar_wait(bars + st, (bt / kMultiStages) & 1);
+    if (!__all_sync(0xffffffffu, ok)) break;
     float f[kQ][16];
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) RP::unpack(cur[q], f[q]);
+    for (int q = 0; q < kQ; ++q) {
+      const float* src = reinterpret_cast<const float*>(ring + st * kMultiBatchBytes) +
+                         (4 * q + grp) * d + 4 * sub;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float4 v = *reinterpret_cast<const float4*>(src + 32 * m);
+        f[q][4 * m] = v.x, f[q][4 * m + 1] = v.y, f[q][4 * m + 2] = v.z, f[q][4 * m + 3] = v.w;
+      }
+    }
+    __syncwarp();  // every lane has read the stage: it takes batch bt + kMultiStages next
+    if (lane == 0 && issued < nbatch) {
+      fence_proxy_async_smem();
+      issue(issued++);
+    }
     for (int t = 0; t < k; ++t) {
       const float* yt = y_s + t * (2 + R) * d;
       const float kq = red_s[t * 3 + 2];
@@ -403,8 +460,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_multi_kernel(DecodeA
     }
 #pragma unroll
     for (int q = 0; q < kQ; ++q) RP::store(S + row_off(r0 + 4 * q + grp), sub, f[q]);
-#pragma unroll
-    for (int q = 0; q < kQ; ++q) cur[q] = nxt[q];
+  }
+  if (bt < nbatch) {
+    // a wait ran out: report it, let the copies still in flight land (bounded), leave the rest
+    if (lane == 0) {
+      report_status(a.status, GDN_ERR_TIMEOUT);
+      for (int b2 = bt; b2 < issued; ++b2)
+        mbar_wait(bars + b2 % kMultiStages, (b2 / kMultiStages) & 1);
+    }
+    __syncwarp();
   }
   __syncthreads();
   // ---- gated RMSNorm (or plain output) per token, one warp per (token, value head)
@@ -460,11 +524,10 @@ cudaError_t launch_decode_multi(bool bf16, const gdn::DecodeArgs& a, int k, floa
                                 cudaStream_t s) {
   if (a.B == 0 || k == 0) return cudaSuccess;
   const int R = a.Hv / a.Hk;
-  const size_t smem = (gdn::multi_smem_floats(k, R) + 1) * sizeof(float);
+  const size_t smem = gdn::multi_smem_bytes(k, R);
   static bool attr = false;
   if (!attr) {  // the largest request: kMaxTokens tokens, kMaxR value heads per key head
-    const int most =
-        (int)((gdn::multi_smem_floats(gdn::kMaxTokens, gdn::kMaxR) + 1) * sizeof(float));
+    const int most = (int)gdn::multi_smem_bytes(gdn::kMaxTokens, gdn::kMaxR);
     cudaError_t e = cudaFuncSetAttribute(gdn::decode_multi_kernel<__nv_bfloat16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, most);
     if (e == cudaSuccess)
