@@ -381,6 +381,10 @@ __device__ __forceinline__ bool prep_unit(const PrefillArgs& a, const CUtensorMa
     mbar_arrive_expect_tx(bar_k, 2 * kTile);
     tma_load_2d(sm + kPrepKs, &mapK, bar_k, 0, rowK);
     tma_load_2d(sm + kPrepKs + kTile, &mapK, bar_k, 64, rowK);
+    // V is loaded once the joins have released its buffer; bring it into L2 meanwhile
+    const int rowV = (c * Hv + h) * kC;
+    tma_prefetch_2d(&mapV, 0, rowV);
+    tma_prefetch_2d(&mapV, 64, rowV);
   }
   // ---------------- gates: G = inclusive cumsum of g inside the chunk, beta
   if (warp < 4) {
@@ -1197,238 +1201,6 @@ __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(Pr
   chain_body<DV, MID>(a, mapW, mapK, blockIdx.x, sm);
 }
 
-// ----------------------------------------------------------------------------------- out
-// One CTA per (chunk, value head), 8 warps, two CTAs per SM.  Warp w reads TMEM lanes
-// 32*(w%4).. (token rows) and handles the column half w/4 of each 128-wide row.
-//   Q K^T (tcgen05, both operands from smem) -> P = mask(e^(G_i - G_j)) * Q K^T and
-//   Q^ = diag(e^G) Q, both written to TMEM as bf16 A operands -> O = Q^ S^T + P U accumulated
-//   in one TMEM region (A from TMEM, B from smem) -> z-gated RMSNorm -> bf16 output.
-// S^T is loaded into K's buffer once the gram has consumed K.
-constexpr uint32_t kOutQ = 0, kOutKS = 32768, kOutU = 65536;
-constexpr uint32_t kOutEnd = 98304;
-constexpr uint32_t kOutSmem = kOutEnd + 1024 + 4096;
-constexpr uint32_t kColQK = 0, kColP = 0, kColQh = 64, kColO = 128;  // 256 TMEM columns
-constexpr int kOutThreads = 256;
-
-
-__global__ void __launch_bounds__(kOutThreads, 2) gdn_out_kernel(
-    PrefillArgs a, const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
-    const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapU) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
-  uint64_t* bar_qk = reinterpret_cast<uint64_t*>(sm + kOutEnd);
-  uint64_t* bar_s = bar_qk + 1;
-  uint64_t* bar_u = bar_qk + 2;
-  uint64_t* bar_mma = bar_qk + 3;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bar_qk + 4);
-  float* G_s = reinterpret_cast<float*>(sm + kOutEnd + 64);   // [128]
-  float* red_s = G_s + kC;                                    // [2][128] partial sums of squares
-  float* w_s = red_s + 2 * kC;                                // [128] norm weight
-  float* F_s = w_s + kC;                                      // [128] column factors
-
-  const int c = a.c0 + blockIdx.x, h = blockIdx.y;
-  const int total_chunks = a.ws.seq_first[a.N];
-  if (c >= total_chunks) {
-    pdl_wait();
-    return;
-  }
-  const ChunkInfo ci = a.ws.chunks[c];
-  if (!GDN_IN_BOUNDS(ci.t0 >= 0 && ci.L > 0 && ci.L <= kC && ci.t0 + ci.L <= a.T, a.status)) {
-    pdl_wait();
-    return;
-  }
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int quarter = warp & 3, half = warp >> 2;
-  const int i = quarter * 32 + lane;  // token row of this thread
-  const bool valid = i < ci.L;
-  const int Hv = a.Hv;
-  const int hk = h / (Hv / a.Hk);
-  // Q, K (q/k/v kernel) and the gates (prep) are complete before the chain starts, so their
-  // loads go out at once; U comes from the chain, which thread 32 waits for
-  if (tid == 32) {
-    mbar_init(bar_qk, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_u, 1);
-    mbar_init(bar_mma, 1);
-    fence_barrier_init();
-    const int rowQK = (c * a.Hk + hk) * kC, rowV = (c * Hv + h) * kC;
-    mbar_arrive_expect_tx(bar_qk, 4 * kTile);
-    tma_load_2d(sm + kOutQ, &mapQ, bar_qk, 0, rowQK);
-    tma_load_2d(sm + kOutQ + kTile, &mapQ, bar_qk, 64, rowQK);
-    tma_load_2d(sm + kOutKS, &mapK, bar_qk, 0, rowQK);
-    tma_load_2d(sm + kOutKS + kTile, &mapK, bar_qk, 64, rowQK);
-    pdl_wait();
-    mbar_arrive_expect_tx(bar_u, 2 * kTile);
-    tma_load_2d(sm + kOutU, &mapU, bar_u, 0, rowV);
-    tma_load_2d(sm + kOutU + kTile, &mapU, bar_u, 64, rowV);
-  }
-  if (warp == 0) tmem_alloc(tslot, 256);
-  if (tid < kC) G_s[tid] = a.ws.Gw[((size_t)c * Hv + h) * kC + tid];
-  else w_s[tid - kC] = a.norm_w ? __bfloat162float(a.norm_w[tid - kC]) : 1.f;
-  uint4 zreg[8];
-  if (a.z && valid) {
-    const uint4* zp = reinterpret_cast<const uint4*>(a.z + ((size_t)(ci.t0 + i) * Hv + h) * kD +
-                                                     half * 64);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) zreg[q] = __ldg(zp + q);
-  }
-  __syncthreads();
-  tc_fence_after();
-  // column factors exp(G_m - G_j), m = last column of j's 32-column chunk (exponent <= 0);
-  // read after the barriers of the gram wait below
-  if (tid < kC) F_s[tid] = __expf(G_s[tid | 31] - G_s[tid]);
-  const uint32_t tmem = *tslot;
-  const uint32_t lane_addr = tmem_at(tmem, quarter * 32, 0);
-  const uint32_t sQ = smem_u32(sm + kOutQ), sKS = smem_u32(sm + kOutKS), sU = smem_u32(sm + kOutU);
-  bool ok = true;
-  uint32_t mma_phase = 0;
-  // ---- Q K^T
-  if (tid == 0) {
-    ok = mbar_wait(bar_qk, 0, a.wait_ns);
-    tc_fence_after();
-    if (ok) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tmem + kColQK, desc_kmajor(sQ, kk, kTile), desc_kmajor(sKS, kk, kTile),
-                 idesc_bf16(128, 128, false, false), kk > 0);
-      mma_commit(bar_mma);
-    }
-  }
-  if (__syncthreads_or(!ok)) goto done;
-  ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
-  mma_phase ^= 1;
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
-  if (tid == 0) {  // K is consumed: S^T of this chunk and value head into the same buffer
-    pdl_wait();    // returns at once: thread 32 has seen the chain complete
-    const int rowS = (c * Hv + h) * kC;
-    mbar_arrive_expect_tx(bar_s, 2 * kTile);
-    tma_load_2d(sm + kOutKS, &mapS, bar_s, 0, rowS);
-    tma_load_2d(sm + kOutKS + kTile, &mapS, bar_s, 64, rowS);
-  }
-  {
-    // ---- P row half and Q^ row half, packed bf16 pairs in registers
-    const float Gi = G_s[i];
-    uint32_t pp[32], qq[32];
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int j0 = half * 64 + cc * 32;
-      const bool any_lower = j0 <= quarter * 32 + 31;  // warp-uniform
-      const bool all_lower = j0 + 31 < quarter * 32;   // warp-uniform: every j < every i
-      float v[32];
-      if (any_lower) {
-        tmem_ld32(lane_addr + kColQK + j0, v);
-        tmem_ld_wait();
-      }
-      if (all_lower) {
-        // exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31: both exponents <= 0
-        const float rf = __expf(Gi - G_s[j0 + 31]);
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          pp[cc * 16 + e / 2] =
-              pack_bf16x2(rf * F_s[j0 + e] * v[e], rf * F_s[j0 + e + 1] * v[e + 1]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int j = j0 + e;
-          const float p0 = lower_decay(any_lower && j <= i, Gi, G_s[j], v[e]);
-          const float p1 = lower_decay(any_lower && j + 1 <= i, Gi, G_s[j + 1], v[e + 1]);
-          pp[cc * 16 + e / 2] = pack_bf16x2(p0, p1);
-        }
-      }
-    }
-    const float eg = __expf(Gi);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const int chunk16 = half * 8 + q;
-      const uint4 u = *reinterpret_cast<const uint4*>(sm + kOutQ + (chunk16 >> 3) * kTile +
-                                                      sw128_off(i, chunk16 & 7));
-      const __nv_bfloat162* hq = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(hq[e]);
-        qq[q * 4 + e] = pack_bf16x2(f.x * eg, f.y * eg);
-      }
-    }
-    // every thread has read its gram columns: the gram region may now take P and Q^
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    tmem_st32(lane_addr + kColP + half * 32, *reinterpret_cast<float(*)[32]>(pp));
-    tmem_st32(lane_addr + kColQh + half * 32, *reinterpret_cast<float(*)[32]>(qq));
-    tmem_st_wait();
-  }
-  tc_fence_before();
-  __syncthreads();
-  // ---- O = Q^ S^T + P U   (A operands from TMEM)
-  if (tid == 0) {
-    ok = mbar_wait(bar_s, 0, a.wait_ns) && mbar_wait(bar_u, 0, a.wait_ns);
-    tc_fence_after();
-    if (ok) {
-      constexpr uint32_t id = idesc_bf16(128, 128, false, true);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ts(tmem + kColO, tmem + kColQh + kk * 8, desc_mnmajor(sKS, kk, kTile), id, kk > 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ts(tmem + kColO, tmem + kColP + kk * 8, desc_mnmajor(sU, kk, kTile), id, 1);
-      mma_commit(bar_mma);
-    }
-  }
-  if (__syncthreads_or(!ok)) goto done;
-  ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
-  mma_phase ^= 1;
-  if (__syncthreads_or(!ok)) goto done;
-  tc_fence_after();
-  {
-    // ---- epilogue: gated RMSNorm, bf16 out
-    float o[64];
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      float y[32];
-      tmem_ld32(lane_addr + kColO + half * 64 + cc * 32, y);
-      tmem_ld_wait();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) o[cc * 32 + e] = y[e];
-    }
-    if (a.z) {
-      float ss = 0.f;
-#pragma unroll
-      for (int e = 0; e < 64; ++e) ss += o[e] * o[e];
-      red_s[half * kC + i] = ss;
-      __syncthreads();
-      const float inv = rsqrtf((red_s[i] + red_s[kC + i]) / kD + a.norm_eps);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const __nv_bfloat162* zh = reinterpret_cast<const __nv_bfloat162*>(&zreg[q]);
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const float2 zf = __bfloat1622float2(zh[e2]);
-          const int e = q * 8 + e2 * 2;
-          o[e] = o[e] * inv * w_s[half * 64 + e] * silu_fast(zf.x);
-          o[e + 1] = o[e + 1] * inv * w_s[half * 64 + e + 1] * silu_fast(zf.y);
-        }
-      }
-    }
-    if (valid) {
-      __nv_bfloat16* dst = a.out + ((size_t)(ci.t0 + i) * Hv + h) * kD + half * 64;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float o8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o8[e] = o[q * 8 + e];
-        store8(dst + q * 8, o8);
-      }
-    }
-  }
-done:
-  if (tid == 0 && !ok) report_status(a.status, GDN_ERR_TIMEOUT);
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, 256);
-}
-
 // --------------------------------------------------------------------------- out, persistent
 // The output step as a persistent, warp-specialised kernel: each CTA takes a contiguous range of
 // (chunk, value head) units and pipelines them over two shared-memory stages, so that the tiles
@@ -1566,6 +1338,9 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
         mbar_arrive_expect_tx(ctl.u_full + st, 2 * kTile);
         tma_load_2d(stage + kOpU, &mapU, ctl.u_full + st, 0, rowV);
         tma_load_2d(stage + kOpU + kTile, &mapU, ctl.u_full + st, 64, rowV);
+        // S^T is loaded into K's place once Q K^T has run; bring it into L2 meanwhile
+        tma_prefetch_2d(&mapS, 0, rowV);
+        tma_prefetch_2d(&mapS, 64, rowV);
         last_qk[st] = i;
       }
       if (!ok) *abort = 1;
@@ -2055,9 +1830,6 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
     cudaError_t e = cudaFuncSetAttribute(gdn::gdn_prep_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          gdn::kPrepSmem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(gdn::gdn_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               gdn::kOutSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(gdn::gdn_qkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                gdn::kQkvSmem);
