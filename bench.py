@@ -80,7 +80,7 @@ def load_peaks():
 # source files of each kernel family (a change to any of them invalidates its ncu traffic figure)
 KERNEL_SOURCES = {
     "prefill": ("prefill_tc.cu", "args.cuh", "common.cuh", "tc.cuh"),
-    "decode_step": ("decode.cu", "args.cuh", "common.cuh"),
+    "decode_step": ("decode.cu", "args.cuh", "common.cuh", "tc.cuh"),
 }
 
 
@@ -639,6 +639,9 @@ def main():
     ap.add_argument("--prefill-only", type=int, default=None, metavar="CONFIG",
                     help="profiling aid: only the step graph of prefill workload CONFIG (0-4), "
                          "--warmup + --steps replays, no other leg; prints its ms per step")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="profiling aid: only the decode legs (fp32 state, bf16 state, 4-token "
+                         "calls) of the decode workload, --decode-steps steps each")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -664,6 +667,14 @@ def main():
     n = world
     if args.prefill_only is not None:
         print(json.dumps(profile_prefill(args, args.prefill_only, dev, gdn)), flush=True)
+        return
+    if args.decode_only:
+        w3, s3 = inputs.CONFIGS[3], inputs.config_seed(3)
+        f32_ms = bench_decode(w3, s3, dev, gdn, args.decode_steps)[0]
+        b16_ms = bench_decode(w3, s3, dev, gdn, args.decode_steps, torch.bfloat16)[0]
+        multi_ms = bench_decode_multi(w3, s3, dev, gdn, reps=args.decode_steps)[0]
+        print(json.dumps({"workload": w3.name, "decode_ms": f32_ms, "bf16_state_ms": b16_ms,
+                          "multi_token_ms": multi_ms}), flush=True)
         return
 
     def run_prefill(idx, steps, e2e):
@@ -722,7 +733,7 @@ def main():
                                  "roofline": {"bound": "hbm", "achieved": d16_gbs / n,
                                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                               "frac": d16_gbs / n / peaks["hbm_gbs"],
-                                              "traffic": None,
+                                              "traffic": ncu_traffic("decode_step_bf16_state"),
                                               "peak_source": f"{peak_src} (copy)"},
                                  "clocks": d16_clk},
                   "multi_token": {"tokens_per_call": 4, "ms_per_call": dm_ms,
@@ -733,7 +744,7 @@ def main():
                                                "achieved": dm_bytes / (dm_ms * 1e-3) / 1e9,
                                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                                "frac": dm_bytes / (dm_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                               "traffic": None,
+                                               "traffic": ncu_traffic("decode_multi"),
                                                "peak_source": f"{peak_src} (copy)"}}}
         w1 = inputs.CONFIGS[1]
         chunk_states = bench_chunk_states(args, w1, inputs.config_seed(1), dev, gdn)

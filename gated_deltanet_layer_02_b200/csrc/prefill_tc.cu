@@ -1444,10 +1444,8 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
           for (int e = 0; e < 16; ++e) p16[e] = 0u;
         } else {
           float v[32];
-          if (jb == 0 && i_row == 96) stamp(6, i, 0);
           tmem_ld32(lane_addr + colPQ + j0, v);
           tmem_ld_wait();
-          if (jb == 0 && i_row == 96) stamp(6, i, 1);
           if (jb < rq) {
             // every j < every i: exp(G_i - G_j) = exp(G_i - G_m) exp(G_m - G_j), m = j0 + 31
             const float rf = __expf(Gi - ctl.G_s[j0 + 31]);
@@ -1471,9 +1469,7 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
             }
           }
         }
-        if (stamps && i_row == 96 && i < 8) stamps[512 + i * 16 + 2 * jb] = global_timer_ns();
         tmem_st16(lane_addr + colPQ + jb * 16, p16);
-        if (stamps && i_row == 96 && i < 8) stamps[512 + i * 16 + 2 * jb + 1] = global_timer_ns();
       }
       if (i_row == 96) stamp(4, i, 0);
       // Q^ = e^(G_i) Q row into columns 64.. (the gram columns there are read by now)
@@ -1495,7 +1491,6 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
           }
         }
         tmem_st16(lane_addr + colPQ + 64 + qb * 16, q16);
-        if (stamps && i_row == 96 && i < 8) stamps[640 + i * 8 + qb] = global_timer_ns();
       }
       if (i_row == 96) stamp(4, i, 1);
       tmem_st_wait();
@@ -1538,9 +1533,11 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
       tc_fence_after();
       const uint32_t colO = kColO0 + st * 128;
       float inv = 1.f;
+      // loops kept rolled (the code stays small: four roles share each SM sub-partition's
+      // instruction cache); the z words of column block q are picked by selects
       if (a.z) {
         float ss = 0.f;
-#pragma unroll
+#pragma unroll 1
         for (int q = 0; q < 4; ++q) {
           float v[32];
           if (q == 0 && i_row == 0) stamp(5, i, 0);
@@ -1554,15 +1551,19 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
       }
       __nv_bfloat16* dst = a.out + ((size_t)(ci.t0 + i_row) * Hv + h) * kD;
       const bool valid = i_row < ci.L;
-#pragma unroll
+#pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float v[32];
         tmem_ld32(lane_addr + colO + q * 32, v);
         tmem_ld_wait();
         if (a.z) {
+          uint4 zq[4];
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            zq[r] = q == 0 ? zreg[r] : q == 1 ? zreg[4 + r] : q == 2 ? zreg[8 + r] : zreg[12 + r];
 #pragma unroll
           for (int r = 0; r < 4; ++r) {
-            const __nv_bfloat162* zh = reinterpret_cast<const __nv_bfloat162*>(&zreg[q * 4 + r]);
+            const __nv_bfloat162* zh = reinterpret_cast<const __nv_bfloat162*>(&zq[r]);
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
               const float2 zf = __bfloat1622float2(zh[e2]);
