@@ -25,7 +25,7 @@ cudaError_t launch_decode_multi(bool bf16, const gdn::DecodeArgs& a, int k, floa
 cudaError_t launch_recurrent_f32(const gdn::RecArgs& a, cudaStream_t s);
 cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t s);
 size_t prefill_tc_workspace(int N, int T, int Hk, int Hv);
-int choose_nsplit(int N, int Hv);
+int choose_nsplit(int N, int T, int Hv);
 
 // ------------------------------------------------------------------------------ tracing
 struct TraceRec {
@@ -278,7 +278,7 @@ static int prefill_impl(const gdn_dims* dims, gdn_dtype dtype, const void* x,
   a.T = num_tokens;
   a.Hk = dims->num_k_heads;
   a.Hv = dims->num_v_heads;
-  a.nsplit = gdn_host::choose_nsplit(num_seqs, dims->num_v_heads);
+  a.nsplit = gdn_host::choose_nsplit(num_seqs, num_tokens, dims->num_v_heads);
   a.q_scale = dims->q_scale;
   a.l2_eps = dims->l2_eps;
   a.norm_eps = dims->norm_eps;

@@ -1648,17 +1648,19 @@ static cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 bl
 // the sequential chain overlaps the parallel kernels instead of following them.  The parallel
 // kernels already fill every SM (two CTAs each, bound by shared memory), so the overlap only
 // pays where the chain is long: by default the table is cut only from 512 chunks on, into
-// segments of 64.  The debug option segment_chunks sets the segment length (a value at or above
-// the chunk count gives a single launch of each kernel).
+// segments of 64 (of 128 from 1024 chunks on: at 262,144 tokens, 9.84 ms per call against 9.92
+// with 64).  The debug option segment_chunks sets the segment length (a value at or above the
+// chunk count gives a single launch of each kernel).
 struct SegPlan {
   int nseg, seg;
 };
+constexpr int kPipelineChunks = 512;  // chunk count from which a call is pipelined
 
 static SegPlan seg_plan(int N, int T) {
   const int NC = T / kC + N;
   if (T == 0 || NC <= 1) return {1, NC > 0 ? NC : 1};
   int target = debug_opts().segment_chunks;
-  if (target <= 0) target = NC >= 512 ? 64 : NC;
+  if (target <= 0) target = NC >= 2 * kPipelineChunks ? 128 : (NC >= kPipelineChunks ? 64 : NC);
   int nseg = (NC + target - 1) / target;
   if (nseg < 1) nseg = 1;
   const int seg = (NC + nseg - 1) / nseg;
@@ -1750,13 +1752,19 @@ static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW
   return e;
 }
 
-int choose_nsplit(int N, int Hv) {
+// d_v blocks per chain state.  More blocks shorten each chunk step of the chain (fewer columns
+// per CTA) but hold more SMs: a chain CTA leaves no room for an output CTA on its SM.  A call
+// that runs as one launch of each kernel wants the shortest chain (up to 4 blocks, while the
+// chains fill fewer than the SMs); a pipelined call (from 512 chunks on) overlaps the chain with
+// the parallel kernels of later segments and takes at most 2 blocks (measured at 262,144 tokens,
+// 16/32 heads: 9.84 ms per call with 2 blocks, 10.06 with 4, 12.99 with 1).
+int choose_nsplit(int N, int T, int Hv) {
   const int forced = debug_opts().chain_split;
   if (forced == 1 || forced == 2 || forced == 4) return forced;
   const int units = N * Hv;
   if (units >= 148) return 1;
   if (units * 2 >= 148) return 2;
-  return 4;
+  return T / kC + N >= kPipelineChunks ? 2 : 4;
 }
 
 // Helper streams of the pipeline, per device and host thread (a capture on one thread never
