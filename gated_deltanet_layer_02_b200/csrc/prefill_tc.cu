@@ -1898,7 +1898,11 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   auto launch_out = [&](const gdn::PrefillArgs& sa, cudaStream_t st, bool pdl) -> cudaError_t {
     // persistent: one CTA per SM at most, each taking a contiguous range of units
     const int units = (sa.c1 - sa.c0) * sa.Hv;
-    const int grid = std::max(1, std::min(units, num_sms));
+    // pipelined: the SMs that hold a chain CTA take no output CTA (shared memory), so the
+    // output kernel's contiguous ranges go to the others only
+    const int chain_ctas = a.N * a.Hv * a.nsplit;
+    const int sms = plan.nseg > 1 && 2 * chain_ctas < num_sms ? num_sms - chain_ctas : num_sms;
+    const int grid = std::max(1, std::min(units, sms));
     trace_begin("gdn_out", st);
     cudaError_t e2 = launch_k(pdl, gdn::gdn_out_persistent_kernel, dim3(grid),
                               dim3(gdn::kOutPThreads), gdn::kOutPSmem, st, sa, mQ, mK, mS, mU);
