@@ -821,8 +821,14 @@ struct ChainCfg {
 // The chain of CTA `bid` = (sequence, value head, d_v block).
 template <int DV, bool MID>
 __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorMap& mapW,
-                                           const CUtensorMap& mapK, int bid, uint8_t* sm) {
+                                           const CUtensorMap& mapK, const CUtensorMap& mapS,
+                                           const CUtensorMap& mapU, int bid, uint8_t* sm) {
   using Cfg = ChainCfg<DV, MID>;
+  // From a d_v block of 64 on (without mid-chunk states), S_c and U leave for the workspace as
+  // TMA stores of the bf16 operand tiles (whole 128-byte rows, instead of 16-byte pieces of 128
+  // rows from every thread), and the decay of the state update goes onto K (the operand tile
+  // then holds U itself): S^T += (diag(e^(G_L - G)) K)^T U.
+  constexpr bool kTmaOut = DV >= 64 && !MID;
   // the chain's own threads (the first Cfg::kThreads of the block) synchronise on barrier 1
 #define CSYNC() bar_sync_n(1, Cfg::kThreads)
 #define CSYNC_OR(x) bar_or_n(1, Cfg::kThreads, (x))
@@ -978,12 +984,14 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
       for (int q = 0; q < 4; ++q)
         st_row8_bf16(OP, kTile, k_row, (cs + gi * 32 + 8 * q) >> 3, sreg[gi] + 8 * q);
       if constexpr (!kOverlap) {
+        if constexpr (!kTmaOut) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float w8[8];
+          for (int q = 0; q < 4; ++q) {
+            float w8[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
-          store8(Srow + gi * 32 + 8 * q, w8);
+            for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
+            store8(Srow + gi * 32 + 8 * q, w8);
+          }
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e) sreg[gi][e] *= gam;
@@ -994,6 +1002,13 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     fence_proxy_async_smem();
     tc_fence_before();
     CSYNC();
+    const int row_cv = (c * a.Hv + h) * kC;  // first workspace row of (chunk, value head)
+    if (kTmaOut && tid == 0) {  // S_c (bf16) to the workspace from the operand tile
+#pragma unroll
+      for (uint32_t t = 0; t < Cfg::kOpTiles; ++t)
+        tma_store_2d(&mapS, OP + t * kTile, v0 + 64 * t, row_cv);
+      bulk_commit();
+    }
     // ---- X = W S_b^T  (M = 128 tokens, N = DV, K = d_k)
     if (tid == 0) {
       ok = mbar_wait(bar_w + wst, wphase, a.wait_ns);
@@ -1013,12 +1028,14 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     if constexpr (kOverlap) {
 #pragma unroll
       for (int gi = 0; gi < kGroups; ++gi) {
+        if constexpr (!kTmaOut) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float w8[8];
+          for (int q = 0; q < 4; ++q) {
+            float w8[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
-          store8(Srow + gi * 32 + 8 * q, w8);
+            for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
+            store8(Srow + gi * 32 + 8 * q, w8);
+          }
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e) sreg[gi][e] *= gam;
@@ -1026,9 +1043,32 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
       }
       tmem_st_wait();
     }
+    if constexpr (kTmaOut) {
+      // K^ = diag(e^(G_L - G)) K in place, once K has landed: this thread's token row, the
+      // 64 d_k columns of its half (two threads per row)
+      const bool k_ok = mbar_wait(bar_k, ci & 1, a.wait_ns);
+      ok = ok && k_ok;
+      if (k_ok) {
+        const float dec = __expf(Gl_cur - Gi_cur);
+        uint8_t* kt = sm + Cfg::kK + (tid >> 7) * kTile;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint4* p = reinterpret_cast<uint4*>(kt + sw128_off(k_row, q));
+          uint4 u = *p;
+          __nv_bfloat162* hv = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(hv[e]);
+            hv[e] = __floats2bfloat162_rn(f.x * dec, f.y * dec);
+          }
+          *p = u;
+        }
+      }
+    }
     if (ci + 1 < nch) load_chunk_rows(ci + 1, ut_nxt, Gi_nxt, Gl_nxt, Gm_nxt, L_nxt);
     if ((failed = CSYNC_OR(!ok))) break;
     ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
+    if (kTmaOut && tid == 0) bulk_wait_reads();  // the S_c store has read the operand tile
     if ((failed = CSYNC_OR(!ok))) break;
     mma_phase ^= 1;
     mma_pending = false;
@@ -1064,14 +1104,14 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
             u8[2 * e2 + 1] = f.y - v[8 * q + 2 * e2 + 1];
           }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) h8[e] = u8[e] * dec;
+          for (int e = 0; e < 8; ++e) h8[e] = kTmaOut ? u8[e] : u8[e] * dec;
           st_row8_bf16(OP, kTile, k_row, (cs >> 3) + vq, h8);
           if (MID && k_row < 64) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) h8[e] = u8[e] * decm;
             st_row8_bf16(sm + Cfg::kOpMid, kTile, k_row, (cs >> 3) + vq, h8);
           }
-          if constexpr (!kOverlap) {
+          if constexpr (!kOverlap && !kTmaOut) {
             float w8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) w8[e] = u8[e];
@@ -1083,7 +1123,13 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     fence_proxy_async_smem();
     tc_fence_before();
     CSYNC();
-    // ---- S^T += K^T U^  (M = d_k, N = DV, K = tokens)
+    if (kTmaOut && tid == 0) {  // U (bf16) to the workspace from the operand tile
+#pragma unroll
+      for (uint32_t t = 0; t < Cfg::kOpTiles; ++t)
+        tma_store_2d(&mapU, OP + t * kTile, v0 + 64 * t, row_cv);
+      bulk_commit();
+    }
+    // ---- S^T += K^T U^  (M = d_k, N = DV, K = tokens); with kTmaOut: K^^T U
     if (tid == 0) {
       ok = mbar_wait(bar_k, ci & 1, a.wait_ns);
       tc_fence_after();
@@ -1108,7 +1154,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
       }
     }
     // while the state update runs: U to the workspace
-    if constexpr (kOverlap) {
+    if constexpr (kOverlap && !kTmaOut) {
 #pragma unroll
       for (int q = 0; q < kCPT / 8; ++q) {
         float u8[8];
@@ -1119,6 +1165,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     }
     if ((failed = CSYNC_OR(!ok))) break;
     ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
+    if (kTmaOut && tid == 0) bulk_wait_reads();  // the U store has read the operand tile
     if ((failed = CSYNC_OR(!ok))) break;
     mma_phase ^= 1;
     mma_pending = false;
@@ -1183,6 +1230,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     for (int j = k_done; j < k_issued; ++j) mbar_wait(bar_k, j & 1, a.wait_ns);
     if (mma_pending) mbar_wait(bar_mma, mma_phase, a.wait_ns);
   }
+  if (kTmaOut && tid == 0) bulk_wait_all();  // the workspace stores are complete
   tc_fence_before();
   CSYNC();
   if (warp == 0) tmem_dealloc(tmem, Cfg::kTmemCols);
@@ -1193,12 +1241,14 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
 template <int DV, bool MID>
 __global__ void __launch_bounds__(ChainCfg<DV>::kThreads, 1) gdn_chain_kernel(PrefillArgs a,
                                                            const __grid_constant__ CUtensorMap mapW,
-                                                           const __grid_constant__ CUtensorMap mapK) {
+                                                           const __grid_constant__ CUtensorMap mapK,
+                                                           const __grid_constant__ CUtensorMap mapS,
+                                                           const __grid_constant__ CUtensorMap mapU) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   pdl_trigger();
-  chain_body<DV, MID>(a, mapW, mapK, blockIdx.x, sm);
+  chain_body<DV, MID>(a, mapW, mapK, mapS, mapU, blockIdx.x, sm);
 }
 
 // --------------------------------------------------------------------------- out, persistent
@@ -1736,7 +1786,8 @@ static bool make_map_x(CUtensorMap* m, const void* base, int T, int Cc) {
 
 template <int DV, bool MID>
 static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW,
-                                const CUtensorMap& mK, cudaStream_t s, bool pdl) {
+                                const CUtensorMap& mK, const CUtensorMap& mS,
+                                const CUtensorMap& mU, cudaStream_t s, bool pdl) {
   using Cfg = gdn::ChainCfg<DV, MID>;
   static bool attr = false;
   if (!attr) {
@@ -1747,7 +1798,7 @@ static cudaError_t launch_chain(const gdn::PrefillArgs& a, const CUtensorMap& mW
   }
   trace_begin("gdn_chain", s);
   cudaError_t e = launch_k(pdl, gdn::gdn_chain_kernel<DV, MID>, dim3(a.N * a.Hv * a.nsplit),
-                           dim3(Cfg::kThreads), Cfg::kSmem, s, a, mW, mK);
+                           dim3(Cfg::kThreads), Cfg::kSmem, s, a, mW, mK, mS, mU);
   trace_end(s);
   return e;
 }
@@ -1884,15 +1935,15 @@ cudaError_t launch_prefill_tc(gdn::PrefillArgs a, void* workspace, cudaStream_t 
   auto launch_chain_any = [&](gdn::PrefillArgs sa, cudaStream_t st, bool pdl) -> cudaError_t {
     if (sa.page64) {
       switch (sa.nsplit) {
-        case 4: return launch_chain<32, true>(sa, mW, mK, st, pdl);
-        case 2: return launch_chain<64, true>(sa, mW, mK, st, pdl);
-        default: sa.nsplit = 1; return launch_chain<128, true>(sa, mW, mK, st, pdl);
+        case 4: return launch_chain<32, true>(sa, mW, mK, mS, mU, st, pdl);
+        case 2: return launch_chain<64, true>(sa, mW, mK, mS, mU, st, pdl);
+        default: sa.nsplit = 1; return launch_chain<128, true>(sa, mW, mK, mS, mU, st, pdl);
       }
     }
     switch (sa.nsplit) {
-      case 4: return launch_chain<32, false>(sa, mW, mK, st, pdl);
-      case 2: return launch_chain<64, false>(sa, mW, mK, st, pdl);
-      default: sa.nsplit = 1; return launch_chain<128, false>(sa, mW, mK, st, pdl);
+      case 4: return launch_chain<32, false>(sa, mW, mK, mS, mU, st, pdl);
+      case 2: return launch_chain<64, false>(sa, mW, mK, mS, mU, st, pdl);
+      default: sa.nsplit = 1; return launch_chain<128, false>(sa, mW, mK, mS, mU, st, pdl);
     }
   };
   auto launch_out = [&](const gdn::PrefillArgs& sa, cudaStream_t st, bool pdl) -> cudaError_t {
