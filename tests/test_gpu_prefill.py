@@ -127,26 +127,28 @@ def test_bf16_pipelined_matches_single_launch_bitwise():
 
 
 @pytest.mark.parametrize("segmented", [False, True])
-def test_chain_wait_runs_out_and_the_context_stays_usable(segmented):
+@pytest.mark.parametrize("split", [0, 2, 1])
+def test_chain_wait_runs_out_and_the_context_stays_usable(segmented, split):
     # A load the chain waits for is left out on purpose (debug fault injection): the chain's
     # bounded wait must run out within its limit (5 ms here), write GDN_ERR_TIMEOUT, let its
-    # other copies land, free its TMEM and end; afterwards the same stream runs a normal
-    # prefill that matches the one before the fault bit for bit.
+    # other copies land (TMA loads, and with d_v blocks of 64 or 128 the TMA stores of S and U),
+    # free its TMEM and end; afterwards the same stream runs a normal prefill that matches the
+    # one before the fault bit for bit.
     w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(700, 300), s0_std=0.1)
     inp = inputs.prefill_inputs(w, 1350, with_conv0=True)
     seg = 2 if segmented else 0
-    with gdn.debug_options(segment_chunks=seg):
+    with gdn.debug_options(segment_chunks=seg, chain_split=split):
         good = gpu_prefill(w, inp)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     import time
     t0 = time.perf_counter()
-    with gdn.debug_options(wait_limit_us=5000, segment_chunks=seg,
+    with gdn.debug_options(wait_limit_us=5000, segment_chunks=seg, chain_split=split,
                            fault=gdn.GDN_FAULT_SKIP_CHAIN_LOAD, fault_chunk=2):
         gpu_prefill(w, inp, dev_status=status)
     elapsed = time.perf_counter() - t0
     assert int(status.item()) == gdn.GDN_ERR_TIMEOUT
     assert elapsed < 1.0, elapsed     # gave up after its 5 ms limit, not the 2 s default
-    with gdn.debug_options(segment_chunks=seg):
+    with gdn.debug_options(segment_chunks=seg, chain_split=split):
         again = gpu_prefill(w, inp)
     for a, b, name in zip(good, again, ("out", "final state", "conv state")):
         assert torch.equal(a, b), name
