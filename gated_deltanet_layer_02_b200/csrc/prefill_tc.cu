@@ -985,13 +985,8 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
         st_row8_bf16(OP, kTile, k_row, (cs + gi * 32 + 8 * q) >> 3, sreg[gi] + 8 * q);
       if constexpr (!kOverlap) {
         if constexpr (!kTmaOut) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float w8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
-            store8(Srow + gi * 32 + 8 * q, w8);
-          }
+          store16(Srow + gi * 32, sreg[gi]);
+          store16(Srow + gi * 32 + 16, sreg[gi] + 16);
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e) sreg[gi][e] *= gam;
@@ -1029,13 +1024,8 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
 #pragma unroll
       for (int gi = 0; gi < kGroups; ++gi) {
         if constexpr (!kTmaOut) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float w8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = sreg[gi][8 * q + e];
-            store8(Srow + gi * 32 + 8 * q, w8);
-          }
+          store16(Srow + gi * 32, sreg[gi]);
+          store16(Srow + gi * 32 + 16, sreg[gi] + 16);
         }
 #pragma unroll
         for (int e = 0; e < 32; ++e) sreg[gi][e] *= gam;
@@ -1156,12 +1146,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     // while the state update runs: U to the workspace
     if constexpr (kOverlap && !kTmaOut) {
 #pragma unroll
-      for (int q = 0; q < kCPT / 8; ++q) {
-        float u8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) u8[e] = ureg[q * 8 + e];
-        store8(Urow + q * 8, u8);
-      }
+      for (int q = 0; q < kCPT / 16; ++q) store16(Urow + q * 16, ureg + q * 16);
     }
     if ((failed = CSYNC_OR(!ok))) break;
     ok = mbar_wait(bar_mma, mma_phase, a.wait_ns);
