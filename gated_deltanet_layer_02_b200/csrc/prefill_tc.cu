@@ -1538,6 +1538,7 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
     // ----------------------------------------------- group B: gated RMSNorm epilogue, row
     const int i_row = tid - 128;
     const uint32_t lane_addr = tmem_at(tmem, (warp & 3) * 32, 0);
+    const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     uint4 zreg[16];
     // chunk entries two units ahead, z rows one unit ahead (two dependent loads otherwise)
     auto entry = [&](int i) {
@@ -1609,12 +1610,17 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
           }
         }
         if (valid) {
+          if (out32) {  // 32-byte stores (whole sectors) when the output allows them
+            store16(dst + q * 32, v);
+            store16(dst + q * 32 + 16, v + 16);
+          } else {
 #pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            float o8[8];
+            for (int r = 0; r < 4; ++r) {
+              float o8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) o8[e] = v[r * 8 + e];
-            store8(dst + q * 32 + r * 8, o8);
+              for (int e = 0; e < 8; ++e) o8[e] = v[r * 8 + e];
+              store8(dst + q * 32 + r * 8, o8);
+            }
           }
         }
       }

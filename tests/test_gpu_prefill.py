@@ -262,3 +262,18 @@ def test_bf16_page128_states_equal_chunk_states():
     assert torch.equal(cs, ps)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_bf16_output_at_a_16_byte_offset():
+    # The output kernel writes whole 32-byte sectors when the output allows it and 16-byte
+    # pieces otherwise (the ABI asks for 16-byte alignment only): both give the same bits.
+    w = inputs.custom(2, 4, 128, torch.bfloat16, lengths=(300, 130), s0_std=0.1)
+    inp = inputs.prefill_inputs(w, 1400)
+    T, Hv, d = w.tokens, w.num_v_heads, w.head_dim
+    base = torch.empty(T * Hv * d + 8, dtype=torch.bfloat16, device="cuda")
+    aligned = base[:T * Hv * d].view(T, Hv, d)
+    shifted = base[8:].view(T, Hv, d)    # 16 bytes past a 256-byte aligned allocation
+    assert shifted.data_ptr() % 32 == 16
+    a = gpu_prefill(w, inp, out=aligned)[0].clone()
+    b = gpu_prefill(w, inp, out=shifted)[0]
+    assert torch.equal(a, b)
