@@ -46,6 +46,21 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
   for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
   *reinterpret_cast<uint4*>(p) = u;
 }
+// 32 bytes in one read-only load (a whole L2 sector per lane; p 32-byte aligned).
+__device__ __forceinline__ void load32_nc(const void* p, uint4& lo, uint4& hi) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y),
+                 "=r"(hi.z), "=r"(hi.w)
+               : "l"(p));
+}
+// 32 bytes in one load (p 32-byte aligned).
+__device__ __forceinline__ void load32(const void* p, uint4& lo, uint4& hi) {
+  asm volatile("ld.global.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y),
+                 "=r"(hi.z), "=r"(hi.w)
+               : "l"(p)
+               : "memory");
+}
 // 16 values as bf16 (round to nearest even) in one 32-byte store: a whole L2 sector per lane
 // (p 32-byte aligned).
 __device__ __forceinline__ void store16(__nv_bfloat16* p, const float* v) {

@@ -950,7 +950,7 @@ __device__ __forceinline__ void chain_body(const PrefillArgs& a, const CUtensorM
     const uint4* src = reinterpret_cast<const uint4*>(
         a.ws.Uw + (((size_t)c * a.Hv + h) * kC + k_row) * kD + v0 + cs);
 #pragma unroll
-    for (int q = 0; q < kVec; ++q) ut[q] = src[q];
+    for (int q = 0; q < kVec; q += 2) load32(src + q, ut[q], ut[q + 1]);  // 32-byte aligned
   };
   if (nch > 0) load_chunk_rows(0, ut_cur, Gi_cur, Gl_cur, Gm_cur, L_cur);
   for (int ci = 0; ci < nch; ++ci) {
@@ -1539,6 +1539,7 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
     const int i_row = tid - 128;
     const uint32_t lane_addr = tmem_at(tmem, (warp & 3) * 32, 0);
     const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
+    const bool z32 = (reinterpret_cast<uintptr_t>(a.z) & 31u) == 0;
     uint4 zreg[16];
     // chunk entries two units ahead, z rows one unit ahead (two dependent loads otherwise)
     auto entry = [&](int i) {
@@ -1552,8 +1553,13 @@ __global__ void __launch_bounds__(kOutPThreads, 1) gdn_out_persistent_kernel(
       if (a.z && i_row < ci_next.L) {
         const uint4* zp =
             reinterpret_cast<const uint4*>(a.z + ((size_t)(ci_next.t0 + i_row) * Hv + h) * kD);
+        if (z32) {  // whole sectors when z allows it
 #pragma unroll
-        for (int q = 0; q < 16; ++q) zreg[q] = __ldg(zp + q);
+          for (int q = 0; q < 16; q += 2) load32_nc(zp + q, zreg[q], zreg[q + 1]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) zreg[q] = __ldg(zp + q);
+        }
       }
     };
     if (count > 0) prefetch(0);
