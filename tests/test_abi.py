@@ -349,3 +349,23 @@ def test_debug_options_are_checked(L):
         seg = L.gdn_chunk_prefill_workspace_size(d, 1, 1, 4096)
     assert seg > plain
     assert L.gdn_chunk_prefill_workspace_size(d, 1, 1, 4096) == plain
+
+
+def test_default_pipeline_segments(L):
+    # Calls are cut into segments from 512 chunks on (64 chunks each, 128 from 1024 chunks),
+    # one fp32 carry state [Hv, d, d] per segment boundary in the workspace: the workspace size
+    # shows the number of segments the library chose.
+    d = ctypes.byref(gdn.Dims())
+    carry = 32 * 128 * 128 * 4
+
+    def carries(T):
+        size = L.gdn_chunk_prefill_workspace_size(d, 1, 1, T)
+        with gdn.debug_options(segment_chunks=1 << 19):   # one launch of each kernel
+            single = L.gdn_chunk_prefill_workspace_size(d, 1, 1, T)
+        assert (size - single) % carry == 0
+        return (size - single) // carry
+
+    assert carries(510 * 128) == 0       # 511 chunks: one launch
+    assert carries(511 * 128) == 7       # 512 chunks: 8 segments of 64
+    assert carries(1023 * 128) == 7      # 1024 chunks: 8 segments of 128
+    assert carries(262144) == 16         # 2049 chunks: 17 segments of 121
